@@ -1,0 +1,315 @@
+"""fp64 oracle: exact attention written out from its definition (test infrastructure).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline legs of
+``bench.py`` use this module. Page keys ([card], [interview], [essay],
+[explainer]) are defined in ``oracle/__init__.py``.
+
+Every function takes float64 arrays and materialises what the definition names.
+Matrix products go through numpy (a library primitive); no blocking, fusion or
+reordering is applied beyond what a definition states, except that rows of S are
+independent by definition, so the long-sequence mode computes them a group of
+rows at a time.
+
+Readings of points the pages leave open:
+  * scale: S = scale·QKᵀ with the scale passed in (1/√d in every workload);
+    [essay] section 二 writes softmax(QKᵀ/√d), [interview] 二.1 omits the scale.
+  * the statistic saved for the backward is lse = m + ln ℓ (natural log, in the
+    units of the scaled scores); [essay] 二 and [interview] 三.3 save (m, ℓ),
+    which carries the same information.
+  * softmax gradient: dS = P∘(dP − rowsum(P∘dP)) with dP = dO·Vᵀ (textbook
+    softmax Jacobian); the formula printed in [explainer] "梯度计算优化" is not
+    dimensionally consistent and is not used.
+  * causal: top-left aligned, query i sees keys j ≤ i ([essay] 三.1), N_q = N_k.
+  * block mask: one uint8 entry per 128×128 tile of S, shared by every batch
+    and head, composed with the causal mask by AND ([card] Block-Sparse).
+  * a row with no allowed key: O = 0, lse = −inf, zero gradient (pages silent).
+"""
+from __future__ import annotations
+
+import os
+from concurrent.futures import ThreadPoolExecutor
+
+import numpy as np
+
+TILE = 128  # one block-mask entry covers a TILE x TILE tile of S
+
+
+# --------------------------------------------------------------------------- masks
+
+def allowed_mask(nq: int, nk: int, causal: bool = False, block_mask=None, tile: int = TILE) -> np.ndarray:
+    """Boolean [nq, nk]: True where query i may attend to key j.
+
+    Causal ([essay] 三.1): P_ij = 0 for j > i. Block mask ([card] Block-Sparse):
+    entry (I, J) = 0 removes every pair (i, j) with i // tile == I and
+    j // tile == J. The two compose by AND.
+    """
+    a = np.ones((nq, nk), dtype=bool)
+    if causal:
+        a &= np.arange(nk)[None, :] <= np.arange(nq)[:, None]
+    if block_mask is not None:
+        bm = np.asarray(block_mask).astype(bool)
+        a &= bm[np.arange(nq)[:, None] // tile, np.arange(nk)[None, :] // tile]
+    return a
+
+
+# --------------------------------------------------------------------------- forward
+
+def _softmax_rows(S: np.ndarray):
+    """Safe softmax of each row ([explainer] 工作原理; [interview] 三.2).
+
+    Subtract the row maximum, exponentiate, divide by the row sum. Returns P and
+    lse = max + ln(sum). A row of only −inf gives P = 0 and lse = −inf.
+    """
+    m = S.max(axis=-1, keepdims=True)
+    m_safe = np.where(np.isfinite(m), m, 0.0)
+    E = np.exp(S - m_safe)
+    l = E.sum(axis=-1, keepdims=True)
+    P = np.divide(E, l, out=np.zeros_like(E), where=l > 0)
+    l1 = l[..., 0]
+    lse = np.full(l1.shape, -np.inf)
+    pos = l1 > 0
+    lse[pos] = m_safe[..., 0][pos] + np.log(l1[pos])
+    return P, lse
+
+
+def _head_forward(q, k, v, scale, allowed):
+    S = scale * (q @ k.T)                       # S = scale·QKᵀ   ([interview] 二.1, [essay] 二)
+    S = np.where(allowed, S, -np.inf)           # masked scores
+    P, lse = _softmax_rows(S)                   # P = softmax(S)
+    O = P @ v                                   # O = PV
+    return O, lse, P
+
+
+def forward(q, k, v, scale: float, causal: bool = False, block_mask=None, tile: int = TILE,
+            return_p: bool = False):
+    """Exact attention forward for q, k, v of shape [..., N, d] (float64).
+
+    Returns (O [..., N, d], lse [..., N]) and, if ``return_p``, P [..., N, N].
+    Leading dimensions (batch, heads) are independent problems.
+    """
+    q, k, v = (np.asarray(t, dtype=np.float64) for t in (q, k, v))
+    lead = q.shape[:-2]
+    n, d = q.shape[-2:]
+    allowed = allowed_mask(n, k.shape[-2], causal, block_mask, tile)
+    O = np.empty(lead + (n, v.shape[-1]))
+    lse = np.empty(lead + (n,))
+    Ps = np.empty(lead + (n, k.shape[-2])) if return_p else None
+    for idx in np.ndindex(*lead):
+        o, s, P = _head_forward(q[idx], k[idx], v[idx], scale, allowed)
+        O[idx], lse[idx] = o, s
+        if return_p:
+            Ps[idx] = P
+    return (O, lse, Ps) if return_p else (O, lse)
+
+
+# --------------------------------------------------------------------------- backward
+
+def _head_backward(q, k, v, do, scale, allowed):
+    _, _, P = _head_forward(q, k, v, scale, allowed)   # P recomputed from the definition
+    dV = P.T @ do                                      # dV = Pᵀ dO
+    dP = do @ v.T                                      # dP = dO Vᵀ
+    D = (P * dP).sum(axis=1, keepdims=True)            # D_i = Σ_j P_ij dP_ij
+    dS = P * (dP - D)                                  # softmax Jacobian
+    dQ = scale * (dS @ k)                              # S = scale·QKᵀ
+    dK = scale * (dS.T @ q)
+    return dQ, dK, dV, D[:, 0]
+
+
+def backward(q, k, v, do, scale: float, causal: bool = False, block_mask=None, tile: int = TILE,
+             return_d: bool = False):
+    """Gradients of a loss L with ∂L/∂O = dO, by the chain rule through the definition.
+
+    dV = Pᵀ dO, dP = dO Vᵀ, dS = P∘(dP − rowsum(P∘dP)), dQ = scale·dS K,
+    dK = scale·dSᵀ Q. P is recomputed here from Q and K ([card] 反向：重算而非存储).
+    Returns (dQ, dK, dV) and, if ``return_d``, D = rowsum(P∘dP) [..., N].
+    """
+    q, k, v, do = (np.asarray(t, dtype=np.float64) for t in (q, k, v, do))
+    lead = q.shape[:-2]
+    n = q.shape[-2]
+    allowed = allowed_mask(n, k.shape[-2], causal, block_mask, tile)
+    dQ, dK, dV = np.empty_like(q), np.empty_like(k), np.empty_like(v)
+    D = np.empty(lead + (n,))
+    for idx in np.ndindex(*lead):
+        dQ[idx], dK[idx], dV[idx], D[idx] = _head_backward(q[idx], k[idx], v[idx], do[idx], scale, allowed)
+    return (dQ, dK, dV, D) if return_d else (dQ, dK, dV)
+
+
+# --------------------------------------------------------------------------- online recurrence
+
+def online_forward(q, k, v, scale: float, bounds, causal: bool = False, block_mask=None,
+                   tile: int = TILE):
+    """Forward by the online-softmax recurrence of [interview] 三.2, for one head [N, d].
+
+    Keys are split into consecutive blocks at ``bounds`` (0 = b_0 < … < b_T = N).
+    Each block gives local statistics m̃ = rowmax(S_blk), ℓ̃ = rowsum(exp(S_blk − m̃))
+    and an unnormalised local output Õ = exp(S_blk − m̃)·V_blk. They are merged
+    into the running (m, ℓ, O):
+        m' = max(m, m̃),  ℓ' = e^{m−m'}·ℓ + e^{m̃−m'}·ℓ̃,  O' = e^{m−m'}·O + e^{m̃−m'}·Õ,
+    and O/ℓ is returned at the end with lse = m + ln ℓ. A factor e^{x−m'} whose
+    exponent is −inf − (−inf) (no allowed key seen yet on either side) is taken as 0.
+    This routine exists to check the two-pass oracle; it is not used for parity.
+    """
+    q, k, v = (np.asarray(t, dtype=np.float64) for t in (q, k, v))
+    n = q.shape[0]
+    allowed = allowed_mask(n, k.shape[0], causal, block_mask, tile)
+    m = np.full(n, -np.inf)
+    l = np.zeros(n)
+    O = np.zeros((n, v.shape[1]))
+
+    def factor(a, b):
+        out = np.zeros_like(a)
+        ok = np.isfinite(a)
+        out[ok] = np.exp(a[ok] - b[ok])
+        return out
+
+    bounds = list(bounds)
+    for lo, hi in zip(bounds[:-1], bounds[1:]):
+        S = scale * (q @ k[lo:hi].T)
+        S = np.where(allowed[:, lo:hi], S, -np.inf)
+        m_t = S.max(axis=1)
+        m_t_safe = np.where(np.isfinite(m_t), m_t, 0.0)
+        E = np.exp(S - m_t_safe[:, None])
+        l_t = E.sum(axis=1)
+        O_t = E @ v[lo:hi]
+        m_new = np.maximum(m, m_t)
+        a_old = factor(m, m_new)
+        a_new = factor(m_t, m_new)
+        l = a_old * l + a_new * l_t
+        O = a_old[:, None] * O + a_new[:, None] * O_t
+        m = m_new
+    lse = np.full(n, -np.inf)
+    pos = l > 0
+    O = np.divide(O, l[:, None], out=np.zeros_like(O), where=pos[:, None])
+    lse[pos] = m[pos] + np.log(l[pos])
+    return O, lse
+
+
+# --------------------------------------------------------------------------- tile enumeration
+
+def causal_tile_set(n: int, br: int, bc: int):
+    """The valid-tile set of [essay] 三.1: {(i, j) | j·B_c ≤ i·B_r + B_r − 1}.
+
+    i ranges over the ⌈n/B_r⌉ query tiles and j over the ⌈n/B_c⌉ key tiles.
+    Returned as a sorted list of (i, j) pairs.
+    """
+    tr, tc = -(-n // br), -(-n // bc)
+    return [(i, j) for i in range(tr) for j in range(tc) if j * bc <= i * br + br - 1]
+
+
+def _visited(n, causal, block_mask, br, bc, mask_tile=TILE):
+    """Set of (i, j) tile pairs the method processes: the causal valid-tile set
+    (or all pairs) intersected with the non-zero entries of the block mask.
+    A query tile of B_r rows inside mask row I = i·B_r // mask_tile (B_r divides mask_tile)."""
+    tr, tc = -(-n // br), -(-n // bc)
+    pairs = set(causal_tile_set(n, br, bc)) if causal else {(i, j) for i in range(tr) for j in range(tc)}
+    if block_mask is not None:
+        bm = np.asarray(block_mask)
+        pairs = {(i, j) for (i, j) in pairs
+                 if bm[(i * br) // mask_tile, (j * bc) // mask_tile]}
+    return pairs
+
+
+def forward_tile_lists(n: int, causal: bool, block_mask=None, br: int = 128, bc: int = 128):
+    """For each query tile i, the sorted key tiles j it streams ([essay] 三.1; [card] Block-Sparse:
+    zero tiles skipped)."""
+    tr = -(-n // br)
+    pairs = _visited(n, causal, block_mask, br, bc)
+    return [sorted(j for (ii, j) in pairs if ii == i) for i in range(tr)]
+
+
+def backward_tile_lists(n: int, causal: bool, block_mask=None, br: int = 128, bc: int = 128):
+    """For each key tile j, the sorted query tiles i that reach it (the transpose of the forward lists)."""
+    tc = -(-n // bc)
+    pairs = _visited(n, causal, block_mask, br, bc)
+    return [sorted(i for (i, jj) in pairs if jj == j) for j in range(tc)]
+
+
+# --------------------------------------------------------------------------- long sequences
+
+def _head_sampled(q, k, v, do, scale, causal, block_mask, tile, rows_q, rows_k, chunk):
+    n = q.shape[0]
+    O = np.empty_like(q)
+    lse = np.empty(n)
+    # Pass 1: O and lse of every row, a group of rows at a time (rows are independent).
+    for r0 in range(0, n, chunk):
+        r1 = min(n, r0 + chunk)
+        kend = r1 if causal else n          # keys beyond r1 are masked for every row of the group
+        allowed = _allowed_pairs(np.arange(r0, r1), np.arange(kend), causal, block_mask, tile)
+        S = scale * (q[r0:r1] @ k[:kend].T)
+        S = np.where(allowed, S, -np.inf)
+        P, lse[r0:r1] = _softmax_rows(S)
+        O[r0:r1] = P @ v[:kend]
+    D = (do * O).sum(axis=1)                # D_i = rowsum(dO∘O)
+    out = {"o": O[rows_q], "lse": lse[rows_q]}
+    # dQ at the sampled query rows: dQ_i = scale·Σ_j dS_ij k_j.
+    Sq = scale * (q[rows_q] @ k.T)
+    aq = _allowed_pairs(rows_q, np.arange(n), causal, block_mask, tile)
+    Pq = np.where(aq, np.exp(np.where(aq, Sq, 0.0) - lse[rows_q][:, None]), 0.0)
+    dPq = do[rows_q] @ v.T
+    dSq = Pq * (dPq - D[rows_q][:, None])
+    out["dq"] = scale * (dSq @ k)
+    # dK, dV at the sampled key rows: dK_j = scale·Σ_i dS_ij q_i, dV_j = Σ_i P_ij dO_i.
+    Sk = scale * (q @ k[rows_k].T)
+    ak = _allowed_pairs(np.arange(n), rows_k, causal, block_mask, tile)
+    Pk = np.where(ak, np.exp(np.where(ak, Sk, 0.0) - lse[:, None]), 0.0)
+    dPk = do @ v[rows_k].T
+    dSk = Pk * (dPk - D[:, None])
+    out["dk"] = scale * (dSk.T @ q)
+    out["dv"] = Pk.T @ do
+    return out
+
+
+def _allowed_pairs(rows, cols, causal, block_mask, tile):
+    a = np.ones((rows.size, cols.size), dtype=bool)
+    if causal:
+        a &= cols[None, :] <= rows[:, None]
+    if block_mask is not None:
+        bm = np.asarray(block_mask).astype(bool)
+        a &= bm[rows[:, None] // tile, cols[None, :] // tile]
+    return a
+
+
+def sampled_forward_backward(q, k, v, do, scale: float, causal: bool, rows_q, rows_k,
+                             block_mask=None, tile: int = TILE, chunk: int = 1024,
+                             workers: int | None = None):
+    """Long-sequence mode for inputs [..., N, d]: full-N×N matrices never exist.
+
+    Pass 1 computes O and lse for every row of every head, a group of ``chunk``
+    rows at a time, and D = rowsum(dO∘O). Then the same formulas as
+    :func:`backward`, restricted to the rows ``rows_q`` (O, lse, dQ) and the key
+    rows ``rows_k`` (dK, dV). Heads run in a thread pool (numpy releases the GIL
+    in its kernels); the arithmetic of each head is unchanged by that.
+    Returns a dict of arrays with leading dims [..., len(rows)].
+    """
+    q, k, v, do = (np.asarray(t, dtype=np.float64) for t in (q, k, v, do))
+    rows_q, rows_k = np.asarray(rows_q), np.asarray(rows_k)
+    lead = q.shape[:-2]
+    heads = list(np.ndindex(*lead))
+    if workers is None:
+        workers = max(1, min(len(heads), os.cpu_count() or 1))
+
+    def run(idx):
+        return idx, _head_sampled(q[idx], k[idx], v[idx], do[idx], scale, causal, block_mask, tile,
+                                  rows_q, rows_k, chunk)
+
+    results = {}
+    try:
+        from threadpoolctl import threadpool_limits
+        limiter = threadpool_limits(1) if workers > 1 else None
+    except ImportError:  # pragma: no cover
+        limiter = None
+    try:
+        with ThreadPoolExecutor(max_workers=workers) as ex:
+            for idx, res in ex.map(run, heads):
+                results[idx] = res
+    finally:
+        if limiter is not None:
+            limiter.restore_original_limits()
+    out = {}
+    for key in ("o", "lse", "dq", "dk", "dv"):
+        first = results[heads[0]][key]
+        arr = np.empty(lead + first.shape)
+        for idx in heads:
+            arr[idx] = results[idx][key]
+        out[key] = arr
+    return out

@@ -1,0 +1,260 @@
+"""Checks that pin the fp64 oracle to facts fixed by the pages and by mathematics.
+
+Each ``check_*`` takes the oracle functions it exercises and raises
+AssertionError on a mismatch, so the same checks run against the real oracle
+(``test_oracle_pins.py``) and against copies of it with planted mistakes
+(``test_oracle_mutants.py``), where at least one check must fail.
+
+What pins what:
+  * closed forms worked out by hand (tests/golden/closed_forms.json);
+  * rows of P sum to 1; equal keys give the mean of the values; one key gives
+    that key's value; causal row 0 returns V_0; a constant value column passes
+    through; shifting every key by one vector leaves O unchanged;
+  * the two-pass softmax equals the online-softmax recurrence of the
+    interview explainer (section 三.2) for any split of the keys;
+  * central finite differences of L = <dO, O> confirm dQ, dK, dV;
+  * gradient identities: D = rowsum(dO∘O) = rowsum(P∘dP), Σ_j dK_j = 0,
+    Σ_j dV_j = Σ_i dO_i;
+  * block-sparse with an all-ones mask equals dense, and a block-diagonal mask
+    equals independent attention on each block;
+  * pure-Python loops on tiny inputs (a second, loop-level reading of the
+    definition).
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import numpy as np
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "closed_forms.json")
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def _close(a, b, tol, what):
+    a, b = np.asarray(a, dtype=np.float64), np.asarray(b, dtype=np.float64)
+    assert a.shape == b.shape, f"{what}: shape {a.shape} vs {b.shape}"
+    both_inf = np.isinf(a) & np.isinf(b) & (np.sign(a) == np.sign(b))
+    err = np.where(both_inf, 0.0, np.abs(a - b))
+    m = float(np.max(err)) if err.size else 0.0
+    assert m <= tol, f"{what}: max abs err {m:.3e} > {tol:.1e}"
+
+
+# ----------------------------------------------------------------------------- closed forms
+
+def check_closed_forms(forward, backward):
+    with open(GOLDEN) as f:
+        cases = json.load(f)["cases"]
+    for c in cases:
+        q, k, v, do = (np.array(c[n], dtype=np.float64) for n in ("q", "k", "v", "do"))
+        O, lse = forward(q, k, v, c["scale"], causal=c["causal"])
+        _close(O, c["o"], 1e-12, c["name"] + " O")
+        _close(lse, c["lse"], 1e-12, c["name"] + " lse")
+        if q.shape[0] == k.shape[0]:
+            dq, dk, dv = backward(q, k, v, do, c["scale"], causal=c["causal"])
+            _close(dq, c["dq"], 1e-12, c["name"] + " dQ")
+            _close(dk, c["dk"], 1e-12, c["name"] + " dK")
+            _close(dv, c["dv"], 1e-12, c["name"] + " dV")
+
+
+# ----------------------------------------------------------------------------- invariants
+
+def check_rows_sum_to_one(forward):
+    r = _rng(1)
+    for causal, mask in ((False, None), (True, None), (False, np.array([[1, 0], [1, 1]]))):
+        q, k, v = (r.standard_normal((2, 8, 3)) for _ in range(3))
+        _, _, P = forward(q, k, v, 0.5, causal=causal, block_mask=mask, tile=4, return_p=True)
+        _close(P.sum(-1), np.ones((2, 8)), 1e-12, "rows of P sum to 1")
+        assert np.all(P >= 0), "P has a negative entry"
+
+
+def check_equal_keys(forward):
+    r = _rng(2)
+    n, d, scale = 7, 5, 0.37
+    q = r.standard_normal((n, d))
+    krow = r.standard_normal(d)
+    k = np.tile(krow, (n, 1))
+    v = r.standard_normal((n, d))
+    O, lse = forward(q, k, v, scale)
+    _close(O, np.tile(v.mean(0), (n, 1)), 1e-12, "equal keys: O = mean of V")
+    _close(lse, scale * q @ krow + math.log(n), 1e-12, "equal keys: lse")
+    O, lse = forward(q, k, v, scale, causal=True)
+    exp_o = np.stack([v[: i + 1].mean(0) for i in range(n)])
+    _close(O, exp_o, 1e-12, "equal keys causal: O = running mean of V")
+    _close(lse, scale * q @ krow + np.log(np.arange(1, n + 1)), 1e-12, "equal keys causal: lse")
+
+
+def check_single_key(forward):
+    r = _rng(3)
+    q, k, v = (r.standard_normal((1, 4)) for _ in range(3))
+    O, lse = forward(q, k, v, 0.8)
+    _close(O, v, 1e-15, "N=1: O = V")
+    _close(lse, 0.8 * q @ k.T[:, 0], 1e-15, "N=1: lse = scale q.k")
+
+
+def check_causal_first_row(forward):
+    r = _rng(4)
+    q, k, v = (r.standard_normal((6, 3)) for _ in range(3))
+    O, lse = forward(q, k, v, 1.3, causal=True)
+    _close(O[0], v[0], 1e-15, "causal row 0: O_0 = V_0")
+    _close(lse[0], 1.3 * q[0] @ k[0], 1e-14, "causal row 0: lse_0 = S_00")
+
+
+def check_constant_value_column(forward):
+    r = _rng(5)
+    q, k, v = (r.standard_normal((9, 4)) for _ in range(3))
+    v[:, 2] = -1.75
+    for causal in (False, True):
+        O, _ = forward(q, k, v, 0.5, causal=causal)
+        _close(O[:, 2], np.full(9, -1.75), 1e-14, "constant V column passes through")
+
+
+def check_key_shift(forward):
+    r = _rng(6)
+    q, k, v = (r.standard_normal((8, 3)) for _ in range(3))
+    u = r.standard_normal(3)
+    for causal in (False, True):
+        O1, lse1 = forward(q, k, v, 0.7, causal=causal)
+        O2, lse2 = forward(q, k + u, v, 0.7, causal=causal)
+        _close(O1, O2, 1e-12, "key shift leaves O unchanged")
+        _close(lse2 - lse1, 0.7 * q @ u, 1e-12, "key shift moves lse by scale q.u")
+
+
+def check_online_equals_two_pass(forward, online_forward):
+    r = _rng(7)
+    n, d = 13, 4
+    q, k, v = (r.standard_normal((n, d)) for _ in range(3))
+    q *= 3.0  # spread the scores so the running maximum moves
+    mask = np.array([[1, 0, 1, 0], [0, 1, 1, 0], [1, 1, 1, 0], [0, 0, 1, 1]])
+    splits = [list(range(n + 1)), [0, n], [0, 5, n], [0, 1, 2, 7, 12, n]]
+    for _ in range(4):
+        cuts = sorted(r.choice(np.arange(1, n), size=r.integers(1, 6), replace=False).tolist())
+        splits.append([0] + cuts + [n])
+    for causal in (False, True):
+        for bm in (None, mask):
+            O, lse = forward(q, k, v, 0.6, causal=causal, block_mask=bm, tile=4)
+            for b in splits:
+                O2, lse2 = online_forward(q, k, v, 0.6, b, causal=causal, block_mask=bm, tile=4)
+                _close(O2, O, 1e-12, f"online recurrence vs two-pass, split {b}")
+                _close(lse2, lse, 1e-12, f"online lse vs two-pass, split {b}")
+
+
+# ----------------------------------------------------------------------------- gradients
+
+def check_finite_differences(forward, backward):
+    r = _rng(8)
+    n, d, h = 6, 3, 1e-5
+    mask = np.array([[1, 0, 1], [1, 1, 0], [0, 1, 1]])
+    for causal, bm in ((False, None), (True, None), (False, mask), (True, mask)):
+        q, k, v, do = (r.standard_normal((n, d)) for _ in range(4))
+        dq, dk, dv = backward(q, k, v, do, 0.45, causal=causal, block_mask=bm, tile=2)
+
+        def L(q_, k_, v_):
+            O, _ = forward(q_, k_, v_, 0.45, causal=causal, block_mask=bm, tile=2)
+            return float(np.sum(do * O))
+
+        for _ in range(3):
+            for which, grad in (("q", dq), ("k", dk), ("v", dv)):
+                R = r.standard_normal((n, d))
+                args_p = {"q_": q, "k_": k, "v_": v}
+                args_m = dict(args_p)
+                args_p[which + "_"] = args_p[which + "_"] + h * R
+                args_m[which + "_"] = args_m[which + "_"] - h * R
+                fd = (L(**args_p) - L(**args_m)) / (2 * h)
+                an = float(np.sum(grad * R))
+                rel = abs(fd - an) / max(1e-12, abs(an), abs(fd))
+                assert rel <= 1e-7, f"finite differences d{which} (causal={causal}, mask={bm is not None}): rel {rel:.2e}"
+
+
+def check_gradient_identities(forward, backward):
+    r = _rng(9)
+    n, d = 10, 4
+    mask = np.array([[1, 0, 0], [1, 1, 0], [0, 1, 1]])
+    for causal, bm in ((False, None), (True, None), (False, mask)):
+        q, k, v, do = (r.standard_normal((n, d)) for _ in range(4))
+        O, _ = forward(q, k, v, 0.5, causal=causal, block_mask=bm, tile=4)
+        dq, dk, dv, D = backward(q, k, v, do, 0.5, causal=causal, block_mask=bm, tile=4, return_d=True)
+        _close(D, (do * O).sum(1), 1e-12, "D = rowsum(dO∘O) = rowsum(P∘dP)")
+        _close(dk.sum(0), np.zeros(d), 1e-12, "Σ_j dK_j = 0")
+        _close(dv.sum(0), do.sum(0), 1e-12, "Σ_j dV_j = Σ_i dO_i")
+
+
+# ----------------------------------------------------------------------------- block-sparse
+
+def check_blocksparse_reductions(forward, backward):
+    r = _rng(10)
+    n, d, t = 12, 3, 4
+    q, k, v, do = (r.standard_normal((n, d)) for _ in range(4))
+    ones = np.ones((3, 3), dtype=np.uint8)
+    for causal in (False, True):
+        a = forward(q, k, v, 0.6, causal=causal)
+        b = forward(q, k, v, 0.6, causal=causal, block_mask=ones, tile=t)
+        _close(a[0], b[0], 0, "all-ones mask = dense (O)")
+        _close(a[1], b[1], 0, "all-ones mask = dense (lse)")
+        ga = backward(q, k, v, do, 0.6, causal=causal)
+        gb = backward(q, k, v, do, 0.6, causal=causal, block_mask=ones, tile=t)
+        for x, y in zip(ga, gb):
+            _close(x, y, 0, "all-ones mask = dense (grads)")
+    # An asymmetric mask fixes its orientation: row I of the mask selects the key
+    # tiles J seen by query tile I, so query tile I equals dense attention over
+    # the keys of those tiles only.
+    asym = np.array([[1, 0, 0], [1, 0, 1], [0, 1, 0]], dtype=np.uint8)
+    O, lse = forward(q, k, v, 0.6, block_mask=asym, tile=t)
+    for I in range(3):
+        rows = slice(I * t, (I + 1) * t)
+        keys = np.concatenate([np.arange(J * t, (J + 1) * t) for J in range(3) if asym[I, J]])
+        Oi, lsei = forward(q[rows], k[keys], v[keys], 0.6)
+        _close(O[rows], Oi, 1e-12, "mask row I selects the key tiles of query tile I (O)")
+        _close(lse[rows], lsei, 1e-12, "mask row I selects the key tiles of query tile I (lse)")
+    diag = np.eye(3, dtype=np.uint8)
+    O, lse = forward(q, k, v, 0.6, block_mask=diag, tile=t)
+    g = backward(q, k, v, do, 0.6, block_mask=diag, tile=t)
+    for c in range(3):
+        s = slice(c * t, (c + 1) * t)
+        Oc, lsec = forward(q[s], k[s], v[s], 0.6)
+        gc = backward(q[s], k[s], v[s], do[s], 0.6)
+        _close(O[s], Oc, 1e-12, "block-diagonal = independent blocks (O)")
+        _close(lse[s], lsec, 1e-12, "block-diagonal = independent blocks (lse)")
+        for x, y in zip(g, gc):
+            _close(x[s], y, 1e-12, "block-diagonal = independent blocks (grads)")
+
+
+# ----------------------------------------------------------------------------- brute force
+
+def brute_forward(q, k, v, scale, causal):
+    """Loop-level reading of the definition, for tiny inputs."""
+    n, d = len(q), len(q[0])
+    dv = len(v[0])
+    O = [[0.0] * dv for _ in range(n)]
+    lse = [0.0] * n
+    for i in range(n):
+        keys = [j for j in range(len(k)) if (not causal or j <= i)]
+        s = {j: scale * sum(q[i][t] * k[j][t] for t in range(d)) for j in keys}
+        mx = max(s.values())
+        e = {j: math.exp(s[j] - mx) for j in keys}
+        z = sum(e.values())
+        for c in range(dv):
+            O[i][c] = sum(e[j] * v[j][c] for j in keys) / z
+        lse[i] = mx + math.log(z)
+    return O, lse
+
+
+def check_bruteforce(forward):
+    r = _rng(11)
+    for n, d, causal in ((1, 1, False), (3, 2, False), (5, 3, True), (6, 4, False), (4, 4, True)):
+        q, k, v = (r.standard_normal((n, d)) for _ in range(3))
+        v2 = r.standard_normal((n, d + 1))
+        Ob, lseb = brute_forward(q.tolist(), k.tolist(), v2.tolist(), 0.9, causal)
+        O, lse = forward(q, k, v2, 0.9, causal=causal)
+        _close(O, Ob, 1e-13, f"brute force O n={n} d={d}")
+        _close(lse, lseb, 1e-13, f"brute force lse n={n} d={d}")
+
+
+ALL_FORWARD_CHECKS = (
+    check_rows_sum_to_one, check_equal_keys, check_single_key, check_causal_first_row,
+    check_constant_value_column, check_key_shift, check_bruteforce,
+)

@@ -1,0 +1,75 @@
+"""Plant plausible mistakes in a copy of the oracle and require that a pin catches each.
+
+The copy is made from the oracle's source text with one substitution, executed
+as a fresh module on the CPU; the real oracle is never modified.
+"""
+import importlib.util
+import os
+import types
+
+import pytest
+
+from tests import oracle_pins as pins
+
+SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "oracle", "attention.py")
+
+MUTANTS = {
+    "scale dropped from S": ("S = scale * (q @ k.T)                       #", "S = (q @ k.T)                       #"),
+    "P transposed in PV": ("O = P @ v ", "O = P.T @ v "),
+    "sign flipped in dS": ("dS = P * (dP - D)", "dS = P * (dP + D)"),
+    "D term dropped from dS": ("dS = P * (dP - D)", "dS = P * dP"),
+    "causal mask off by one": ("<= np.arange(nq)[:, None]", "< np.arange(nq)[:, None]"),
+    "scale dropped from dQ": ("dQ = scale * (dS @ k)", "dQ = (dS @ k)"),
+    "dS not transposed in dK": ("dK = scale * (dS.T @ q)", "dK = scale * (dS @ q.T).T"),
+    "max dropped from lse": ("lse[pos] = m_safe[..., 0][pos] + np.log(l1[pos])", "lse[pos] = np.log(l1[pos])"),
+    "P not transposed in dV": ("dV = P.T @ do", "dV = P @ do"),
+    "dP operands swapped": ("dP = do @ v.T", "dP = v @ do.T"),
+    "block mask transposed": ("a &= bm[np.arange(nq)[:, None] // tile, np.arange(nk)[None, :] // tile]",
+                              "a &= bm.T[np.arange(nq)[:, None] // tile, np.arange(nk)[None, :] // tile]"),
+    "online rescale of l dropped": ("l = a_old * l + a_new * l_t", "l = l + a_new * l_t"),
+    "online rescale of O dropped": ("O = a_old[:, None] * O + a_new[:, None] * O_t", "O = O + a_new[:, None] * O_t"),
+}
+
+
+def _mutant(old, new):
+    with open(SRC) as f:
+        text = f.read()
+    assert text.count(old) >= 1, f"mutation site not found: {old!r}"
+    text = text.replace(old, new)
+    mod = types.ModuleType("oracle_mutant")
+    mod.__file__ = SRC
+    exec(compile(text, SRC + " (mutant)", "exec"), mod.__dict__)
+    return mod
+
+
+def _run_all(mod):
+    failures = []
+    checks = [
+        lambda: pins.check_closed_forms(mod.forward, mod.backward),
+        lambda: pins.check_online_equals_two_pass(mod.forward, mod.online_forward),
+        lambda: pins.check_finite_differences(mod.forward, mod.backward),
+        lambda: pins.check_gradient_identities(mod.forward, mod.backward),
+        lambda: pins.check_blocksparse_reductions(mod.forward, mod.backward),
+    ] + [lambda c=c: c(mod.forward) for c in pins.ALL_FORWARD_CHECKS]
+    for c in checks:
+        try:
+            c()
+        except AssertionError as e:
+            failures.append(str(e))
+        except Exception as e:  # a crash also counts as caught
+            failures.append(repr(e))
+    return failures
+
+
+def test_unmutated_copy_passes():
+    with open(SRC) as f:
+        text = f.read()
+    mod = types.ModuleType("oracle_copy")
+    exec(compile(text, SRC, "exec"), mod.__dict__)
+    assert _run_all(mod) == []
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name):
+    old, new = MUTANTS[name]
+    assert _run_all(_mutant(old, new)), f"no pin caught the planted mistake: {name}"
