@@ -1,0 +1,144 @@
+/*
+ * fa.h — C ABI of the B200 (sm_100a) exact attention library (libfa.so).
+ *
+ * The operation is exact scaled-dot-product attention as FlashAttention
+ * computes it:
+ *   S = scale * Q K^T, P = softmax(S) row by row, O = P V
+ * ("FlashAttention" interview explainer, mstx.cn/posts/485, section 2.1,
+ * standard attention; the 1/sqrt(d) scale as in the nanhubrain.csdn.net
+ * FlashAttention essay, section 2). The forward streams K/V tiles past each
+ * resident Q tile with the online-softmax recurrence (same explainer, section
+ * 3.2) and writes only O and the per-row logsumexp. The backward recomputes P
+ * from Q, K and the saved logsumexp instead of storing it ("FlashAttention"
+ * concept card, lukebest.github.io, "反向：重算而非存储").
+ *
+ * Conventions shared by every entry point
+ *   - Tensors q, k, v, o, dout, dq, dk, dv are contiguous [B, H, N, d] in the
+ *     element type given by `dtype` (fp16 or bf16); lse is contiguous fp32
+ *     [B, H, N]. All are DEVICE pointers, 16-byte aligned.
+ *   - lse_i = ln sum_j exp(scale * q_i . k_j) over the keys row i may see
+ *     (natural log, in the units of the scaled scores).
+ *   - d must be 64 or 128; N >= 1 (any value; ragged last tiles are handled);
+ *     B, H >= 1.
+ *   - causal != 0 masks key j > query i (top-left aligned; the essay's
+ *     section 3.1 causal mask P_ij = 0 for j > i).
+ *   - The caller owns all memory. The library allocates no device memory; the
+ *     backward takes a caller-provided workspace of fa_bwd_workspace_size()
+ *     bytes. Host-side tensor-map descriptors are built per call.
+ *   - Every call is asynchronous on `stream` and never synchronises. Argument
+ *     errors are reported before any launch; a failed launch returns
+ *     FA_ERR_CUDA. Device-side time-outs (a wait that could not complete) are
+ *     recorded in a device status word read by fa_device_status().
+ *   - A row with no allowed key (possible only with a block mask) gets O = 0,
+ *     lse = -inf and contributes zero gradients.
+ */
+#ifndef FA_H_
+#define FA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, non-positive size, bad dtype */
+  FA_ERR_UNSUPPORTED = 2, /* valid but unsupported shape (d not 64/128, size limits) */
+  FA_ERR_CUDA = 3,        /* a CUDA runtime call or kernel launch failed */
+  FA_ERR_TIMEOUT = 4      /* a device-side wait gave up (see fa_device_status) */
+} fa_status;
+
+typedef enum { FA_FP16 = 0, FA_BF16 = 1 } fa_dtype;
+
+/* Human-readable name of a status code (static string). */
+const char* fa_status_string(fa_status s);
+
+/*
+ * Forward. Writes o [B,H,N,d] (dtype) and lse [B,H,N] (fp32).
+ * q, k, v are read only. softmax_scale is usually 1/sqrt(d).
+ */
+fa_status fa_fwd(fa_dtype dtype, const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                 int N, int d, float softmax_scale, int causal, cudaStream_t stream);
+
+/*
+ * Bytes of device workspace fa_bwd / fa_blocksparse_bwd need for these sizes:
+ * an fp32 dQ accumulator [B,H,N,d] plus two fp32 row vectors [B,H,ceil(N/128)*128]
+ * (D = rowsum(dO o O) and a padded copy of lse). Linear in N. Returns 0 for
+ * invalid sizes.
+ */
+size_t fa_bwd_workspace_size(int B, int H, int N, int d);
+
+/*
+ * Backward. Given the forward's inputs, its outputs o and lse, and the
+ * incoming gradient dout = dL/dO, writes dq, dk, dv [B,H,N,d] (dtype):
+ *   D = rowsum(dO o O), P = exp(scale*Q K^T - lse), dV = P^T dO,
+ *   dP = dO V^T, dS = P o (dP - D), dQ = scale*dS K, dK = scale*dS^T Q.
+ * workspace: device buffer of at least fa_bwd_workspace_size() bytes, 256-byte
+ * aligned; its contents on entry do not matter and are overwritten.
+ */
+fa_status fa_bwd(fa_dtype dtype, const void* q, const void* k, const void* v, const void* o, const float* lse,
+                 const void* dout, void* dq, void* dk, void* dv, void* workspace, int B, int H, int N, int d,
+                 float softmax_scale, int causal, cudaStream_t stream);
+
+/*
+ * Block-sparse forward ("FlashAttention" concept card, "Block-Sparse
+ * FlashAttention": a fixed block mask whose zero blocks are skipped).
+ * block_mask: DEVICE pointer to uint8 [N/128][N/128], row-major, shared by all
+ * (b, h); entry (I, J) != 0 lets query tile I (rows 128I..128I+127) attend to
+ * key tile J. Zero tiles are never loaded. Composes with `causal` by AND.
+ * Requires N % 128 == 0 and N/128 <= 2048 (else FA_ERR_UNSUPPORTED).
+ */
+fa_status fa_blocksparse_fwd(fa_dtype dtype, const void* q, const void* k, const void* v, void* o, float* lse,
+                             int B, int H, int N, int d, float softmax_scale, int causal,
+                             const uint8_t* block_mask, cudaStream_t stream);
+
+/* Block-sparse backward; arguments as fa_bwd plus block_mask as in fa_blocksparse_fwd. */
+fa_status fa_blocksparse_bwd(fa_dtype dtype, const void* q, const void* k, const void* v, const void* o,
+                             const float* lse, const void* dout, void* dq, void* dk, void* dv, void* workspace,
+                             int B, int H, int N, int d, float softmax_scale, int causal,
+                             const uint8_t* block_mask, cudaStream_t stream);
+
+/*
+ * Debug: the forward / backward with a record of the tiles each CTA loaded.
+ * trace: DEVICE int32 buffer of fa_*_trace_size() entries. For CTA c the
+ * record starts at c * (stride) where stride = T_kv + 1 for the forward
+ * (T_kv = ceil(N/128) key tiles) and T_q + 1 for the backward (T_q = query
+ * tiles of the backward's row step, fa_bwd_row_tile(d) rows each); entry 0 is
+ * the count and entries 1.. are (tile index) | (flags << 16). Forward CTA c
+ * covers query tiles 2p and 2p+1 (p = c % n_pairs) of head c / n_pairs, flags
+ * bit q = tile is used by query tile 2p+q; backward CTA c covers key tile
+ * c % T_kv of head c / T_kv, flags = 1.
+ */
+size_t fa_fwd_trace_size(int B, int H, int N);
+size_t fa_bwd_trace_size(int B, int H, int N, int d);
+int fa_bwd_row_tile(int d);
+fa_status fa_debug_fwd_trace(fa_dtype dtype, const void* q, const void* k, const void* v, void* o, float* lse,
+                             int B, int H, int N, int d, float softmax_scale, int causal,
+                             const uint8_t* block_mask, int32_t* trace, cudaStream_t stream);
+fa_status fa_debug_bwd_trace(fa_dtype dtype, const void* q, const void* k, const void* v, const void* o,
+                             const float* lse, const void* dout, void* dq, void* dk, void* dv, void* workspace,
+                             int B, int H, int N, int d, float softmax_scale, int causal,
+                             const uint8_t* block_mask, int32_t* trace, cudaStream_t stream);
+
+/*
+ * Device status: synchronises `stream`, returns the status word that kernels
+ * set when a device-side wait timed out (FA_OK if none), and clears it.
+ */
+fa_status fa_device_status(cudaStream_t stream);
+
+/*
+ * Debug: launches one CTA that waits on a barrier nothing will complete, with
+ * a time limit of `timeout_ms`; the wait gives up, records FA_ERR_TIMEOUT in
+ * the status word and the CTA exits normally. Used to test the time-out path.
+ */
+fa_status fa_debug_timeout_probe(int timeout_ms, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_H_ */

@@ -1,0 +1,238 @@
+// C ABI of the attention library: argument checks, the device status word and
+// dispatch to the launchers. Declarations and contracts are in include/fa.h.
+#include "../../include/fa.h"
+
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <mutex>
+
+#include "fa_internal.h"
+#include "sm100.cuh"
+
+namespace {
+
+// Status word written by kernels whose waits time out; one per device, in the
+// library's static device memory, so no allocation is needed.
+__device__ int g_fa_status;
+
+__global__ void timeout_probe_kernel(int* status, uint64_t timeout_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    fa::sm100::mbar_init(fa::sm100::smem_u32(&bar), 1);
+    fa::sm100::fence_barrier_init();
+  }
+  __syncthreads();
+  fa::sm100::WaitCtx ctx{&abort_flag, status, timeout_ns};
+  // Nothing ever arrives on this barrier: the wait runs out and records the time-out.
+  fa::sm100::mbar_wait(fa::sm100::smem_u32(&bar), 0, ctx);
+}
+
+int* status_word() {
+  static std::mutex mu;
+  static int* ptrs[128] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_fa_status) != cudaSuccess) return nullptr;
+    ptrs[dev] = static_cast<int*>(p);
+  }
+  return ptrs[dev];
+}
+
+bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+fa_status check_common(fa_dtype dtype, int B, int H, int N, int d) {
+  if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || N < 1 || d < 1) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  const long long bh = static_cast<long long>(B) * H;
+  const long long tiles = (static_cast<long long>(N) + 127) / 128;
+  // grid.y = pairs of query tiles (<= 65535); key-tile indices fit 16 bits.
+  if (bh > 0x7FFFFFFFLL || (tiles + 1) / 2 > 65535 || tiles > 65535) return FA_ERR_UNSUPPORTED;
+  return FA_OK;
+}
+
+fa_status check_mask(int N, int d, const uint8_t* block_mask) {
+  (void)d;
+  if (block_mask == nullptr) return FA_ERR_INVALID_ARG;
+  if (N % 128 != 0 || N / 128 > 2048) return FA_ERR_UNSUPPORTED;
+  return FA_OK;
+}
+
+fa_status fwd_impl(fa_dtype dtype, const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                   int N, int d, float scale, int causal, const uint8_t* mask, int32_t* trace,
+                   cudaStream_t stream) {
+  fa_status s = check_common(dtype, B, H, N, d);
+  if (s != FA_OK) return s;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return FA_ERR_INVALID_ARG;
+  fa::AttnArgs a{};
+  a.dtype = dtype;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.o = o;
+  a.lse = lse;
+  a.B = B;
+  a.H = H;
+  a.N = N;
+  a.d = d;
+  a.scale = scale;
+  a.causal = causal ? 1 : 0;
+  a.block_mask = mask;
+  a.trace = trace;
+  a.status = status_word();
+  if (!a.status) return FA_ERR_CUDA;
+  return fa::launch_fwd(a, stream) == 0 ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status bwd_impl(fa_dtype dtype, const void* q, const void* k, const void* v, const void* o, const float* lse,
+                   const void* dout, void* dq, void* dk, void* dv, void* workspace, int B, int H, int N, int d,
+                   float scale, int causal, const uint8_t* mask, int32_t* trace, cudaStream_t stream) {
+  fa_status s = check_common(dtype, B, H, N, d);
+  if (s != FA_OK) return s;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) || !aligned16(dout) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return FA_ERR_INVALID_ARG;
+  if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FA_ERR_INVALID_ARG;
+  fa::AttnArgs a{};
+  a.dtype = dtype;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.o = o;
+  a.lse = const_cast<float*>(lse);
+  a.dout = dout;
+  a.dq = dq;
+  a.dk = dk;
+  a.dv = dv;
+  a.workspace = workspace;
+  a.B = B;
+  a.H = H;
+  a.N = N;
+  a.d = d;
+  a.scale = scale;
+  a.causal = causal ? 1 : 0;
+  a.block_mask = mask;
+  a.trace = trace;
+  a.status = status_word();
+  if (!a.status) return FA_ERR_CUDA;
+  return fa::launch_bwd(a, stream) == 0 ? FA_OK : FA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* fa_status_string(fa_status s) {
+  switch (s) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_INVALID_ARG: return "FA_ERR_INVALID_ARG";
+    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED";
+    case FA_ERR_CUDA: return "FA_ERR_CUDA";
+    case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT";
+  }
+  return "FA_ERR_UNKNOWN";
+}
+
+fa_status fa_fwd(fa_dtype dtype, const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                 int N, int d, float softmax_scale, int causal, cudaStream_t stream) {
+  return fwd_impl(dtype, q, k, v, o, lse, B, H, N, d, softmax_scale, causal, nullptr, nullptr, stream);
+}
+
+fa_status fa_blocksparse_fwd(fa_dtype dtype, const void* q, const void* k, const void* v, void* o, float* lse,
+                             int B, int H, int N, int d, float softmax_scale, int causal,
+                             const uint8_t* block_mask, cudaStream_t stream) {
+  fa_status s = check_mask(N, d, block_mask);
+  if (s != FA_OK) return s;
+  return fwd_impl(dtype, q, k, v, o, lse, B, H, N, d, softmax_scale, causal, block_mask, nullptr, stream);
+}
+
+size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
+  if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 128)) return 0;
+  return fa::bwd_workspace_layout(B, H, N, d).total;
+}
+
+int fa_bwd_row_tile(int d) { return fa::bwd_row_tile(d); }
+
+fa_status fa_bwd(fa_dtype dtype, const void* q, const void* k, const void* v, const void* o, const float* lse,
+                 const void* dout, void* dq, void* dk, void* dv, void* workspace, int B, int H, int N, int d,
+                 float softmax_scale, int causal, cudaStream_t stream) {
+  return bwd_impl(dtype, q, k, v, o, lse, dout, dq, dk, dv, workspace, B, H, N, d, softmax_scale, causal, nullptr,
+                  nullptr, stream);
+}
+
+fa_status fa_blocksparse_bwd(fa_dtype dtype, const void* q, const void* k, const void* v, const void* o,
+                             const float* lse, const void* dout, void* dq, void* dk, void* dv, void* workspace,
+                             int B, int H, int N, int d, float softmax_scale, int causal,
+                             const uint8_t* block_mask, cudaStream_t stream) {
+  fa_status s = check_mask(N, d, block_mask);
+  if (s != FA_OK) return s;
+  return bwd_impl(dtype, q, k, v, o, lse, dout, dq, dk, dv, workspace, B, H, N, d, softmax_scale, causal,
+                  block_mask, nullptr, stream);
+}
+
+size_t fa_fwd_trace_size(int B, int H, int N) {
+  if (B < 1 || H < 1 || N < 1) return 0;
+  const size_t tiles = (static_cast<size_t>(N) + 127) / 128;
+  const size_t pairs = (tiles + 1) / 2;
+  return static_cast<size_t>(B) * H * pairs * (tiles + 1);
+}
+
+size_t fa_bwd_trace_size(int B, int H, int N, int d) {
+  if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 128)) return 0;
+  const size_t tkv = (static_cast<size_t>(N) + 127) / 128;
+  const size_t br = static_cast<size_t>(fa::bwd_row_tile(d));
+  const size_t tq = (static_cast<size_t>(N) + br - 1) / br;
+  return static_cast<size_t>(B) * H * tkv * (tq + 1);
+}
+
+fa_status fa_debug_fwd_trace(fa_dtype dtype, const void* q, const void* k, const void* v, void* o, float* lse,
+                             int B, int H, int N, int d, float softmax_scale, int causal,
+                             const uint8_t* block_mask, int32_t* trace, cudaStream_t stream) {
+  if (trace == nullptr) return FA_ERR_INVALID_ARG;
+  if (block_mask) {
+    fa_status s = check_mask(N, d, block_mask);
+    if (s != FA_OK) return s;
+  }
+  return fwd_impl(dtype, q, k, v, o, lse, B, H, N, d, softmax_scale, causal, block_mask, trace, stream);
+}
+
+fa_status fa_debug_bwd_trace(fa_dtype dtype, const void* q, const void* k, const void* v, const void* o,
+                             const float* lse, const void* dout, void* dq, void* dk, void* dv, void* workspace,
+                             int B, int H, int N, int d, float softmax_scale, int causal,
+                             const uint8_t* block_mask, int32_t* trace, cudaStream_t stream) {
+  if (trace == nullptr) return FA_ERR_INVALID_ARG;
+  if (block_mask) {
+    fa_status s = check_mask(N, d, block_mask);
+    if (s != FA_OK) return s;
+  }
+  return bwd_impl(dtype, q, k, v, o, lse, dout, dq, dk, dv, workspace, B, H, N, d, softmax_scale, causal,
+                  block_mask, trace, stream);
+}
+
+fa_status fa_device_status(cudaStream_t stream) {
+  int* w = status_word();
+  if (!w) return FA_ERR_CUDA;
+  int h = 0;
+  if (cudaMemcpyAsync(&h, w, sizeof(int), cudaMemcpyDeviceToHost, stream) != cudaSuccess) return FA_ERR_CUDA;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return FA_ERR_CUDA;
+  if (cudaMemsetAsync(w, 0, sizeof(int), stream) != cudaSuccess) return FA_ERR_CUDA;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return FA_ERR_CUDA;
+  return static_cast<fa_status>(h);
+}
+
+fa_status fa_debug_timeout_probe(int timeout_ms, cudaStream_t stream) {
+  if (timeout_ms < 1 || timeout_ms > 5000) return FA_ERR_INVALID_ARG;
+  int* w = status_word();
+  if (!w) return FA_ERR_CUDA;
+  timeout_probe_kernel<<<1, 32, 0, stream>>>(w, static_cast<uint64_t>(timeout_ms) * 1000000ull);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,48 @@
+// Host launcher of the fused forward kernel.
+#include "fa_fwd.cuh"
+#include "fa_internal.h"
+#include "tma_host.h"
+
+namespace fa {
+
+namespace {
+
+template <int D, bool BF16>
+int launch_fwd_t(const AttnArgs& a, cudaStream_t stream) {
+  using L = fwd::Smem<D>;
+  const int BH = a.B * a.H;
+  const CUtensorMapDataType dt = BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  CUtensorMap tq, tk, tv;
+  bool ok = host::make_map_3d(&tq, dt, 2, a.q, D, a.N, BH, 64, fwd::kBlockM, CU_TENSOR_MAP_SWIZZLE_128B) &&
+            host::make_map_3d(&tk, dt, 2, a.k, D, a.N, BH, 64, fwd::kBlockN, CU_TENSOR_MAP_SWIZZLE_128B) &&
+            host::make_map_3d(&tv, dt, 2, a.v, D, a.N, BH, 64, fwd::kBlockN, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!ok) return static_cast<int>(cudaErrorInvalidValue);
+  fwd::Params p;
+  p.o = const_cast<void*>(a.o);
+  p.lse = a.lse;
+  p.block_mask = a.block_mask;
+  p.trace = a.trace;
+  p.status = a.status;
+  p.N = a.N;
+  p.BH = BH;
+  const int Tq = (a.N + fwd::kBlockM - 1) / fwd::kBlockM;
+  p.n_pairs = (Tq + 1) / 2;
+  p.Tc = (a.N + fwd::kBlockN - 1) / fwd::kBlockN;
+  p.causal = a.causal;
+  p.scale_log2 = a.scale * 1.4426950408889634f;
+  auto kern = fwd::fa_fwd_kernel<D, BF16>;
+  cudaError_t e = host::ensure_dynamic_smem(reinterpret_cast<const void*>(kern), L::kAlloc);
+  if (e != cudaSuccess) return static_cast<int>(e);
+  dim3 grid(BH, p.n_pairs);
+  kern<<<grid, fwd::kThreads, L::kAlloc, stream>>>(tq, tk, tv, p);
+  return static_cast<int>(cudaGetLastError());
+}
+
+}  // namespace
+
+int launch_fwd(const AttnArgs& a, cudaStream_t stream) {
+  if (a.d == 64) return a.dtype == 1 ? launch_fwd_t<64, true>(a, stream) : launch_fwd_t<64, false>(a, stream);
+  return a.dtype == 1 ? launch_fwd_t<128, true>(a, stream) : launch_fwd_t<128, false>(a, stream);
+}
+
+}  // namespace fa

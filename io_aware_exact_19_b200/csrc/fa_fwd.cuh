@@ -1,0 +1,457 @@
+// Fused exact attention forward for sm_100a.
+//
+// One CTA owns two 128-row query tiles (2p, 2p+1) of one (batch, head) and
+// streams the 128-key tiles of K and V past them, as in FlashAttention's
+// tiling ("FlashAttention" interview explainer, mstx.cn/posts/485, section 3.1)
+// with the loop nest inverted so that the running statistics of a query tile
+// stay on chip for its whole pass. Per key tile j and query tile q:
+//   S = Q_q K_j^T                       tcgen05.mma, fp32 accumulator in TMEM
+//   online softmax on S (running max m, sum l)   -- same explainer, section 3.2
+//   O_q = alpha * O_q + P V_j           tcgen05.mma, P read from TMEM
+// and only O = O_q / l and lse = (m + log2 l) * ln 2 are written to HBM.
+//
+// Warp roles (384 threads, one CTA per SM):
+//   warp 0      TMA producer: Q once, then K_j and V_j into two smem rings
+//   warp 1      MMA issuer (one lane) and TMEM owner
+//   warp 2      builds the key-tile list of a block-sparse CTA
+//   warps 4-7   softmax for query tile 0 (thread = row, lane of TMEM)
+//   warps 8-11  softmax for query tile 1
+// The two softmax warpgroups alternate with the tensor core: while one turns
+// its S into P, the tensor core runs the other tile's P V and next Q K^T.
+//
+// TMEM (512 columns): S/P of tile q at columns 128q .. 128q+127 (P is written
+// over the first 64 columns as packed 16-bit pairs), O of tile q at 256 + q*D.
+//
+// Softmax detail: scores are used in the log2 domain, s2 = S * scale * log2(e),
+// so exp is one FFMA plus ex2. The running max used for exponentiation is only
+// moved when the new row max exceeds it by more than 8 (a factor 256), which
+// leaves P <= 256 and keeps O and l consistent; the final O / l and lse are the
+// same quantities in exact arithmetic, and the rescale of O (read, scale, write
+// back in TMEM) is skipped for almost every tile.
+#pragma once
+
+#include "sm100.cuh"
+
+namespace fa {
+namespace fwd {
+
+using namespace fa::sm100;
+
+constexpr int kBlockM = 128;  // query rows per tile
+constexpr int kBlockN = 128;  // keys per tile
+constexpr int kThreads = 384;
+constexpr int kMaxSparseTiles = 2048;
+constexpr float kRescaleThreshold = 8.0f;
+
+struct Params {
+  void* o;
+  float* lse;
+  const uint8_t* block_mask;  // null unless block-sparse
+  int32_t* trace;             // null unless tracing
+  int* status;
+  int N;
+  int BH;
+  int n_pairs;  // ceil(T_q / 2)
+  int Tc;       // ceil(N / 128)
+  int causal;
+  float scale_log2;  // softmax scale * log2(e)
+};
+
+template <int D>
+struct Smem {
+  static constexpr int kStages = (D == 128) ? 2 : 3;
+  static constexpr int kTileBytes = kBlockN * D * 2;  // one K or V tile (and one Q tile)
+  static constexpr int kQOff = 0;
+  static constexpr int kKOff = kQOff + 2 * kTileBytes;
+  static constexpr int kVOff = kKOff + kStages * kTileBytes;
+  static constexpr int kBarOff = kVOff + kStages * kTileBytes;
+  // barriers: q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_full[2], o_full[2]
+  static constexpr int kNumBars = 1 + 4 * kStages + 6;
+  static constexpr int kListOff = kBarOff + 8 * kNumBars + 16;  // + tmem slot, abort flag, list length
+  static constexpr int kBytes = kListOff + 4 * kMaxSparseTiles;
+  static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1024
+};
+
+// Key-tile iteration shared by every role: entry n of the CTA's list is key
+// tile j(n) with flags f(n) (bit q set: query tile 2p+q uses it).
+struct TileList {
+  int len;
+  int mode;  // 0 dense, 1 causal, 2 list in shared memory
+  int q0;    // first query tile index (2p)
+  int q1_active;
+  const uint32_t* list;
+
+  __device__ __forceinline__ uint32_t entry(int n) const {
+    if (mode == 2) return list[n];
+    uint32_t f;
+    if (mode == 0) {
+      f = 1u | (q1_active ? 2u : 0u);
+    } else {
+      f = (n <= q0 ? 1u : 0u) | ((q1_active && n <= q0 + 1) ? 2u : 0u);
+    }
+    return static_cast<uint32_t>(n) | (f << 16);
+  }
+};
+
+template <int D, bool BF16>
+__global__ void __launch_bounds__(kThreads, 1)
+    fa_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
+                  const __grid_constant__ CUtensorMap tmap_v, const Params p) {
+  using L = Smem<D>;
+  constexpr int S = L::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kBarOff + 8 * L::kNumBars);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kBarOff + 8 * L::kNumBars + 4);
+  int* list_len = reinterpret_cast<int*>(smem + L::kBarOff + 8 * L::kNumBars + 8);
+  uint32_t* list = reinterpret_cast<uint32_t*>(smem + L::kListOff);
+
+  const uint32_t bar_q_full = smem_u32(&bars[0]);
+  auto bar_k_full = [&](int s) { return smem_u32(&bars[1 + s]); };
+  auto bar_k_empty = [&](int s) { return smem_u32(&bars[1 + S + s]); };
+  auto bar_v_full = [&](int s) { return smem_u32(&bars[1 + 2 * S + s]); };
+  auto bar_v_empty = [&](int s) { return smem_u32(&bars[1 + 3 * S + s]); };
+  auto bar_s_full = [&](int q) { return smem_u32(&bars[1 + 4 * S + q]); };
+  auto bar_p_full = [&](int q) { return smem_u32(&bars[1 + 4 * S + 2 + q]); };
+  auto bar_o_full = [&](int q) { return smem_u32(&bars[1 + 4 * S + 4 + q]); };
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  // Heaviest query tiles first: blocks are dispatched x-fastest, x runs over heads.
+  const int bh = blockIdx.x;
+  const int pair = p.n_pairs - 1 - static_cast<int>(blockIdx.y);
+  const int q0 = 2 * pair;
+  const int Tq = (p.N + kBlockM - 1) / kBlockM;
+  const int q1_active = (q0 + 1) < Tq;
+  const int cta = bh * p.n_pairs + pair;
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    mbar_init(bar_q_full, 1);
+    for (int s = 0; s < S; ++s) {
+      mbar_init(bar_k_full(s), 1);
+      mbar_init(bar_k_empty(s), 1);
+      mbar_init(bar_v_full(s), 1);
+      mbar_init(bar_v_empty(s), 1);
+    }
+    for (int q = 0; q < 2; ++q) {
+      mbar_init(bar_s_full(q), 1);
+      mbar_init(bar_p_full(q), 128);
+      mbar_init(bar_o_full(q), 1);
+    }
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  if (warp == 2) {
+    if (p.block_mask != nullptr) {
+      // Union of the non-zero key tiles of mask rows q0 and q0+1, in order, with
+      // the causal valid-tile rule (j <= q for 128x128 tiles) applied by AND.
+      const uint8_t* row0 = p.block_mask + static_cast<size_t>(q0) * p.Tc;
+      const uint8_t* row1 = row0 + p.Tc;
+      int count = 0;
+      for (int base = 0; base < p.Tc; base += 32) {
+        const int j = base + lane;
+        uint32_t f = 0;
+        if (j < p.Tc) {
+          if (row0[j] && (!p.causal || j <= q0)) f |= 1u;
+          if (q1_active && row1[j] && (!p.causal || j <= q0 + 1)) f |= 2u;
+        }
+        const uint32_t ballot = __ballot_sync(0xffffffffu, f != 0);
+        if (f != 0) {
+          const int pos = count + __popc(ballot & ((1u << lane) - 1u));
+          if (pos < kMaxSparseTiles) list[pos] = static_cast<uint32_t>(j) | (f << 16);
+        }
+        count += __popc(ballot);
+      }
+      if (lane == 0) *list_len = count < kMaxSparseTiles ? count : kMaxSparseTiles;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  const uint32_t tmem = *tmem_slot;
+  WaitCtx ctx{abort_flag, p.status};
+
+  TileList tl;
+  tl.q0 = q0;
+  tl.q1_active = q1_active;
+  tl.list = list;
+  if (p.block_mask != nullptr) {
+    tl.mode = 2;
+    tl.len = *list_len;
+  } else if (p.causal) {
+    tl.mode = 1;
+    tl.len = min(p.Tc, q1_active ? q0 + 2 : q0 + 1);
+  } else {
+    tl.mode = 0;
+    tl.len = p.Tc;
+  }
+
+  uint8_t* sQ = smem + L::kQOff;
+  uint8_t* sK = smem + L::kKOff;
+  uint8_t* sV = smem + L::kVOff;
+  constexpr int kChunkBytes = 128 * 128;  // one 128-row x 64-column swizzled chunk
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0 && tl.len > 0) {
+      prefetch_tmap(&tmap_q);
+      prefetch_tmap(&tmap_k);
+      prefetch_tmap(&tmap_v);
+      const int nq = 1 + q1_active;
+      mbar_arrive_expect_tx(bar_q_full, nq * L::kTileBytes);
+      for (int q = 0; q < nq; ++q)
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_3d(smem_u32(sQ + q * L::kTileBytes + c * kChunkBytes), &tmap_q, bar_q_full, c * 64,
+                      (q0 + q) * kBlockM, bh);
+      if (p.trace) p.trace[static_cast<size_t>(cta) * (p.Tc + 1)] = tl.len;
+      for (int n = 0; n < tl.len; ++n) {
+        const uint32_t e = tl.entry(n);
+        const int j = static_cast<int>(e & 0xFFFFu);
+        if (p.trace) p.trace[static_cast<size_t>(cta) * (p.Tc + 1) + 1 + n] = static_cast<int32_t>(e);
+        const int s = n % S;
+        const uint32_t ph = ((n / S) & 1) ^ 1;
+        if (!mbar_wait(bar_k_empty(s), ph, ctx)) break;
+        mbar_arrive_expect_tx(bar_k_full(s), L::kTileBytes);
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_3d(smem_u32(sK + s * L::kTileBytes + c * kChunkBytes), &tmap_k, bar_k_full(s), c * 64,
+                      j * kBlockN, bh);
+        if (!mbar_wait(bar_v_empty(s), ph, ctx)) break;
+        mbar_arrive_expect_tx(bar_v_full(s), L::kTileBytes);
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_3d(smem_u32(sV + s * L::kTileBytes + c * kChunkBytes), &tmap_v, bar_v_full(s), c * 64,
+                      j * kBlockN, bh);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && tl.len > 0) {
+      constexpr uint32_t idesc_s = idesc_f16(BF16, kBlockM, kBlockN, false, false);
+      constexpr uint32_t idesc_pv = idesc_f16(BF16, kBlockM, D, false, true);
+      uint32_t p_count[2] = {0, 0};
+      uint32_t started[2] = {0, 0};
+      bool ok = mbar_wait(bar_q_full, 0, ctx);
+
+      auto issue_s = [&](int q, int n) {
+        const int s = n % S;
+        const uint32_t d_tmem = tmem + q * 128;
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const int kk = k * 16;
+          const uint32_t off = (kk / 64) * kChunkBytes + (kk % 64) * 2;
+          const uint64_t a = sdesc_sw128(smem_u32(sQ + q * L::kTileBytes + off), 16, 1024);
+          const uint64_t b = sdesc_sw128(smem_u32(sK + s * L::kTileBytes + off), 16, 1024);
+          umma_ss(d_tmem, a, b, idesc_s, k > 0);
+        }
+        umma_commit(bar_s_full(q));
+      };
+      auto issue_pv = [&](int q, int n) {
+        const int s = n % S;
+        const uint32_t d_tmem = tmem + 256 + q * D;
+        const uint32_t a_tmem = tmem + q * 128;
+#pragma unroll
+        for (int k = 0; k < kBlockN / 16; ++k) {
+          const int kk = k * 16;
+          const uint64_t b = sdesc_sw128(smem_u32(sV + s * L::kTileBytes + kk * 128), kChunkBytes, 1024);
+          umma_ts(d_tmem, a_tmem + kk / 2, b, idesc_pv, (started[q] | static_cast<uint32_t>(k > 0)));
+        }
+        started[q] = 1;
+      };
+
+      // Prologue: S of the first key tile for each query tile that uses it.
+      if (ok) ok = mbar_wait(bar_k_full(0), 0, ctx);
+      if (ok) {
+        tc_fence_after();
+        const uint32_t f0 = tl.entry(0) >> 16;
+        for (int q = 0; q < 2; ++q)
+          if (f0 & (1u << q)) issue_s(q, 0);
+        umma_commit(bar_k_empty(0));
+      }
+      for (int n = 0; ok && n < tl.len; ++n) {
+        const uint32_t f = tl.entry(n) >> 16;
+        const bool has_next = (n + 1) < tl.len;
+        const uint32_t fn = has_next ? (tl.entry(n + 1) >> 16) : 0u;
+        if (has_next) {
+          if (!(ok = mbar_wait(bar_k_full((n + 1) % S), ((n + 1) / S) & 1, ctx))) break;
+        }
+        if (!(ok = mbar_wait(bar_v_full(n % S), (n / S) & 1, ctx))) break;
+        tc_fence_after();
+        for (int q = 0; q < 2; ++q) {
+          if (f & (1u << q)) {
+            if (!(ok = mbar_wait(bar_p_full(q), p_count[q] & 1, ctx))) break;
+            ++p_count[q];
+            tc_fence_after();
+            issue_pv(q, n);
+          }
+          if (fn & (1u << q)) issue_s(q, n + 1);
+        }
+        if (!ok) break;
+        umma_commit(bar_v_empty(n % S));
+        if (has_next) umma_commit(bar_k_empty((n + 1) % S));
+      }
+      if (ok) {
+        for (int q = 0; q < 2; ++q)
+          if (started[q]) umma_commit(bar_o_full(q));
+      }
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ softmax
+    const int q = (warp - 4) / 4;  // query tile within the pair
+    const int wq = warp % 4;       // TMEM lane quarter
+    const int qt = q0 + q;
+    const int row_local = wq * 32 + lane;
+    const int row = qt * kBlockM + row_local;
+    const bool tile_active = (q == 0) || q1_active;
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t t_s = tmem + lane_off + q * 128;
+    const uint32_t t_o = tmem + lane_off + 256 + q * D;
+    const float sl2 = p.scale_log2;
+
+    float m_ref = -INFINITY;  // log2-domain reference max
+    float l_sum = 0.0f;
+    int count = 0;
+    bool ok = true;
+
+    if (tile_active) {
+      for (int n = 0; n < tl.len; ++n) {
+        const uint32_t e = tl.entry(n);
+        if (!((e >> 16) & (1u << q))) continue;
+        const int j = static_cast<int>(e & 0xFFFFu);
+        if (!(ok = mbar_wait_warp(bar_s_full(q), count & 1, ctx))) break;
+        tc_fence_after();
+        uint32_t sr[128];
+        tmem_ld32(t_s + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+        tmem_ld32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+        tmem_ld32(t_s + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
+        tmem_ld32(t_s + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
+        tmem_ld_wait();
+        float* s = reinterpret_cast<float*>(sr);
+
+        // Element mask: causal diagonal tile (key > row) and keys past N.
+        int limit = kBlockN - 1;
+        if (p.causal && j == qt) limit = row_local;
+        const int kv_left = p.N - j * kBlockN - 1;
+        if (kv_left < limit) limit = kv_left;
+        if (limit < kBlockN - 1) {
+#pragma unroll
+          for (int c = 0; c < kBlockN; ++c)
+            if (c > limit) s[c] = -INFINITY;
+        }
+
+        float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+#pragma unroll
+        for (int c = 4; c < kBlockN; c += 4) {
+          mx0 = fmaxf(mx0, s[c]);
+          mx1 = fmaxf(mx1, s[c + 1]);
+          mx2 = fmaxf(mx2, s[c + 2]);
+          mx3 = fmaxf(mx3, s[c + 3]);
+        }
+        const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+
+        if (count == 0) {
+          m_ref = mx;
+        } else {
+          const bool need = mx > m_ref + kRescaleThreshold;
+          if (__any_sync(0xffffffffu, need)) {
+            const float alpha = need ? ex2(m_ref - mx) : 1.0f;
+            if (need) {
+              l_sum *= alpha;
+              m_ref = mx;
+            }
+#pragma unroll
+            for (int c = 0; c < D; c += 32) {
+              uint32_t o[32];
+              tmem_ld32(t_o + c, o);
+              tmem_ld_wait();
+#pragma unroll
+              for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+              tmem_st32(t_o + c, o);
+            }
+            tmem_st_wait();
+          }
+        }
+        const float m_use = (m_ref == -INFINITY) ? 0.0f : m_ref;
+
+        float ls0 = 0.f, ls1 = 0.f, ls2 = 0.f, ls3 = 0.f;
+#pragma unroll
+        for (int c = 0; c < kBlockN; c += 4) {
+          s[c] = ex2(fmaf(s[c], sl2, -m_use));
+          s[c + 1] = ex2(fmaf(s[c + 1], sl2, -m_use));
+          s[c + 2] = ex2(fmaf(s[c + 2], sl2, -m_use));
+          s[c + 3] = ex2(fmaf(s[c + 3], sl2, -m_use));
+          ls0 += s[c];
+          ls1 += s[c + 1];
+          ls2 += s[c + 2];
+          ls3 += s[c + 3];
+        }
+        l_sum += (ls0 + ls1) + (ls2 + ls3);
+
+        uint32_t pk[64];
+#pragma unroll
+        for (int i = 0; i < 64; ++i) pk[i] = pack2<BF16>(s[2 * i], s[2 * i + 1]);
+        tmem_st32(t_s + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+        tmem_st32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(bar_p_full(q));
+        ++count;
+      }
+
+      // Epilogue: O / l and lse for the rows of this tile that exist.
+      bool have_o = false;
+      if (ok && count > 0) {
+        ok = mbar_wait_warp(bar_o_full(q), 0, ctx);
+        have_o = ok;
+      }
+      tc_fence_after();
+      const size_t row_base = static_cast<size_t>(bh) * p.N;
+      const bool row_valid = row < p.N;
+      const float inv_l = (l_sum > 0.0f) ? 1.0f / l_sum : 0.0f;
+      uint16_t* orow = reinterpret_cast<uint16_t*>(p.o) + (row_base + (row_valid ? row : 0)) * D;
+      if (ok) {
+#pragma unroll
+        for (int c = 0; c < D; c += 32) {
+          uint32_t o[32];
+          if (have_o) {
+            tmem_ld32(t_o + c, o);
+            tmem_ld_wait();
+          }
+          uint32_t w[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float a = have_o ? __uint_as_float(o[2 * i]) * inv_l : 0.0f;
+            const float b = have_o ? __uint_as_float(o[2 * i + 1]) * inv_l : 0.0f;
+            w[i] = pack2<BF16>(a, b);
+          }
+          if (row_valid) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + c);
+            dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+            dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+            dst[2] = make_uint4(w[8], w[9], w[10], w[11]);
+            dst[3] = make_uint4(w[12], w[13], w[14], w[15]);
+          }
+        }
+        if (row_valid) {
+          const float lse = (l_sum > 0.0f) ? (m_ref + lg2(l_sum)) * 0.6931471805599453f : -INFINITY;
+          p.lse[row_base + row] = lse;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace fwd
+}  // namespace fa

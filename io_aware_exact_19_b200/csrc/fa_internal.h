@@ -1,0 +1,44 @@
+// Internal host interface between the C API (fa_api.cu) and the launchers.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+namespace fa {
+
+struct AttnArgs {
+  int dtype;  // 0 fp16, 1 bf16
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* o;  // forward: output
+  float* lse;     // forward: output; backward: input
+  const void* dout;
+  void* dq;
+  void* dk;
+  void* dv;
+  void* workspace;
+  int B, H, N, d;
+  float scale;
+  int causal;
+  const uint8_t* block_mask;
+  int32_t* trace;
+  int* status;
+};
+
+// Return 0 on success, a cudaError_t value otherwise.
+int launch_fwd(const AttnArgs& a, cudaStream_t stream);
+int launch_bwd(const AttnArgs& a, cudaStream_t stream);
+
+// Workspace layout of the backward, in bytes from the workspace base.
+struct BwdWorkspace {
+  size_t dq_acc;    // fp32 [BH][N][d]
+  size_t delta;     // fp32 [BH][Npad]  D = rowsum(dO o O)
+  size_t lse2;      // fp32 [BH][Npad]  lse * log2(e), +inf on padding rows
+  size_t total;
+};
+BwdWorkspace bwd_workspace_layout(int B, int H, int N, int d);
+int bwd_row_tile(int d);
+
+}  // namespace fa

@@ -25,6 +25,7 @@ Readings where the pages are silent or garbled are listed per function.
 from .attention import (  # noqa: F401
     allowed_mask,
     forward,
+    forward_rows,
     backward,
     online_forward,
     causal_tile_set,

@@ -102,6 +102,28 @@ def forward(q, k, v, scale: float, causal: bool = False, block_mask=None, tile: 
     return (O, lse, Ps) if return_p else (O, lse)
 
 
+def forward_rows(q, k, v, scale: float, rows, causal: bool = False, block_mask=None, tile: int = TILE):
+    """O and lse of the query rows ``rows`` only, for inputs [..., N, d].
+
+    The definition restricted to those rows: S[rows, :] = scale·Q[rows] Kᵀ,
+    masked, softmax per row, times V. Rows are independent, so nothing else is
+    needed; used where the full N×N problem is too large for the CPU.
+    """
+    q, k, v = (np.asarray(t, dtype=np.float64) for t in (q, k, v))
+    rows = np.asarray(rows)
+    lead = q.shape[:-2]
+    n = k.shape[-2]
+    allowed = _allowed_pairs(rows, np.arange(n), causal, block_mask, tile)
+    O = np.empty(lead + (rows.size, v.shape[-1]))
+    lse = np.empty(lead + (rows.size,))
+    for idx in np.ndindex(*lead):
+        S = scale * (q[idx][rows] @ k[idx].T)
+        S = np.where(allowed, S, -np.inf)
+        P, lse[idx] = _softmax_rows(S)
+        O[idx] = P @ v[idx]
+    return O, lse
+
+
 # --------------------------------------------------------------------------- backward
 
 def _head_backward(q, k, v, do, scale, allowed):

@@ -1,0 +1,170 @@
+"""Forward parity: the CUDA path through the C ABI against the fp64 oracle.
+
+Tolerances: O max-abs <= 1e-2 and lse max-abs <= 1e-3 for fp16/bf16 inputs drawn
+from N(0, 1); tile indexing bit-exact.
+"""
+import numpy as np
+import pytest
+import torch
+
+import fa_synth as S
+import io_aware_exact_19_b200 as fa
+import oracle
+from tests.gpu_inputs import Case, max_abs, to_device
+
+pytestmark = pytest.mark.gpu
+
+O_TOL, LSE_TOL = 1e-2, 1e-3
+
+
+def _run_fwd(c: Case, causal, mask_dev=None):
+    o, lse = fa.attention_forward(c.dev["q"], c.dev["k"], c.dev["v"], causal=causal, block_mask=mask_dev)
+    torch.cuda.synchronize()
+    assert fa.fa_device_status() == fa.FA_OK
+    return o, lse
+
+
+def _check_full(c: Case, causal, mask=None, heads=None):
+    mask_dev = None if mask is None else torch.from_numpy(mask).cuda()
+    o, lse = _run_fwd(c, causal, mask_dev)
+    O, L = oracle.forward(c.values("q", heads), c.values("k", heads), c.values("v", heads), c.scale,
+                          causal=causal, block_mask=mask)
+    eo = max_abs(c.flat(o, heads), O)
+    el = max_abs(c.flat(lse, heads), L)
+    assert eo <= O_TOL and el <= LSE_TOL, f"O err {eo:.3e}, lse err {el:.3e}"
+    return eo, el
+
+
+def test_tiny_fp16_exact_check():
+    _check_full(Case(1, 1, 128, 64, "fp16"), causal=False)
+
+
+@pytest.mark.parametrize("B,H,N,d,fmt,causal", [
+    (2, 3, 1000, 64, "bf16", False), (2, 3, 1000, 64, "bf16", True),
+    (1, 2, 1000, 128, "bf16", True), (1, 2, 777, 128, "fp16", False),
+    (1, 1, 1, 64, "bf16", False), (1, 1, 1, 128, "fp16", True),
+    (1, 2, 129, 64, "bf16", True), (2, 1, 256, 128, "bf16", False),
+    (1, 1, 384, 64, "fp16", True), (1, 3, 640, 128, "bf16", True),
+])
+def test_ragged_and_small(B, H, N, d, fmt, causal):
+    _check_full(Case(B, H, N, d, fmt, seed=N + d), causal)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_gpt2_small_shape(causal):
+    _check_full(Case(8, 12, 1024, 64, "bf16"), causal)
+
+
+def test_long_context_d128_causal_heads():
+    c = Case(4, 16, 4096, 128, "bf16")
+    _check_full(c, True, heads=[0, 21, 42, 63])
+
+
+def test_linear_memory_stress_sampled_rows():
+    c = Case(1, 16, 65536, 64, "bf16")
+    o, lse = _run_fwd(c, True)
+    rows = S.sample_rows(65536, 256, seed=1)
+    O, L = oracle.forward_rows(c.values("q"), c.values("k"), c.values("v"), c.scale, rows, causal=True)
+    eo = max_abs(c.flat(o)[:, rows], O)
+    el = max_abs(c.flat(lse)[:, rows], L)
+    assert eo <= O_TOL and el <= LSE_TOL, f"O err {eo:.3e}, lse err {el:.3e}"
+
+
+def test_block_sparse_workload_sampled_rows():
+    c = Case(2, 16, 8192, 64, "bf16")
+    mask = S.block_mask_recipe(64)
+    o, lse = _run_fwd(c, False, torch.from_numpy(mask).cuda())
+    rows = S.sample_rows(8192, 512, seed=1)
+    O, L = oracle.forward_rows(c.values("q"), c.values("k"), c.values("v"), c.scale, rows, block_mask=mask)
+    eo = max_abs(c.flat(o)[:, rows], O)
+    el = max_abs(c.flat(lse)[:, rows], L)
+    assert eo <= O_TOL and el <= LSE_TOL, f"O err {eo:.3e}, lse err {el:.3e}"
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("d", [64, 128])
+def test_block_sparse_full(causal, d):
+    mask = S.block_mask_recipe(8, seed=4)
+    _check_full(Case(2, 2, 1024, d, "bf16", seed=9), causal, mask=mask)
+
+
+def test_block_sparse_empty_row_tile():
+    # Query tile 1 has no key tile at all: O = 0 and lse = -inf there.
+    mask = np.ones((4, 4), dtype=np.uint8)
+    mask[1, :] = 0
+    _check_full(Case(1, 2, 512, 64, "bf16", seed=3), False, mask=mask)
+
+
+def test_unused_tiles_are_never_read():
+    # Key tile 5 is in no mask row: poison its K and V rows with NaN; the output must not change.
+    mask = S.block_mask_recipe(8, seed=5)
+    mask[:, 5] = 0
+    c = Case(1, 2, 1024, 64, "bf16", seed=11)
+    mdev = torch.from_numpy(mask).cuda()
+    o1, l1 = _run_fwd(c, False, mdev)
+    k, v = c.dev["k"].clone(), c.dev["v"].clone()
+    k[:, :, 640:768] = float("nan")
+    v[:, :, 640:768] = float("nan")
+    o2, l2 = fa.attention_forward(c.dev["q"], k, v, block_mask=mdev)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_identity_values_expose_exact_zeros(d):
+    # V = I (N = d): O = P, so every masked (causal) entry must be exactly 0.
+    N = d
+    c = Case(1, 1, N, d, "bf16", seed=2)
+    v = torch.eye(N, dtype=torch.bfloat16, device="cuda").reshape(1, 1, N, d).contiguous()
+    o, _ = fa.attention_forward(c.dev["q"], c.dev["k"], v, causal=True)
+    torch.cuda.synchronize()
+    upper = torch.triu(torch.ones(N, N, dtype=torch.bool, device="cuda"), diagonal=1)
+    assert torch.all(o[0, 0][upper] == 0)
+    assert torch.all(o[0, 0][~upper] > 0)
+
+
+def _expected_fwd_trace(N, causal, mask, BH):
+    lists = oracle.forward_tile_lists(N, causal, mask, 128, 128)
+    tq = len(lists)
+    pairs = (tq + 1) // 2
+    tc = -(-N // 128)
+    exp = np.zeros((BH, pairs, tc + 1), dtype=np.int64)
+    for p in range(pairs):
+        js = {}
+        for qq in (0, 1):
+            i = 2 * p + qq
+            if i < tq:
+                for j in lists[i]:
+                    js[j] = js.get(j, 0) | (1 << qq)
+        entries = [j | (f << 16) for j, f in sorted(js.items())]
+        exp[:, p, 0] = len(entries)
+        exp[:, p, 1:1 + len(entries)] = entries
+    return exp
+
+
+@pytest.mark.parametrize("N,causal,use_mask", [(1000, False, False), (1000, True, False), (1024, False, True),
+                                               (1024, True, True), (128, True, False), (1408, True, True)])
+def test_tile_trace_matches_oracle_enumeration(N, causal, use_mask):
+    B, H, d = 1, 2, 64
+    c = Case(B, H, N, d, "bf16", seed=1)
+    mask = S.block_mask_recipe(N // 128, seed=6) if use_mask else None
+    mdev = torch.from_numpy(mask).cuda() if use_mask else None
+    trace = torch.full((fa.fa_fwd_trace_size(B, H, N),), -1, dtype=torch.int32, device="cuda")
+    o = torch.empty_like(c.dev["q"])
+    lse = torch.empty((B, H, N), dtype=torch.float32, device="cuda")
+    fa.fa_debug_fwd_trace(c.dev["q"], c.dev["k"], c.dev["v"], o, lse, trace, causal=causal, block_mask=mdev)
+    torch.cuda.synchronize()
+    exp = _expected_fwd_trace(N, causal, mask, B * H)
+    got = trace.cpu().numpy().astype(np.int64).reshape(exp.shape)
+    for bh in range(B * H):
+        for p in range(exp.shape[1]):
+            n = exp[bh, p, 0]
+            assert got[bh, p, 0] == n
+            assert np.array_equal(got[bh, p, 1:1 + n], exp[bh, p, 1:1 + n]), (bh, p)
+
+
+def test_device_timeout_is_reported_and_cleared():
+    assert fa.fa_device_status() == fa.FA_OK
+    fa.fa_debug_timeout_probe(20)
+    assert fa.fa_device_status() == fa.FA_ERR_TIMEOUT
+    assert fa.fa_device_status() == fa.FA_OK

@@ -90,3 +90,15 @@ def test_tile_lists_match_mask_and_transpose(causal, br):
     pairs_b = {(i, j) for j, is_ in enumerate(bwd) for i in is_}
     assert pairs_f == pairs_b
     assert pairs_f == _tiles_with_allowed_pair(n, br, 128, causal, bm)
+
+
+def test_forward_rows_matches_full():
+    r = np.random.default_rng(13)
+    q, k, v = (r.standard_normal((2, 300, 8)) for _ in range(3))
+    rows = np.array([0, 1, 150, 255, 256, 299])
+    mask = np.array([[1, 0, 1], [0, 1, 1], [1, 1, 0]], dtype=np.uint8)
+    for causal, bm in ((False, None), (True, None), (False, mask), (True, mask)):
+        O, lse = oracle.forward(q, k, v, 0.3, causal=causal, block_mask=bm)
+        Or, lser = oracle.forward_rows(q, k, v, 0.3, rows, causal=causal, block_mask=bm)
+        np.testing.assert_allclose(Or, O[:, rows], rtol=0, atol=1e-13)
+        np.testing.assert_allclose(lser, lse[:, rows], rtol=0, atol=1e-13)
