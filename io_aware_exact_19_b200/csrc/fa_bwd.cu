@@ -1,9 +1,12 @@
-// Host launcher of the backward kernels (placeholder until the kernels land).
+// Host launchers of the backward kernels: prep (D, lse2, zero dQacc), the fused
+// main kernel, and finish (dQacc -> dQ).
+#include "fa_bwd.cuh"
 #include "fa_internal.h"
+#include "tma_host.h"
 
 namespace fa {
 
-int bwd_row_tile(int d) { return d == 128 ? 64 : 128; }
+int bwd_row_tile(int d) { return d == 128 ? bwd::Cfg<128>::BR : bwd::Cfg<64>::BR; }
 
 BwdWorkspace bwd_workspace_layout(int B, int H, int N, int d) {
   BwdWorkspace w{};
@@ -17,6 +20,84 @@ BwdWorkspace bwd_workspace_layout(int B, int H, int N, int d) {
   return w;
 }
 
-int launch_bwd(const AttnArgs&, cudaStream_t) { return static_cast<int>(cudaErrorNotSupported); }
+namespace {
+
+template <int D, bool BF16>
+int launch_bwd_t(const AttnArgs& a, cudaStream_t stream) {
+  using C = bwd::Cfg<D>;
+  const int BH = a.B * a.H;
+  const CUtensorMapDataType dt = BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  const BwdWorkspace ws = bwd_workspace_layout(a.B, a.H, a.N, D);
+  uint8_t* base = static_cast<uint8_t*>(a.workspace);
+
+  bwd::Params p;
+  p.o = a.o;
+  p.dout = a.dout;
+  p.lse = a.lse;
+  p.dq = a.dq;
+  p.dk = a.dk;
+  p.dv = a.dv;
+  p.dq_acc = reinterpret_cast<float*>(base + ws.dq_acc);
+  p.delta = reinterpret_cast<float*>(base + ws.delta);
+  p.lse2 = reinterpret_cast<float*>(base + ws.lse2);
+  p.block_mask = a.block_mask;
+  p.trace = a.trace;
+  p.status = a.status;
+  p.N = a.N;
+  p.Npad = (a.N + 127) / 128 * 128;
+  p.BH = BH;
+  p.Tq = (a.N + C::BR - 1) / C::BR;
+  p.Tc = (a.N + bwd::kBlockN - 1) / bwd::kBlockN;
+  p.causal = a.causal;
+  p.scale = a.scale;
+  p.scale_log2 = a.scale * 1.4426950408889634f;
+
+  CUtensorMap tq, tk, tv, tdo, tdq;
+  bool ok = host::make_map_3d(&tq, dt, 2, a.q, D, a.N, BH, 64, C::BR, CU_TENSOR_MAP_SWIZZLE_128B) &&
+            host::make_map_3d(&tdo, dt, 2, a.dout, D, a.N, BH, 64, C::BR, CU_TENSOR_MAP_SWIZZLE_128B) &&
+            host::make_map_3d(&tk, dt, 2, a.k, D, a.N, BH, 64, bwd::kBlockN, CU_TENSOR_MAP_SWIZZLE_128B) &&
+            host::make_map_3d(&tv, dt, 2, a.v, D, a.N, BH, 64, bwd::kBlockN, CU_TENSOR_MAP_SWIZZLE_128B) &&
+            (D == 64 ? host::make_map_3d(&tdq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, p.dq_acc, D, a.N, BH, 32, C::BR,
+                                         CU_TENSOR_MAP_SWIZZLE_128B)
+                     : host::make_map_3d(&tdq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, p.dq_acc, D, a.N, BH, D, C::BR,
+                                         CU_TENSOR_MAP_SWIZZLE_NONE));
+  if (!ok) return static_cast<int>(cudaErrorInvalidValue);
+
+  // prep: D/8 threads per padded row.
+  {
+    const long long threads = static_cast<long long>(BH) * p.Npad * (D / 8);
+    const long long blocks = threads / 256;  // Npad*(D/8) is a multiple of 1024
+    bwd::fa_bwd_prep_kernel<D, BF16><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return static_cast<int>(e);
+  }
+  // main
+  {
+    auto kern = bwd::fa_bwd_main_kernel<D, BF16>;
+    cudaError_t e = host::ensure_dynamic_smem(reinterpret_cast<const void*>(kern), C::kAlloc);
+    if (e != cudaSuccess) return static_cast<int>(e);
+    dim3 grid(BH, p.Tc);
+    kern<<<grid, bwd::kThreads, C::kAlloc, stream>>>(tq, tk, tv, tdo, tdq, p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return static_cast<int>(e);
+  }
+  // finish
+  {
+    const long long total4 = static_cast<long long>(BH) * a.N * D / 4;
+    long long blocks = (total4 + 255) / 256;
+    if (blocks > 148LL * 16) blocks = 148LL * 16;
+    bwd::fa_bwd_finish_kernel<D, BF16><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return static_cast<int>(e);
+  }
+  return 0;
+}
+
+}  // namespace
+
+int launch_bwd(const AttnArgs& a, cudaStream_t stream) {
+  if (a.d == 64) return a.dtype == 1 ? launch_bwd_t<64, true>(a, stream) : launch_bwd_t<64, false>(a, stream);
+  return a.dtype == 1 ? launch_bwd_t<128, true>(a, stream) : launch_bwd_t<128, false>(a, stream);
+}
 
 }  // namespace fa

@@ -1,0 +1,152 @@
+"""Backward parity: dQ, dK, dV from the CUDA path (forward then backward, through
+the C ABI) against the fp64 oracle. Tolerance: relative Frobenius error <= 2e-2
+per gradient; tile indexing bit-exact."""
+import numpy as np
+import pytest
+import torch
+
+import fa_synth as S
+import io_aware_exact_19_b200 as fa
+import oracle
+from tests.gpu_inputs import Case, rel_fro  # noqa: F401
+
+pytestmark = pytest.mark.gpu
+
+G_TOL = 2e-2
+
+
+def _grad_err(g, G):
+    """Relative Frobenius error; the denominator has a floor of RMS 1e-4 per element so
+    that a gradient that is exactly zero in exact arithmetic (a single key: P = 1,
+    dS = 0) is compared against that absolute scale instead of against 0."""
+    G = np.asarray(G, np.float64)
+    floor = 1e-4 * np.sqrt(G.size)
+    return float(np.linalg.norm(np.asarray(g, np.float64) - G) / max(np.linalg.norm(G), floor))
+
+
+def _run(c: Case, causal, mask=None):
+    mdev = None if mask is None else torch.from_numpy(mask).cuda()
+    q, k, v, do = (c.dev[n] for n in ("q", "k", "v", "do"))
+    o, lse = fa.attention_forward(q, k, v, causal=causal, block_mask=mdev)
+    dq, dk, dv = fa.attention_backward(q, k, v, o, lse, do, causal=causal, block_mask=mdev)
+    torch.cuda.synchronize()
+    assert fa.fa_device_status() == fa.FA_OK
+    return dq, dk, dv
+
+
+def _check_full(c: Case, causal, mask=None, heads=None):
+    dq, dk, dv = _run(c, causal, mask)
+    vals = [c.values(n, heads) for n in ("q", "k", "v", "do")]
+    DQ, DK, DV = oracle.backward(*vals, c.scale, causal=causal, block_mask=mask)
+    errs = [_grad_err(c.flat(g, heads), G) for g, G in ((dq, DQ), (dk, DK), (dv, DV))]
+    assert max(errs) <= G_TOL, f"rel Frobenius dQ/dK/dV = {errs}"
+    for g in (dq, dk, dv):
+        assert torch.isfinite(g).all()
+    return errs
+
+
+def test_tiny_fp16_exact_check():
+    _check_full(Case(1, 1, 128, 64, "fp16"), causal=False)
+
+
+@pytest.mark.parametrize("B,H,N,d,fmt,causal", [
+    (2, 3, 1000, 64, "bf16", False), (2, 3, 1000, 64, "bf16", True),
+    (1, 2, 1000, 128, "bf16", True), (1, 2, 777, 128, "fp16", False),
+    (1, 1, 1, 64, "bf16", False), (1, 1, 1, 128, "fp16", True),
+    (1, 2, 129, 64, "bf16", True), (2, 1, 256, 128, "bf16", False),
+    (1, 1, 384, 64, "fp16", True), (1, 3, 640, 128, "bf16", True),
+    (1, 1, 65, 128, "bf16", False),
+])
+def test_ragged_and_small(B, H, N, d, fmt, causal):
+    _check_full(Case(B, H, N, d, fmt, seed=N + d), causal)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_gpt2_small_shape(causal):
+    _check_full(Case(8, 12, 1024, 64, "bf16"), causal)
+
+
+def test_long_context_d128_causal_heads():
+    _check_full(Case(4, 16, 4096, 128, "bf16"), True, heads=[0, 21, 42, 63])
+
+
+def _check_sampled(c: Case, causal, mask, nq, nk):
+    dq, dk, dv = _run(c, causal, mask)
+    N = c.shape[2]
+    rows_q = S.sample_rows(N, nq, seed=1)
+    rows_k = S.sample_rows(N, nk, seed=2)
+    vals = [c.values(n) for n in ("q", "k", "v", "do")]
+    ref = oracle.sampled_forward_backward(*vals, c.scale, causal, rows_q, rows_k, block_mask=mask)
+    errs = [rel_fro(c.flat(dq)[:, rows_q], ref["dq"]), rel_fro(c.flat(dk)[:, rows_k], ref["dk"]),
+            rel_fro(c.flat(dv)[:, rows_k], ref["dv"])]
+    assert max(errs) <= G_TOL, f"rel Frobenius dQ/dK/dV (sampled rows) = {errs}"
+
+
+def test_linear_memory_stress_sampled_rows():
+    _check_sampled(Case(1, 16, 65536, 64, "bf16"), True, None, 256, 256)
+
+
+def test_block_sparse_workload_sampled_rows():
+    _check_sampled(Case(2, 16, 8192, 64, "bf16"), False, S.block_mask_recipe(64), 256, 256)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("d", [64, 128])
+def test_block_sparse_full(causal, d):
+    _check_full(Case(2, 2, 1024, d, "bf16", seed=9), causal, mask=S.block_mask_recipe(8, seed=4))
+
+
+def test_block_sparse_empty_row_and_column():
+    mask = np.ones((4, 4), dtype=np.uint8)
+    mask[1, :] = 0   # query tile 1 sees no key: zero dQ there
+    mask[:, 2] = 0   # key tile 2 is seen by no query: zero dK, dV there
+    for d in (64, 128):
+        c = Case(1, 2, 512, d, "bf16", seed=3)
+        dq, dk, dv = _run(c, False, mask)
+        assert torch.all(dq[:, :, 128:256] == 0)
+        assert torch.all(dk[:, :, 256:384] == 0) and torch.all(dv[:, :, 256:384] == 0)
+        _check_full(c, False, mask=mask)
+
+
+def test_unused_key_tile_is_never_read():
+    mask = S.block_mask_recipe(8, seed=5)
+    mask[:, 5] = 0
+    c = Case(1, 2, 1024, 64, "bf16", seed=11)
+    g1 = _run(c, False, mask)
+    k, v = c.dev["k"].clone(), c.dev["v"].clone()
+    k[:, :, 640:768] = float("nan")
+    v[:, :, 640:768] = float("nan")
+    mdev = torch.from_numpy(mask).cuda()
+    q, do = c.dev["q"], c.dev["do"]
+    o, lse = fa.attention_forward(q, k, v, block_mask=mdev)
+    g2 = fa.attention_backward(q, k, v, o, lse, do, block_mask=mdev)
+    torch.cuda.synchronize()
+    for a, b in zip(g1, g2):
+        assert torch.isfinite(b).all()
+        # dQ is accumulated by reductions whose order may differ between runs.
+        assert torch.allclose(a.float(), b.float(), rtol=0, atol=2e-3)
+
+
+@pytest.mark.parametrize("N,causal,use_mask,d", [(1000, False, False, 64), (1000, True, False, 128),
+                                                 (1024, False, True, 64), (1024, True, True, 128),
+                                                 (1408, True, True, 64)])
+def test_tile_trace_matches_oracle_enumeration(N, causal, use_mask, d):
+    B, H = 1, 2
+    c = Case(B, H, N, d, "bf16", seed=1)
+    mask = S.block_mask_recipe(N // 128, seed=6) if use_mask else None
+    mdev = torch.from_numpy(mask).cuda() if use_mask else None
+    q, k, v, do = (c.dev[n] for n in ("q", "k", "v", "do"))
+    o, lse = fa.attention_forward(q, k, v, causal=causal, block_mask=mdev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(fa.fa_bwd_workspace_size(B, H, N, d), dtype=torch.uint8, device="cuda")
+    trace = torch.full((fa.fa_bwd_trace_size(B, H, N, d),), -1, dtype=torch.int32, device="cuda")
+    fa.fa_debug_bwd_trace(q, k, v, o, lse, do, dq, dk, dv, ws, trace, causal=causal, block_mask=mdev)
+    torch.cuda.synchronize()
+    br = fa.fa_bwd_row_tile(d)
+    lists = oracle.backward_tile_lists(N, causal, mask, br=br, bc=128)
+    tq = -(-N // br)
+    got = trace.cpu().numpy().astype(np.int64).reshape(B * H, len(lists), tq + 1)
+    for bh in range(B * H):
+        for j, exp in enumerate(lists):
+            assert got[bh, j, 0] == len(exp)
+            assert list(got[bh, j, 1:1 + len(exp)]) == [i | (1 << 16) for i in exp], (bh, j)
