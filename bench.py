@@ -1,0 +1,468 @@
+#!/usr/bin/env python
+"""Benchmark of the exact fused attention path on B200.
+
+One step = one pass of the whole hot path over one batch of synthetic input:
+the forward (fa_fwd) and the backward (its three launches: prep, main, finish)
+of exact attention on the long-context causal workload B=4, H=16, N=4096,
+d=128, bf16, Q/K/V/dO iid N(0, 1).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+Rank 0 prints one JSON line. Multi-GPU runs (torchrun, one process per GPU)
+give every rank its own batch of the same workload (weak scaling); the path has
+no data exchange between ranks, so the only collectives are the barriers and
+the max-over-ranks of the timings.
+
+``--impl reference`` times the fp64 CPU oracle instead, on a bounded sample of
+the same workload per step (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "attention fwd/bwd TFLOP/s and % of B200 BF16 tensor peak (N=1K–64K)"
+UNIT = "TFLOP/s"
+L2_BYTES = 126 * 1024 * 1024
+
+WORKLOADS = {
+    "long_causal_d128": dict(B=4, H=16, N=4096, d=128, causal=True, fmt="bf16", mask=False,
+                             desc="long-context causal attention B=4 H=16 N=4096 d=128 bf16, fwd+bwd"),
+    "gpt2_small": dict(B=8, H=12, N=1024, d=64, causal=False, fmt="bf16", mask=False,
+                       desc="GPT-2-small-shaped attention B=8 H=12 N=1024 d=64 bf16, fwd+bwd"),
+    "gpt2_small_causal": dict(B=8, H=12, N=1024, d=64, causal=True, fmt="bf16", mask=False,
+                              desc="GPT-2-small-shaped causal attention B=8 H=12 N=1024 d=64 bf16, fwd+bwd"),
+    "linear_memory_64k": dict(B=1, H=16, N=65536, d=64, causal=True, fmt="bf16", mask=False,
+                              desc="linear-memory stress causal attention B=1 H=16 N=65536 d=64 bf16, fwd+bwd"),
+    "block_sparse_8k": dict(B=2, H=16, N=8192, d=64, causal=False, fmt="bf16", mask=True,
+                            desc="block-sparse attention B=2 H=16 N=8192 d=64 bf16, 128x128 tile mask, fwd+bwd"),
+}
+DEFAULT_WORKLOAD = "long_causal_d128"
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def workload_density(w) -> float:
+    if not w["mask"]:
+        return 1.0
+    import fa_synth
+    m = fa_synth.block_mask_recipe(w["N"] // 128)
+    return float(m.sum()) / m.size
+
+
+def step_flops(w, density=None):
+    """Algorithmic FLOPs: forward 4·B·H·N²·d, backward 2.5× that, halved for causal,
+    scaled by the non-zero tile fraction for block-sparse."""
+    if density is None:
+        density = workload_density(w)
+    f = 4.0 * w["B"] * w["H"] * w["N"] ** 2 * w["d"] * (0.5 if w["causal"] else 1.0) * density
+    return f, 2.5 * f
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"bf16": float(p["bf16_tflops"]), "bf16_sustained": float(p.get("bf16_tflops_sustained", 0) or 0),
+                "hbm": float(p["hbm_gbs"]), "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"bf16": 1590.0, "bf16_sustained": 1400.0, "hbm": 6650.0, "source": "fallback"}
+
+
+def load_traffic(kernel_key):
+    """DRAM bytes per launch from a committed ncu capture, if the kernel source is unchanged since."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)[kernel_key]
+    except (OSError, KeyError, ValueError):
+        return None
+    import hashlib
+    h = hashlib.sha256()
+    for name in rec.get("sources", []):
+        with open(os.path.join(ROOT, name), "rb") as f:
+            h.update(f.read())
+    if h.hexdigest() != rec.get("sha256"):
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling while the timed region runs."""
+
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str, path: str):
+        self.path = path
+        self.proc = None
+        try:
+            self.fh = open(path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", gpu_id, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.fh, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self, t0: float, t1: float):
+        rows = []
+        try:
+            with open(self.path) as f:
+                for line in f:
+                    parts = [x.strip() for x in line.split(",")]
+                    if len(parts) < 8:
+                        continue
+                    try:
+                        ts = time.mktime(time.strptime(parts[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                        frac = float("0." + parts[0].split(".")[1]) if "." in parts[0] else 0.0
+                        rows.append((ts + frac, float(parts[1]), float(parts[2]), parts[4:8]))
+                    except ValueError:
+                        continue
+        except OSError:
+            return None
+        if not rows:
+            return None
+        inside = [r for r in rows if t0 - 0.15 <= r[0] <= t1 + 0.15]
+        use = inside if len(inside) >= 1 else rows
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({names[i] for r in use for i, v in enumerate(r[3]) if v.lower().startswith("active")})
+        return {"sm_mhz": statistics.median(r[1] for r in use), "sm_max_mhz": max(r[2] for r in use),
+                "reasons": reasons, "samples": len(use), "samples_in_timed_region": len(inside)}
+
+
+def oracle_sample_step(vals, w, rows, head):
+    """One bounded sample of the workload on the CPU oracle: forward and backward of
+    the loss restricted to `rows` query rows of one head."""
+    import oracle
+    q, k, v, do = (vals[n][head] for n in ("q", "k", "v", "do"))
+    scale = 1.0 / math.sqrt(w["d"])
+    mask = None
+    if w["mask"]:
+        import fa_synth
+        mask = fa_synth.block_mask_recipe(w["N"] // 128)
+    oracle.backward_rows(q, k, v, do, scale, rows, causal=w["causal"], block_mask=mask)
+
+
+def oracle_inputs(w, heads, seed=0):
+    import fa_synth
+    bits = fa_synth.attention_input_bits(w["B"], w["H"], w["N"], w["d"], w["fmt"], seed)
+    return {n: fa_synth.bits_to_values(b.reshape((-1,) + b.shape[2:])[heads], w["fmt"]) for n, b in bits.items()}
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max((i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"), default=1)
+    except ImportError:
+        return 1
+
+
+def sample_rows_for(w, n_rows):
+    import numpy as np
+    step = w["N"] // n_rows
+    return np.arange(n_rows) * step + step // 2
+
+
+def cpu_rate(w, vals, n_rows, budget_s, min_steps=1, max_steps=None):
+    """Run oracle samples until `budget_s` seconds pass; returns (TFLOP/s, steps, seconds)."""
+    f_fwd, f_bwd = step_flops(w)
+    per_row = (f_fwd + f_bwd) / (w["B"] * w["H"] * w["N"])
+    rows = sample_rows_for(w, n_rows)
+    nheads = next(iter(vals.values())).shape[0]
+    t0 = time.perf_counter()
+    steps = 0
+    while True:
+        oracle_sample_step(vals, w, rows, steps % nheads)
+        steps += 1
+        el = time.perf_counter() - t0
+        if steps >= min_steps and (el >= budget_s or (max_steps and steps >= max_steps)):
+            break
+    return per_row * n_rows * steps / el / 1e12, steps, el
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+def run_reference(args, w, rank, world):
+    if rank != 0:
+        return 0
+    vals = oracle_inputs(w, list(range(min(4, w["B"] * w["H"]))))
+    f_fwd, f_bwd = step_flops(w)
+    per_row = (f_fwd + f_bwd) / (w["B"] * w["H"] * w["N"])
+    # Size the per-step sample so warm-up plus timed steps stay within about two minutes.
+    rows = sample_rows_for(w, 64)
+    t0 = time.perf_counter()
+    oracle_sample_step(vals, w, rows, 0)
+    t_probe = max(time.perf_counter() - t0, 1e-4)
+    n_rows = 64
+    target = 120.0 / max(1, args.steps + args.warmup)
+    while n_rows < min(w["N"], 2048) and t_probe * (2 * n_rows) / 64 <= target:
+        n_rows *= 2
+    rows = sample_rows_for(w, n_rows)
+    nheads = next(iter(vals.values())).shape[0]
+    for s in range(args.warmup):
+        oracle_sample_step(vals, w, rows, s % nheads)
+    t0 = time.perf_counter()
+    for s in range(args.steps):
+        oracle_sample_step(vals, w, rows, s % nheads)
+    el = time.perf_counter() - t0
+    value = per_row * n_rows * args.steps / el / 1e12
+    sample = f"{n_rows} of {w['N']} query rows of one (batch, head) per step, forward + backward of the loss on those rows"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_block(w, args.workload),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_block(w, name):
+    return {"workload": w["desc"], "name": name, "B": w["B"], "H": w["H"], "N": w["N"], "d": w["d"],
+            "causal": w["causal"], "block_sparse": w["mask"], "dtype": w["fmt"],
+            "l2": "inputs larger than L2 (no flush): " + str(
+                round(4 * w["B"] * w["H"] * w["N"] * w["d"] * 2 / 2 ** 20)) + " MiB of Q/K/V/dO per step",
+            "parallelism": "one independent batch per GPU"}
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+def run_gpu(args, w, rank, world, local_rank):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import fa_synth
+    import io_aware_exact_19_b200 as fa
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    B, H, N, d = w["B"], w["H"], w["N"], w["d"]
+    causal = w["causal"]
+    tdt = torch.bfloat16 if w["fmt"] == "bf16" else torch.float16
+
+    bits = fa_synth.attention_input_bits(B, H, N, d, w["fmt"], seed=rank)
+    host = {n: torch.from_numpy(b.view(np.int16)).view(tdt) for n, b in bits.items()}
+    q, k, v, do = (host[n].to(dev) for n in ("q", "k", "v", "do"))
+    mask = None
+    if w["mask"]:
+        mask = torch.from_numpy(fa_synth.block_mask_recipe(N // 128)).to(dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(fa.fa_bwd_workspace_size(B, H, N, d), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def fwd():
+        if mask is None:
+            fa.fa_fwd(q, k, v, o, lse, causal)
+        else:
+            fa.fa_blocksparse_fwd(q, k, v, o, lse, mask, causal)
+
+    def bwd_phase(ph):
+        fa.fa_debug_bwd_phase(ph, q, k, v, o, lse, do, dq, dk, dv, ws, causal=causal, block_mask=mask)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        fwd()
+        if ev is not None:
+            ev[1].record(stream)
+        bwd_phase(0)
+        if ev is not None:
+            ev[2].record(stream)
+        bwd_phase(1)
+        if ev is not None:
+            ev[3].record(stream)
+        bwd_phase(2)
+        if ev is not None:
+            ev[4].record(stream)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    if fa.fa_device_status() != fa.FA_OK:
+        raise RuntimeError("device status reported a time-out during warm-up")
+
+    import tempfile
+    gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    sampler = ClockSampler(gpu_id, os.path.join(tempfile.gettempdir(), f"fa_bench_clocks_rank{rank}_{os.getpid()}.csv"))
+    time.sleep(0.3)
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    for s in range(args.steps):
+        step(events[s])
+    torch.cuda.synchronize()
+    t_wall1 = time.time()
+    if world > 1:
+        dist.barrier()
+    time.sleep(0.2)
+    sampler.stop()
+    clocks = sampler.summary(t_wall0, t_wall1)
+    status = fa.fa_device_status()
+
+    ms_total = events[0][0].elapsed_time(events[-1][4])
+    fwd_ms = [e[0].elapsed_time(e[1]) for e in events]
+    prep_ms = [e[1].elapsed_time(e[2]) for e in events]
+    main_ms = [e[2].elapsed_time(e[3]) for e in events]
+    fin_ms = [e[3].elapsed_time(e[4]) for e in events]
+    if world > 1:
+        t = torch.tensor([ms_total, sum(main_ms), sum(fwd_ms)], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total, main_sum, fwd_sum = (float(x) for x in t.tolist())
+    else:
+        main_sum, fwd_sum = sum(main_ms), sum(fwd_ms)
+
+    f_fwd, f_bwd = step_flops(w)
+    value = world * (f_fwd + f_bwd) * args.steps / (ms_total * 1e-3) / 1e12
+    peaks = load_peaks()
+    main_avg = main_sum / args.steps
+    fwd_avg = fwd_sum / args.steps
+    achieved = f_bwd / (main_avg * 1e-3) / 1e12
+    bwd_all = statistics.mean(p + m + f for p, m, f in zip(prep_ms, main_ms, fin_ms))
+    prep_avg = statistics.mean(prep_ms)
+    prep_bytes = B * H * N * d * (2 + 2 + 4) + B * H * N * 4 * 3  # read O, dO; zero dQacc; lse in, D and lse2 out
+
+    # ---- end to end through the C ABI: pinned host inputs in, results back to pinned host memory
+    pin = {n: t.pin_memory() for n, t in host.items()}
+    out_host = {n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for n, t in
+                (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv))}
+    e2e_steps = max(1, min(args.steps, 20))
+
+    def e2e_step():
+        q.copy_(pin["q"], non_blocking=True)
+        k.copy_(pin["k"], non_blocking=True)
+        v.copy_(pin["v"], non_blocking=True)
+        do.copy_(pin["do"], non_blocking=True)
+        fwd()
+        if mask is None:
+            fa.fa_bwd(q, k, v, o, lse, do, dq, dk, dv, ws, causal)
+        else:
+            fa.fa_blocksparse_bwd(q, k, v, o, lse, do, dq, dk, dv, ws, mask, causal)
+        for n, t in (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv)):
+            out_host[n].copy_(t, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    h2d = sum(t.numel() * t.element_size() for t in pin.values())
+    d2h = sum(t.numel() * t.element_size() for t in out_host.values())
+    e2e_value = world * (f_fwd + f_bwd) * e2e_steps / (e2e_ms * 1e-3) / 1e12
+
+    if rank != 0:
+        return 0
+
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        vals = oracle_inputs(w, list(range(min(4, B * H))))
+        rate, n_steps, secs = cpu_rate(w, vals, 512 if N >= 4096 else min(N, 256), budget_s=12.0)
+        cpu = {"value": rate, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+               "sample": f"{n_steps} samples x 512 of {N} query rows of one (batch, head), forward + backward "
+                         f"of the loss on those rows, fp64, {secs:.1f} s"}
+
+    kernel_key = f"fa_bwd_main_kernel<{d},{'bf16' if w['fmt'] == 'bf16' else 'fp16'}>"
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": ms_total / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": w["fmt"], "data": "synthetic",
+        "config": config_block(w, args.workload),
+        "roofline": {"kernel": kernel_key, "bound": "tensor", "achieved": achieved, "peak": peaks["bf16"],
+                     "unit": UNIT, "frac": achieved / peaks["bf16"],
+                     "peak_source": f"{peaks['source']} bf16 dense burst", "traffic": load_traffic(kernel_key),
+                     "flops_per_launch": f_bwd},
+        "breakdown": {
+            "fwd_ms": fwd_avg, "fwd_tflops": f_fwd / (fwd_avg * 1e-3) / 1e12,
+            "fwd_frac_of_measured_peak": f_fwd / (fwd_avg * 1e-3) / 1e12 / peaks["bf16"],
+            "bwd_ms": bwd_all, "bwd_tflops": f_bwd / (bwd_all * 1e-3) / 1e12,
+            "bwd_frac_of_measured_peak": f_bwd / (bwd_all * 1e-3) / 1e12 / peaks["bf16"],
+            "bwd_main_ms": main_avg, "bwd_prep_ms": prep_avg, "bwd_finish_ms": statistics.mean(fin_ms),
+            "bwd_prep_gbs": prep_bytes / (prep_avg * 1e-3) / 1e9,
+            "vendor_peak_tflops": 2250.0,
+            "fwd_frac_of_vendor_peak": f_fwd / (fwd_avg * 1e-3) / 1e12 / 2250.0,
+            "bwd_frac_of_vendor_peak": f_bwd / (bwd_all * 1e-3) / 1e12 / 2250.0,
+        },
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "steps": e2e_steps},
+        "gpu_launches": 4 * args.steps,
+        "clocks": clocks,
+        "device_status": int(status),
+        "wall_s_timed_region": t_wall1 - t_wall0,
+    }
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    w = WORKLOADS[args.workload]
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus and "RANK" in os.environ:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
+    if args.impl == "reference":
+        return run_reference(args, w, rank, world)
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        return run_gpu(args, w, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

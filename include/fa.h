@@ -125,6 +125,19 @@ fa_status fa_debug_bwd_trace(fa_dtype dtype, const void* q, const void* k, const
                              const uint8_t* block_mask, int32_t* trace, cudaStream_t stream);
 
 /*
+ * Debug: one of the three launches fa_bwd makes, selected by `phase`:
+ * 0 = prep (D = rowsum(dO o O), lse in log2 units, zero the dQ accumulator),
+ * 1 = main (recompute P, accumulate dK, dV in TMEM and dQ in the workspace),
+ * 2 = finish (dQ = scale * accumulator, cast). Running phases 0, 1, 2 in order
+ * on one stream with the same arguments is exactly fa_bwd. Used to time the
+ * main kernel on its own.
+ */
+fa_status fa_debug_bwd_phase(int phase, fa_dtype dtype, const void* q, const void* k, const void* v,
+                             const void* o, const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                             void* workspace, int B, int H, int N, int d, float softmax_scale, int causal,
+                             const uint8_t* block_mask, cudaStream_t stream);
+
+/*
  * Device status: synchronises `stream`, returns the status word that kernels
  * set when a device-side wait timed out (FA_OK if none), and clears it.
  */

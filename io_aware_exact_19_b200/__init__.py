@@ -24,7 +24,8 @@ FA_FP16, FA_BF16 = 0, 1
 EXPORTED = (
     "fa_status_string", "fa_fwd", "fa_bwd", "fa_blocksparse_fwd", "fa_blocksparse_bwd",
     "fa_bwd_workspace_size", "fa_fwd_trace_size", "fa_bwd_trace_size", "fa_bwd_row_tile",
-    "fa_debug_fwd_trace", "fa_debug_bwd_trace", "fa_device_status", "fa_debug_timeout_probe",
+    "fa_debug_fwd_trace", "fa_debug_bwd_trace", "fa_debug_bwd_phase", "fa_device_status",
+    "fa_debug_timeout_probe",
 )
 
 
@@ -56,6 +57,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "fa_bwd": (bwd_args + [vp], i),
         "fa_blocksparse_bwd": (bwd_args + [vp, vp], i),
         "fa_debug_bwd_trace": (bwd_args + [vp, vp, vp], i),
+        "fa_debug_bwd_phase": ([i] + bwd_args + [vp, vp], i),
         "fa_bwd_workspace_size": ([i, i, i, i], sz),
         "fa_fwd_trace_size": ([i, i, i], sz),
         "fa_bwd_trace_size": ([i, i, i, i], sz),
@@ -197,6 +199,17 @@ def fa_debug_bwd_trace(q, k, v, o, lse, dout, dq, dk, dv, workspace, trace, caus
                                            _scale(scale, d), int(bool(causal)), _ptr(block_mask), _ptr(trace),
                                            _stream(stream))
     _check(st, "fa_debug_bwd_trace")
+
+
+def fa_debug_bwd_phase(phase: int, q, k, v, o, lse, dout, dq, dk, dv, workspace, causal: bool = False,
+                       block_mask=None, scale=None, stream=None) -> None:
+    """One of the backward's three launches (0 prep, 1 main, 2 finish); see include/fa.h."""
+    B, H, N, d = _shape(q)
+    st = load_library().fa_debug_bwd_phase(int(phase), _dtype_code(q), _ptr(q), _ptr(k), _ptr(v), _ptr(o),
+                                           _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace),
+                                           B, H, N, d, _scale(scale, d), int(bool(causal)), _ptr(block_mask),
+                                           _stream(stream))
+    _check(st, "fa_debug_bwd_phase")
 
 
 def fa_device_status(stream=None) -> int:

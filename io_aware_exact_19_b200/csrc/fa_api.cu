@@ -93,7 +93,8 @@ fa_status fwd_impl(fa_dtype dtype, const void* q, const void* k, const void* v, 
 
 fa_status bwd_impl(fa_dtype dtype, const void* q, const void* k, const void* v, const void* o, const float* lse,
                    const void* dout, void* dq, void* dk, void* dv, void* workspace, int B, int H, int N, int d,
-                   float scale, int causal, const uint8_t* mask, int32_t* trace, cudaStream_t stream) {
+                   float scale, int causal, const uint8_t* mask, int32_t* trace, cudaStream_t stream,
+                   int phases = 7) {
   fa_status s = check_common(dtype, B, H, N, d);
   if (s != FA_OK) return s;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) || !aligned16(dout) ||
@@ -120,6 +121,7 @@ fa_status bwd_impl(fa_dtype dtype, const void* q, const void* k, const void* v, 
   a.causal = causal ? 1 : 0;
   a.block_mask = mask;
   a.trace = trace;
+  a.phases = phases;
   a.status = status_word();
   if (!a.status) return FA_ERR_CUDA;
   return fa::launch_bwd(a, stream) == 0 ? FA_OK : FA_ERR_CUDA;
@@ -214,6 +216,19 @@ fa_status fa_debug_bwd_trace(fa_dtype dtype, const void* q, const void* k, const
   }
   return bwd_impl(dtype, q, k, v, o, lse, dout, dq, dk, dv, workspace, B, H, N, d, softmax_scale, causal,
                   block_mask, trace, stream);
+}
+
+fa_status fa_debug_bwd_phase(int phase, fa_dtype dtype, const void* q, const void* k, const void* v,
+                             const void* o, const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                             void* workspace, int B, int H, int N, int d, float softmax_scale, int causal,
+                             const uint8_t* block_mask, cudaStream_t stream) {
+  if (phase < 0 || phase > 2) return FA_ERR_INVALID_ARG;
+  if (block_mask) {
+    fa_status s = check_mask(N, d, block_mask);
+    if (s != FA_OK) return s;
+  }
+  return bwd_impl(dtype, q, k, v, o, lse, dout, dq, dk, dv, workspace, B, H, N, d, softmax_scale, causal,
+                  block_mask, nullptr, stream, 1 << phase);
 }
 
 fa_status fa_device_status(cudaStream_t stream) {

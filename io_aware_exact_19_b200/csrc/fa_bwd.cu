@@ -64,7 +64,7 @@ int launch_bwd_t(const AttnArgs& a, cudaStream_t stream) {
   if (!ok) return static_cast<int>(cudaErrorInvalidValue);
 
   // prep: D/8 threads per padded row.
-  {
+  if (a.phases & 1) {
     const long long threads = static_cast<long long>(BH) * p.Npad * (D / 8);
     const long long blocks = threads / 256;  // Npad*(D/8) is a multiple of 1024
     bwd::fa_bwd_prep_kernel<D, BF16><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p);
@@ -72,7 +72,7 @@ int launch_bwd_t(const AttnArgs& a, cudaStream_t stream) {
     if (e != cudaSuccess) return static_cast<int>(e);
   }
   // main
-  {
+  if (a.phases & 2) {
     auto kern = bwd::fa_bwd_main_kernel<D, BF16>;
     cudaError_t e = host::ensure_dynamic_smem(reinterpret_cast<const void*>(kern), C::kAlloc);
     if (e != cudaSuccess) return static_cast<int>(e);
@@ -82,7 +82,7 @@ int launch_bwd_t(const AttnArgs& a, cudaStream_t stream) {
     if (e != cudaSuccess) return static_cast<int>(e);
   }
   // finish
-  {
+  if (a.phases & 4) {
     const long long total4 = static_cast<long long>(BH) * a.N * D / 4;
     long long blocks = (total4 + 255) / 256;
     if (blocks > 148LL * 16) blocks = 148LL * 16;

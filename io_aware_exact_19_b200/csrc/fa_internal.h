@@ -25,6 +25,7 @@ struct AttnArgs {
   const uint8_t* block_mask;
   int32_t* trace;
   int* status;
+  int phases = 7;  // backward launches to run: bit 0 prep, bit 1 main, bit 2 finish
 };
 
 // Return 0 on success, a cudaError_t value otherwise.

@@ -27,6 +27,7 @@ from .attention import (  # noqa: F401
     forward,
     forward_rows,
     backward,
+    backward_rows,
     online_forward,
     causal_tile_set,
     forward_tile_lists,

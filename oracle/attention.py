@@ -156,6 +156,30 @@ def backward(q, k, v, do, scale: float, causal: bool = False, block_mask=None, t
     return (dQ, dK, dV, D) if return_d else (dQ, dK, dV)
 
 
+def backward_rows(q, k, v, do, scale: float, rows, causal: bool = False, block_mask=None, tile: int = TILE):
+    """Forward and gradients of L = Σ_{i ∈ rows} <dO_i, O_i> for one head [N, d].
+
+    The same definitions as :func:`forward` and :func:`backward`, applied to the
+    query rows ``rows`` only: S_rows = scale·Q_rows Kᵀ (masked), P_rows =
+    softmax(S_rows), O_rows = P_rows V, dV = P_rowsᵀ dO_rows, dP = dO_rows Vᵀ,
+    dS = P∘(dP − rowsum(P∘dP)), dQ_rows = scale·dS K, dK = scale·dSᵀ Q_rows.
+    With ``rows`` = all rows this is the full backward. Returns
+    (O_rows, lse_rows, dQ_rows, dK, dV).
+    """
+    q, k, v, do = (np.asarray(t, dtype=np.float64) for t in (q, k, v, do))
+    rows = np.asarray(rows)
+    allowed = _allowed_pairs(rows, np.arange(k.shape[0]), causal, block_mask, tile)
+    S = scale * (q[rows] @ k.T)
+    S = np.where(allowed, S, -np.inf)
+    P, lse = _softmax_rows(S)
+    O = P @ v
+    dV = P.T @ do[rows]
+    dP = do[rows] @ v.T
+    D = (P * dP).sum(axis=1, keepdims=True)
+    dS = P * (dP - D)
+    return O, lse, scale * (dS @ k), scale * (dS.T @ q[rows]), dV
+
+
 # --------------------------------------------------------------------------- online recurrence
 
 def online_forward(q, k, v, scale: float, bounds, causal: bool = False, block_mask=None,

@@ -102,3 +102,39 @@ def test_forward_rows_matches_full():
         Or, lser = oracle.forward_rows(q, k, v, 0.3, rows, causal=causal, block_mask=bm)
         np.testing.assert_allclose(Or, O[:, rows], rtol=0, atol=1e-13)
         np.testing.assert_allclose(lser, lse[:, rows], rtol=0, atol=1e-13)
+
+
+def test_backward_rows_equals_full_backward_on_all_rows():
+    r = np.random.default_rng(14)
+    q, k, v, do = (r.standard_normal((40, 6)) for _ in range(4))
+    for causal in (False, True):
+        O, lse = oracle.forward(q, k, v, 0.4, causal=causal)
+        dq, dk, dv = oracle.backward(q, k, v, do, 0.4, causal=causal)
+        o2, l2, dq2, dk2, dv2 = oracle.backward_rows(q, k, v, do, 0.4, np.arange(40), causal=causal)
+        for a, b in ((o2, O), (l2, lse), (dq2, dq), (dk2, dk), (dv2, dv)):
+            np.testing.assert_allclose(a, b, rtol=0, atol=1e-12)
+
+
+def test_backward_rows_finite_differences():
+    # L = sum over the chosen rows of <dO_i, O_i>; its gradient by central differences.
+    r = np.random.default_rng(15)
+    q, k, v, do = (r.standard_normal((9, 3)) for _ in range(4))
+    rows = np.array([1, 4, 8])
+    h = 1e-5
+    for causal in (False, True):
+        _, _, dq_r, dk, dv = oracle.backward_rows(q, k, v, do, 0.7, rows, causal=causal)
+        dq = np.zeros_like(q)
+        dq[rows] = dq_r
+
+        def L(q_, k_, v_):
+            O, _ = oracle.forward(q_, k_, v_, 0.7, causal=causal)
+            return float(np.sum(do[rows] * O[rows]))
+
+        for name, g in (("q", dq), ("k", dk), ("v", dv)):
+            R = r.standard_normal(q.shape)
+            args = {"q": q, "k": k, "v": v}
+            plus = {n: a + h * R if n == name else a for n, a in args.items()}
+            minus = {n: a - h * R if n == name else a for n, a in args.items()}
+            fd = (L(plus["q"], plus["k"], plus["v"]) - L(minus["q"], minus["k"], minus["v"])) / (2 * h)
+            an = float(np.sum(g * R))
+            assert abs(fd - an) <= 1e-7 * max(1.0, abs(an)), (name, causal, fd, an)
