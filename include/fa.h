@@ -85,6 +85,27 @@ fa_status fa_bwd(fa_dtype dtype, const void* q, const void* k, const void* v, co
                  float softmax_scale, int causal, cudaStream_t stream);
 
 /*
+ * fa_bwd without a workspace argument, for callers that cannot allocate device
+ * memory (a host application that owns every byte of device memory and gives
+ * this library no allocator, or a latency-critical loop where cudaMalloc is
+ * not allowed). The pages describe no such variant; it has no counterpart
+ * there. Arguments and results are those of fa_bwd (without block mask).
+ * Scratch: a fixed array of FA_BWD_NOALLOC_SCRATCH_BYTES bytes in the
+ * library's static device memory, held by every GPU that loads the library
+ * until the process exits. If fa_bwd_workspace_size(B, H, N, d) exceeds it the
+ * call returns FA_ERR_UNSUPPORTED and launches nothing. All calls on a device
+ * share that array: calls whose kernels may overlap on the GPU race and must be
+ * ordered by the caller. The dQ accumulator is re-zeroed by every call. The
+ * first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) and caches it; make that first call before any stream
+ * capture. Allocates nothing.
+ */
+#define FA_BWD_NOALLOC_SCRATCH_BYTES (32u << 20)
+fa_status fa_bwd_noalloc(fa_dtype dtype, const void* q, const void* k, const void* v, const void* o,
+                         const float* lse, const void* dout, void* dq, void* dk, void* dv, int B, int H, int N,
+                         int d, float softmax_scale, int causal, cudaStream_t stream);
+
+/*
  * Block-sparse forward ("FlashAttention" concept card, "Block-Sparse
  * FlashAttention": a fixed block mask whose zero blocks are skipped).
  * block_mask: DEVICE pointer to uint8 [N/128][N/128], row-major, shared by all

@@ -25,7 +25,7 @@ EXPORTED = (
     "fa_status_string", "fa_fwd", "fa_bwd", "fa_blocksparse_fwd", "fa_blocksparse_bwd",
     "fa_bwd_workspace_size", "fa_fwd_trace_size", "fa_bwd_trace_size", "fa_bwd_row_tile",
     "fa_debug_fwd_trace", "fa_debug_bwd_trace", "fa_debug_bwd_phase", "fa_device_status",
-    "fa_debug_timeout_probe",
+    "fa_debug_timeout_probe", "fa_bwd_noalloc",
 )
 
 
@@ -64,6 +64,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "fa_bwd_row_tile": ([i], i),
         "fa_device_status": ([vp], i),
         "fa_debug_timeout_probe": ([i, vp], i),
+        "fa_bwd_noalloc": (bwd_args[:10] + bwd_args[11:] + [vp], i),
     }
     for name, (argtypes, restype) in sigs.items():
         fn = getattr(lib, name)
@@ -157,6 +158,19 @@ def fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, causal: bool = False, s
                                _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace), B, H, N, d, _scale(scale, d),
                                int(bool(causal)), _stream(stream))
     _check(st, "fa_bwd")
+
+
+def fa_bwd_noalloc(q, k, v, o, lse, dout, dq, dk, dv, causal: bool = False, scale: float | None = None,
+                   stream=None) -> None:
+    """Backward without a workspace argument, for callers that cannot allocate device
+    memory: the scratch lives in a fixed static device array inside the library (see
+    include/fa.h for the size limit and the rule that overlapping calls race)."""
+    B, H, N, d = _shape(q)
+    _check_tensors(q, k, v, o, lse, dout, dq, dk, dv)
+    st = load_library().fa_bwd_noalloc(_dtype_code(q), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout),
+                                       _ptr(dq), _ptr(dk), _ptr(dv), B, H, N, d, _scale(scale, d),
+                                       int(bool(causal)), _stream(stream))
+    _check(st, "fa_bwd_noalloc")
 
 
 def fa_blocksparse_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, block_mask, causal: bool = False,

@@ -129,6 +129,8 @@ fa_status bwd_impl(fa_dtype dtype, const void* q, const void* k, const void* v, 
 
 }  // namespace
 
+int* fa::device_status_word() { return status_word(); }
+
 extern "C" {
 
 const char* fa_status_string(fa_status s) {

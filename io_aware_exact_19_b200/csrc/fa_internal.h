@@ -42,4 +42,7 @@ struct BwdWorkspace {
 BwdWorkspace bwd_workspace_layout(int B, int H, int N, int d);
 int bwd_row_tile(int d);
 
+// Device address of the per-device status word (nullptr on failure).
+int* device_status_word();
+
 }  // namespace fa
