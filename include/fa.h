@@ -19,7 +19,7 @@
  *   - lse_i = ln sum_j exp(scale * q_i . k_j) over the keys row i may see
  *     (natural log, in the units of the scaled scores).
  *   - d must be 64 or 128; N >= 1 (any value; ragged last tiles are handled);
- *     B, H >= 1.
+ *     B, H >= 1 and B*H <= 65535.
  *   - causal != 0 masks key j > query i (top-left aligned; the essay's
  *     section 3.1 causal mask P_ij = 0 for j > i).
  *   - The caller owns all memory. The library allocates no device memory; the

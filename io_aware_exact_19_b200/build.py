@@ -52,11 +52,32 @@ def _compile(src: str, verbose: bool) -> str:
     return obj
 
 
+# Kernels that re-split registers with setmaxnreg: the split assumes this many
+# registers per thread at launch. A smaller launch allocation would leave the
+# setmaxnreg.inc waiting forever, so the build refuses it.
+SETMAXNREG_LAUNCH_REGS = {"fa_fwd_kernel": 168}
+
+
+def _check_launch_registers(src: str) -> None:
+    import re
+    log = os.path.join(BUILD, os.path.splitext(src)[0] + ".log")
+    if not os.path.exists(log):
+        return
+    text = open(log).read()
+    entries = re.findall(r"Compiling entry function '(\S+)'.*?Used (\d+) registers", text, flags=re.S)
+    for mangled, regs in entries:
+        for name, want in SETMAXNREG_LAUNCH_REGS.items():
+            if name in mangled and int(regs) != want:
+                raise RuntimeError(f"{mangled}: {regs} registers at launch, the register split needs {want}")
+
+
 def build(verbose: bool = False) -> str:
     """Compile every CUDA source for sm_100a and link libfa.so; returns its path."""
     os.makedirs(BUILD, exist_ok=True)
     with ThreadPoolExecutor(max_workers=len(SOURCES)) as ex:
         objs = list(ex.map(lambda s: _compile(s, verbose), SOURCES))
+    for src in SOURCES:
+        _check_launch_registers(src)
     if not os.path.exists(LIB) or os.path.getmtime(LIB) < max(os.path.getmtime(o) for o in objs):
         tmp = LIB + ".tmp"
         cmd = [_nvcc(), *ARCH, "-shared", "-o", tmp, *objs]

@@ -76,7 +76,7 @@ int launch_bwd_t(const AttnArgs& a, cudaStream_t stream) {
     auto kern = bwd::fa_bwd_main_kernel<D, BF16>;
     cudaError_t e = host::ensure_dynamic_smem(reinterpret_cast<const void*>(kern), C::kAlloc);
     if (e != cudaSuccess) return static_cast<int>(e);
-    dim3 grid(BH, p.Tc);
+    dim3 grid(p.Tc, BH);
     kern<<<grid, bwd::kThreads, C::kAlloc, stream>>>(tq, tk, tv, tdo, tdq, p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return static_cast<int>(e);

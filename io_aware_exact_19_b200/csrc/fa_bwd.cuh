@@ -220,8 +220,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
-  const int bh = blockIdx.x;
-  const int j = blockIdx.y;  // key tile; small j has the most query tiles under a causal mask
+  // x runs over the key tiles of one head, so the CTAs that share a head's Q, dO
+  // and dQ accumulator in L2 run together; small j (most query tiles under a
+  // causal mask) goes first.
+  const int bh = blockIdx.y;
+  const int j = blockIdx.x;
   const int cta = bh * p.Tc + j;
 
   if (threadIdx.x == 0) {

@@ -42,6 +42,10 @@ constexpr int kBlockN = 128;  // keys per tile
 constexpr int kThreads = 384;
 constexpr int kMaxSparseTiles = 2048;
 constexpr float kRescaleThreshold = 8.0f;
+constexpr int kRegsLaunch = 168;  // 65536 / 384, rounded down to a multiple of 8
+constexpr int kRegsLow = 56;
+constexpr int kRegsHigh = 224;
+static_assert(128 * kRegsLow + 256 * kRegsHigh <= kThreads * kRegsLaunch, "register split exceeds the launch allocation");
 
 struct Params {
   void* o;
@@ -118,7 +122,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
-  // Heaviest query tiles first: blocks are dispatched x-fastest, x runs over heads.
+  // Blocks are dispatched x-fastest and x runs over heads, so every head's
+  // heaviest query-tile pair (the last one, under a causal mask) starts first
+  // and the light pairs fill the tail.
   const int bh = blockIdx.x;
   const int pair = p.n_pairs - 1 - static_cast<int>(blockIdx.y);
   const int q0 = 2 * pair;
@@ -197,7 +203,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sV = smem + L::kVOff;
   constexpr int kChunkBytes = 128 * 128;  // one 128-row x 64-column swizzled chunk
 
-  if (warp == 0) {
+  // Register split: warpgroup 0 (producer, MMA, list builder, idle) needs few
+  // registers; the two softmax warpgroups hold a 128-column row of S each.
+  // 128 x kRegsLow + 256 x kRegsHigh <= 384 x 168, the launch allocation. Each
+  // setmaxnreg sits inside the branch of the roles it serves, so the compiler
+  // sees the budget of every code path.
+  if (warp < 4) {
+   reg_dealloc<kRegsLow>();
+   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0 && tl.len > 0) {
       prefetch_tmap(&tmap_q);
@@ -299,7 +312,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (started[q]) umma_commit(bar_o_full(q));
       }
     }
-  } else if (warp >= 4) {
+  }
+  } else {
+    reg_alloc<kRegsHigh>();
     // ------------------------------------------------------------ softmax
     const int q = (warp - 4) / 4;  // query tile within the pair
     const int wq = warp % 4;       // TMEM lane quarter
