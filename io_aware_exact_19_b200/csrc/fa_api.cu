@@ -1,6 +1,6 @@
 // C ABI of the attention library: argument checks, the device status word and
 // dispatch to the launchers. Declarations and contracts are in include/fa.h.
-#include "../../include/fa.h"
+#include "fa.h"
 
 #include <cuda_runtime.h>
 

@@ -436,8 +436,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!(ok = mbar_wait_warp(bar_qdo_full(s), (n >> 1) & 1, ctx))) break;
       tc_fence_after();
       const bool diag = p.causal && (j * kBlockN + kBlockN - 1 > i * BR);
-      const float* L2 = sL + s * BR;
-      const float* DD = sDv + s * BR;
+      const uint32_t aL = smem_u32(sL + s * BR);
+      const uint32_t aD = smem_u32(sDv + s * BR);
 #pragma unroll
       for (int cc = 0; cc < BR / 64; ++cc) {
         const int qo = half * (BR / 2) + cc * 32;  // first query column of this chunk
@@ -445,16 +445,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(tmem + lane_off + C::kColS + qo, sr);
         tmem_ld32(tmem + lane_off + C::kColDP + qo, dr);
         tmem_ld_wait();
+        // Columns x < lim are masked (causal: key > query; or the key row is past N).
+        int lim = 0;
+        if (!key_valid) lim = 32;
+        else if (diag) lim = min(32, max(0, key - (i * BR + qo)));
         uint32_t pk[16], dk[16];
 #pragma unroll
-        for (int x = 0; x < 32; x += 2) {
-          float p0 = ex2(fmaf(__uint_as_float(sr[x]), sl2, -L2[qo + x]));
-          float p1 = ex2(fmaf(__uint_as_float(sr[x + 1]), sl2, -L2[qo + x + 1]));
-          if (!key_valid || (diag && key > i * BR + qo + x)) p0 = 0.0f;
-          if (!key_valid || (diag && key > i * BR + qo + x + 1)) p1 = 0.0f;
+        for (int x = 0; x < 32; x += 4) {
+          const float4 l4 = lds128(aL + (qo + x) * 4);
+          const float4 d4 = lds128(aD + (qo + x) * 4);
+          float p0 = ex2(fmaf(__uint_as_float(sr[x]), sl2, -l4.x));
+          float p1 = ex2(fmaf(__uint_as_float(sr[x + 1]), sl2, -l4.y));
+          float p2 = ex2(fmaf(__uint_as_float(sr[x + 2]), sl2, -l4.z));
+          float p3 = ex2(fmaf(__uint_as_float(sr[x + 3]), sl2, -l4.w));
+          if (lim > 0) {
+            if (x < lim) p0 = 0.0f;
+            if (x + 1 < lim) p1 = 0.0f;
+            if (x + 2 < lim) p2 = 0.0f;
+            if (x + 3 < lim) p3 = 0.0f;
+          }
           pk[x / 2] = pack2<BF16>(p0, p1);
-          dk[x / 2] = pack2<BF16>(p0 * (__uint_as_float(dr[x]) - DD[qo + x]),
-                                  p1 * (__uint_as_float(dr[x + 1]) - DD[qo + x + 1]));
+          pk[x / 2 + 1] = pack2<BF16>(p2, p3);
+          dk[x / 2] = pack2<BF16>(p0 * (__uint_as_float(dr[x]) - d4.x), p1 * (__uint_as_float(dr[x + 1]) - d4.y));
+          dk[x / 2 + 1] = pack2<BF16>(p2 * (__uint_as_float(dr[x + 2]) - d4.z), p3 * (__uint_as_float(dr[x + 3]) - d4.w));
         }
         if (cc == 0 && n > 0) {
           // P^T of the previous tile must have been consumed by its dV MMA.
@@ -465,13 +478,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!(ok = mbar_wait_warp(bar_ds_empty(b), ((n - 2) >> 1) & 1, ctx))) break;
         }
         // dS^T row r, query columns qo..qo+31 -> four 16-byte pieces of the swizzled row.
-        uint8_t* rowp = sDS + b * C::kDSBytes + (qo / 64) * (kBlockN * 128) + r * 128;
-        const int p0 = (qo % 64) / 8;
+        const uint32_t rowa = smem_u32(sDS + b * C::kDSBytes + (qo / 64) * (kBlockN * 128) + r * 128);
+        const int p0i = (qo % 64) / 8;
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
-          const int phys = (p0 + t) ^ (r & 7);
-          *reinterpret_cast<uint4*>(rowp + phys * 16) =
-              make_uint4(dk[4 * t], dk[4 * t + 1], dk[4 * t + 2], dk[4 * t + 3]);
+          const int phys = (p0i + t) ^ (r & 7);
+          sts128(rowa + phys * 16, dk[4 * t], dk[4 * t + 1], dk[4 * t + 2], dk[4 * t + 3]);
         }
       }
       if (!ok) break;
@@ -535,20 +547,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       if constexpr (D == 64) {
         // lane = query row. Staging is two [128 rows][32] fp32 boxes in the TMA
         // 128-byte swizzle: 16-byte piece x of row t sits at piece x ^ (t & 7).
-        uint8_t* row0 = reinterpret_cast<uint8_t*>(sDQ) + t * 128;
-        uint8_t* row1 = row0 + 128 * 128;
+        const uint32_t row0 = smem_u32(sDQ) + t * 128;
+        const uint32_t row1 = row0 + 128 * 128;
 #pragma unroll
         for (int x = 0; x < 8; ++x) {
           const int phys = (x ^ (t & 7)) * 16;
-          *reinterpret_cast<uint4*>(row0 + phys) = make_uint4(v0[4 * x], v0[4 * x + 1], v0[4 * x + 2], v0[4 * x + 3]);
-          *reinterpret_cast<uint4*>(row1 + phys) = make_uint4(v1[4 * x], v1[4 * x + 1], v1[4 * x + 2], v1[4 * x + 3]);
+          sts128(row0 + phys, v0[4 * x], v0[4 * x + 1], v0[4 * x + 2], v0[4 * x + 3]);
+          sts128(row1 + phys, v1[4 * x], v1[4 * x + 1], v1[4 * x + 2], v1[4 * x + 3]);
         }
       } else {
         // lane = d index; columns are the 64 query rows; staging is [64 rows][128] fp32.
+        const uint32_t base = smem_u32(sDQ) + t * 4;
 #pragma unroll
         for (int x = 0; x < 32; ++x) {
-          sDQ[x * D + t] = __uint_as_float(v0[x]);
-          sDQ[(x + 32) * D + t] = __uint_as_float(v1[x]);
+          sts32(base + x * D * 4, v0[x]);
+          sts32(base + (x + 32) * D * 4, v1[x]);
         }
       }
       fence_proxy_async_smem();

@@ -21,7 +21,7 @@
 //   * The first call on a device looks up the array's device address with
 //     cudaGetSymbolAddress (a host-side stand-in name is not a device address)
 //     and caches it; that first call should come before any stream capture.
-#include "../../include/fa.h"
+#include "fa.h"
 
 #include <cuda_runtime.h>
 
