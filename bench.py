@@ -2,7 +2,7 @@
 """Benchmark of the exact fused attention path on B200.
 
 One step = one pass of the whole hot path over one batch of synthetic input:
-the forward (fa_fwd) and the backward (its three launches: prep, main, finish)
+the forward (fa_fwd) and the backward (its two launches: prep and main)
 of exact attention on the long-context causal workload B=4, H=16, N=4096,
 d=128, bf16, Q/K/V/dO iid N(0, 1).
 
@@ -296,9 +296,6 @@ def run_gpu(args, w, rank, world, local_rank):
         bwd_phase(1)
         if ev is not None:
             ev[3].record(stream)
-        bwd_phase(2)
-        if ev is not None:
-            ev[4].record(stream)
 
     for _ in range(max(args.warmup, 3)):
         step()
@@ -310,7 +307,7 @@ def run_gpu(args, w, rank, world, local_rank):
     gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
     sampler = ClockSampler(gpu_id, os.path.join(tempfile.gettempdir(), f"fa_bench_clocks_rank{rank}_{os.getpid()}.csv"))
     time.sleep(0.3)
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -326,11 +323,10 @@ def run_gpu(args, w, rank, world, local_rank):
     clocks = sampler.summary(t_wall0, t_wall1)
     status = fa.fa_device_status()
 
-    ms_total = events[0][0].elapsed_time(events[-1][4])
+    ms_total = events[0][0].elapsed_time(events[-1][3])
     fwd_ms = [e[0].elapsed_time(e[1]) for e in events]
     prep_ms = [e[1].elapsed_time(e[2]) for e in events]
     main_ms = [e[2].elapsed_time(e[3]) for e in events]
-    fin_ms = [e[3].elapsed_time(e[4]) for e in events]
     if world > 1:
         t = torch.tensor([ms_total, sum(main_ms), sum(fwd_ms)], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -344,9 +340,9 @@ def run_gpu(args, w, rank, world, local_rank):
     main_avg = main_sum / args.steps
     fwd_avg = fwd_sum / args.steps
     achieved = f_bwd / (main_avg * 1e-3) / 1e12
-    bwd_all = statistics.mean(p + m + f for p, m, f in zip(prep_ms, main_ms, fin_ms))
+    bwd_all = statistics.mean(p + m for p, m in zip(prep_ms, main_ms))
     prep_avg = statistics.mean(prep_ms)
-    prep_bytes = B * H * N * d * (2 + 2 + 4) + B * H * N * 4 * 3  # read O, dO; zero dQacc; lse in, D and lse2 out
+    prep_bytes = B * H * N * d * (2 + 2) + B * H * N * 4 * 3  # read O, dO and lse; write D and lse2
 
     # ---- end to end through the C ABI: pinned host inputs in, results back to pinned host memory
     pin = {n: t.pin_memory() for n, t in host.items()}
@@ -412,7 +408,7 @@ def run_gpu(args, w, rank, world, local_rank):
             "fwd_frac_of_measured_peak": f_fwd / (fwd_avg * 1e-3) / 1e12 / peaks["bf16"],
             "bwd_ms": bwd_all, "bwd_tflops": f_bwd / (bwd_all * 1e-3) / 1e12,
             "bwd_frac_of_measured_peak": f_bwd / (bwd_all * 1e-3) / 1e12 / peaks["bf16"],
-            "bwd_main_ms": main_avg, "bwd_prep_ms": prep_avg, "bwd_finish_ms": statistics.mean(fin_ms),
+            "bwd_main_ms": main_avg, "bwd_prep_ms": prep_avg,
             "bwd_prep_gbs": prep_bytes / (prep_avg * 1e-3) / 1e9,
             "vendor_peak_tflops": 2250.0,
             "fwd_frac_of_vendor_peak": f_fwd / (fwd_avg * 1e-3) / 1e12 / 2250.0,
@@ -420,7 +416,7 @@ def run_gpu(args, w, rank, world, local_rank):
         },
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": e2e_steps},
-        "gpu_launches": 4 * args.steps,
+        "gpu_launches": 3 * args.steps,
         "clocks": clocks,
         "device_status": int(status),
         "wall_s_timed_region": t_wall1 - t_wall0,

@@ -66,9 +66,8 @@ fa_status fa_fwd(fa_dtype dtype, const void* q, const void* k, const void* v, vo
 
 /*
  * Bytes of device workspace fa_bwd / fa_blocksparse_bwd need for these sizes:
- * an fp32 dQ accumulator [B,H,N,d] plus two fp32 row vectors [B,H,ceil(N/128)*128]
- * (D = rowsum(dO o O) and a padded copy of lse). Linear in N. Returns 0 for
- * invalid sizes.
+ * two fp32 row vectors [B,H,ceil(N/128)*128] (D = rowsum(dO o O) and lse in
+ * log2 units). Linear in N. Returns 0 for invalid sizes.
  */
 size_t fa_bwd_workspace_size(int B, int H, int N, int d);
 
@@ -125,14 +124,18 @@ fa_status fa_blocksparse_bwd(fa_dtype dtype, const void* q, const void* k, const
 
 /*
  * Debug: the forward / backward with a record of the tiles each CTA loaded.
- * trace: DEVICE int32 buffer of fa_*_trace_size() entries. For CTA c the
- * record starts at c * (stride) where stride = T_kv + 1 for the forward
- * (T_kv = ceil(N/128) key tiles) and T_q + 1 for the backward (T_q = query
- * tiles of the backward's row step, fa_bwd_row_tile(d) rows each); entry 0 is
- * the count and entries 1.. are (tile index) | (flags << 16). Forward CTA c
- * covers query tiles 2p and 2p+1 (p = c % n_pairs) of head c / n_pairs, flags
- * bit q = tile is used by query tile 2p+q; backward CTA c covers key tile
- * c % T_kv of head c / T_kv, flags = 1.
+ * trace: DEVICE int32 buffer of fa_*_trace_size() entries; each record is a
+ * count followed by entries (tile index) | (flags << 16).
+ * Forward: T_kv = ceil(N/128) key tiles; CTA c covers query tiles 2p and 2p+1
+ * (p = c % n_pairs, n_pairs = ceil(T_kv/2)) of head c / n_pairs; its record of
+ * T_kv + 1 entries starts at c * (T_kv + 1); flags bit q = the key tile is used
+ * by query tile 2p+q.
+ * Backward: key-stationary CTA (head h, key tile j) lists the query tiles of
+ * fa_bwd_row_tile(d) rows it visits, record of T_q + 1 entries at
+ * (h * T_kv + j) * (T_q + 1), T_q = ceil(N / fa_bwd_row_tile(d)); after all of
+ * those, query-stationary CTA (head h, 128-row query tile i) lists the key
+ * tiles it visits, record of T_kv + 1 entries at
+ * B*H*T_kv*(T_q + 1) + (h * T_kv + i) * (T_kv + 1). Backward flags = 1.
  */
 size_t fa_fwd_trace_size(int B, int H, int N);
 size_t fa_bwd_trace_size(int B, int H, int N, int d);
@@ -146,12 +149,11 @@ fa_status fa_debug_bwd_trace(fa_dtype dtype, const void* q, const void* k, const
                              const uint8_t* block_mask, int32_t* trace, cudaStream_t stream);
 
 /*
- * Debug: one of the three launches fa_bwd makes, selected by `phase`:
- * 0 = prep (D = rowsum(dO o O), lse in log2 units, zero the dQ accumulator),
- * 1 = main (recompute P, accumulate dK, dV in TMEM and dQ in the workspace),
- * 2 = finish (dQ = scale * accumulator, cast). Running phases 0, 1, 2 in order
- * on one stream with the same arguments is exactly fa_bwd. Used to time the
- * main kernel on its own.
+ * Debug: one of the two launches fa_bwd makes, selected by `phase`:
+ * 0 = prep (D = rowsum(dO o O) and lse in log2 units, into the workspace),
+ * 1 = main (recompute P; dK, dV by key tile and dQ by query tile, all
+ * accumulated in TMEM). Running phases 0 and 1 in order on one stream with the
+ * same arguments is exactly fa_bwd. Used to time the main kernel on its own.
  */
 fa_status fa_debug_bwd_phase(int phase, fa_dtype dtype, const void* q, const void* k, const void* v,
                              const void* o, const float* lse, const void* dout, void* dq, void* dk, void* dv,

@@ -55,7 +55,7 @@ def _compile(src: str, verbose: bool) -> str:
 # Kernels that re-split registers with setmaxnreg: the split assumes this many
 # registers per thread at launch. A smaller launch allocation would leave the
 # setmaxnreg.inc waiting forever, so the build refuses it.
-SETMAXNREG_LAUNCH_REGS = {"fa_fwd_kernel": 168}
+SETMAXNREG_LAUNCH_REGS = {"fa_fwd_kernel": 168, "fa_bwd_main_kernel": 168}
 
 
 def _check_launch_registers(src: str) -> None:

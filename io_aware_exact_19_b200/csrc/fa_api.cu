@@ -191,10 +191,10 @@ size_t fa_fwd_trace_size(int B, int H, int N) {
 
 size_t fa_bwd_trace_size(int B, int H, int N, int d) {
   if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 128)) return 0;
-  const size_t tkv = (static_cast<size_t>(N) + 127) / 128;
+  const size_t t = (static_cast<size_t>(N) + 127) / 128;
   const size_t br = static_cast<size_t>(fa::bwd_row_tile(d));
   const size_t tq = (static_cast<size_t>(N) + br - 1) / br;
-  return static_cast<size_t>(B) * H * tkv * (tq + 1);
+  return static_cast<size_t>(B) * H * t * ((tq + 1) + (t + 1));
 }
 
 fa_status fa_debug_fwd_trace(fa_dtype dtype, const void* q, const void* k, const void* v, void* o, float* lse,
@@ -225,7 +225,7 @@ fa_status fa_debug_bwd_phase(int phase, fa_dtype dtype, const void* q, const voi
                              const void* o, const float* lse, const void* dout, void* dq, void* dk, void* dv,
                              void* workspace, int B, int H, int N, int d, float softmax_scale, int causal,
                              const uint8_t* block_mask, cudaStream_t stream) {
-  if (phase < 0 || phase > 2) return FA_ERR_INVALID_ARG;
+  if (phase < 0 || phase > 1) return FA_ERR_INVALID_ARG;
   if (block_mask) {
     fa_status s = check_mask(N, d, block_mask);
     if (s != FA_OK) return s;

@@ -1,21 +1,20 @@
-// Host launchers of the backward kernels: prep (D, lse2, zero dQacc), the fused
-// main kernel, and finish (dQacc -> dQ).
+// Host launchers of the backward: prep (D and lse in log2 units) and the main
+// kernel (key-stationary dK/dV CTAs and query-stationary dQ CTAs in one grid).
 #include "fa_bwd.cuh"
 #include "fa_internal.h"
 #include "tma_host.h"
 
 namespace fa {
 
-int bwd_row_tile(int d) { return d == 128 ? bwd::Cfg<128>::BR : bwd::Cfg<64>::BR; }
+int bwd_row_tile(int) { return bwd::kBR; }
 
-BwdWorkspace bwd_workspace_layout(int B, int H, int N, int d) {
+BwdWorkspace bwd_workspace_layout(int B, int H, int N, int) {
   BwdWorkspace w{};
   const size_t bh = static_cast<size_t>(B) * H;
   const size_t npad = (static_cast<size_t>(N) + 127) / 128 * 128;
   auto up = [](size_t x) { return (x + 255) / 256 * 256; };
-  w.dq_acc = 0;
-  w.delta = up(bh * N * d * 4);
-  w.lse2 = w.delta + up(bh * npad * 4);
+  w.delta = 0;
+  w.lse2 = up(bh * npad * 4);
   w.total = w.lse2 + up(bh * npad * 4);
   return w;
 }
@@ -37,7 +36,6 @@ int launch_bwd_t(const AttnArgs& a, cudaStream_t stream) {
   p.dq = a.dq;
   p.dk = a.dk;
   p.dv = a.dv;
-  p.dq_acc = reinterpret_cast<float*>(base + ws.dq_acc);
   p.delta = reinterpret_cast<float*>(base + ws.delta);
   p.lse2 = reinterpret_cast<float*>(base + ws.lse2);
   p.block_mask = a.block_mask;
@@ -46,22 +44,11 @@ int launch_bwd_t(const AttnArgs& a, cudaStream_t stream) {
   p.N = a.N;
   p.Npad = (a.N + 127) / 128 * 128;
   p.BH = BH;
-  p.Tq = (a.N + C::BR - 1) / C::BR;
-  p.Tc = (a.N + bwd::kBlockN - 1) / bwd::kBlockN;
+  p.T = (a.N + 127) / 128;
+  p.Tq1 = (a.N + bwd::kBR - 1) / bwd::kBR;
   p.causal = a.causal;
   p.scale = a.scale;
   p.scale_log2 = a.scale * 1.4426950408889634f;
-
-  CUtensorMap tq, tk, tv, tdo, tdq;
-  bool ok = host::make_map_3d(&tq, dt, 2, a.q, D, a.N, BH, 64, C::BR, CU_TENSOR_MAP_SWIZZLE_128B) &&
-            host::make_map_3d(&tdo, dt, 2, a.dout, D, a.N, BH, 64, C::BR, CU_TENSOR_MAP_SWIZZLE_128B) &&
-            host::make_map_3d(&tk, dt, 2, a.k, D, a.N, BH, 64, bwd::kBlockN, CU_TENSOR_MAP_SWIZZLE_128B) &&
-            host::make_map_3d(&tv, dt, 2, a.v, D, a.N, BH, 64, bwd::kBlockN, CU_TENSOR_MAP_SWIZZLE_128B) &&
-            (D == 64 ? host::make_map_3d(&tdq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, p.dq_acc, D, a.N, BH, 32, C::BR,
-                                         CU_TENSOR_MAP_SWIZZLE_128B)
-                     : host::make_map_3d(&tdq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, p.dq_acc, D, a.N, BH, D, C::BR,
-                                         CU_TENSOR_MAP_SWIZZLE_NONE));
-  if (!ok) return static_cast<int>(cudaErrorInvalidValue);
 
   // prep: D/8 threads per padded row.
   if (a.phases & 1) {
@@ -73,21 +60,20 @@ int launch_bwd_t(const AttnArgs& a, cudaStream_t stream) {
   }
   // main
   if (a.phases & 2) {
+    CUtensorMap tq, tk, tv, tdo;
+    // Q and dO are read in 64-row tiles by key-stationary CTAs and in 128-row
+    // tiles by query-stationary CTAs: two 64-row boxes make one 128-row tile.
+    bool ok = host::make_map_3d(&tq, dt, 2, a.q, D, a.N, BH, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B) &&
+              host::make_map_3d(&tdo, dt, 2, a.dout, D, a.N, BH, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B) &&
+              host::make_map_3d(&tk, dt, 2, a.k, D, a.N, BH, 64, bwd::kBlockN, CU_TENSOR_MAP_SWIZZLE_128B) &&
+              host::make_map_3d(&tv, dt, 2, a.v, D, a.N, BH, 64, bwd::kBlockN, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (!ok) return static_cast<int>(cudaErrorInvalidValue);
     auto kern = bwd::fa_bwd_main_kernel<D, BF16>;
     cudaError_t e = host::ensure_dynamic_smem(reinterpret_cast<const void*>(kern), C::kAlloc);
     if (e != cudaSuccess) return static_cast<int>(e);
-    dim3 grid(p.Tc, BH);
-    kern<<<grid, bwd::kThreads, C::kAlloc, stream>>>(tq, tk, tv, tdo, tdq, p);
+    dim3 grid(BH, 2 * p.T);
+    kern<<<grid, bwd::kThreads, C::kAlloc, stream>>>(tq, tk, tv, tdo, p);
     e = cudaGetLastError();
-    if (e != cudaSuccess) return static_cast<int>(e);
-  }
-  // finish
-  if (a.phases & 4) {
-    const long long total4 = static_cast<long long>(BH) * a.N * D / 4;
-    long long blocks = (total4 + 255) / 256;
-    if (blocks > 148LL * 16) blocks = 148LL * 16;
-    bwd::fa_bwd_finish_kernel<D, BF16><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p);
-    cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return static_cast<int>(e);
   }
   return 0;

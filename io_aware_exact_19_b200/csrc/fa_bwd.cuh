@@ -2,36 +2,40 @@
 // instead of storing it ("FlashAttention" concept card, lukebest.github.io,
 // "反向：重算而非存储"; interview explainer mstx.cn/posts/485, section 3.3).
 //
-// Three kernels:
-//   prep     D_i = rowsum(dO_i o O_i), lse2_i = lse_i * log2(e) (+inf on padding
-//            rows and rows without keys, so their P is 0), dQacc = 0.
-//   main     one CTA per 128-key tile j of one (batch, head); it loops over the
-//            query tiles i that reach j (B_r rows each) and, per tile:
-//              S^T  = K_j Q_i^T           P^T = exp2(S^T * scale*log2e - lse2_i)
-//              dP^T = V_j dO_i^T          dS^T = P^T o (dP^T - D_i)
-//              dV_j += P^T dO_i           dK_j += dS^T Q_i
-//              dQ_i (+)= dS K_j           added to fp32 dQacc by a TMA reduce
-//            then writes dV_j and scale * dK_j.
-//   finish   dQ = scale * dQacc in the input dtype.
+// Two kernels:
+//   prep   D_i = rowsum(dO_i o O_i) and lse2_i = lse_i * log2(e) (+inf on padding
+//          rows and rows without keys, so their P is 0).
+//   main   one launch with two kinds of CTA, interleaved heaviest first:
+//     key-stationary (one 128-key tile j of one head; dK_j and dV_j stay in TMEM)
+//       for each 64-row query tile i that reaches j:
+//         S^T  = K_j Q_i^T,  dP^T = V_j dO_i^T                (shared-memory operands)
+//         P^T  = exp2(S^T * scale*log2e - lse2_i),  dS^T = P^T o (dP^T - D_i)
+//         dV_j += P^T dO_i,  dK_j += dS^T Q_i                 (P^T, dS^T read from TMEM)
+//       then dV_j and scale * dK_j are written once.
+//     query-stationary (one 128-row query tile i of one head; dQ_i stays in TMEM)
+//       for each 128-key tile j that i reaches:
+//         S = Q_i K_j^T,  dP = dO_i V_j^T,  P = exp2(S*scale*log2e - lse2),  dS = P o (dP - D)
+//         dQ_i += dS K_j                                        (dS read from TMEM)
+//       then scale * dQ_i is written once.
+// dQ is thus produced without atomics or an fp32 accumulator in global memory,
+// at the price of recomputing S and dP once more (7 MMAs per 128x128 block of
+// scores instead of 5). The P^T, dS^T and dS operands live in TMEM, so no MMA
+// reads more than one operand tile from shared memory per 16-wide K step, which
+// keeps the shared-memory port (128 B/clock) from throttling the tensor core.
 //
-// Main-kernel roles (512 threads, one CTA per SM):
-//   warp 0      TMA producer: K_j, V_j once; Q_i, dO_i, lse2_i, D_i into a 2-stage ring
-//   warp 1      MMA issuer and TMEM owner
-//   warp 2      builds the query-tile list of a block-sparse CTA
-//   warps 4-7   elementwise, query columns [0, B_r/2)   (thread = key row)
-//   warps 8-11  elementwise, query columns [B_r/2, B_r)
-//   warps 12-15 dQ drain: TMEM -> shared -> cp.reduce.async.bulk.tensor (add) into dQacc
+// Roles (384 threads, one CTA per SM, both kinds):
+//   warp 0      TMA producer          warp 1      MMA issuer, TMEM owner
+//   warp 2      counts the tiles of a block-sparse CTA
+//   warps 4-7   elementwise, first half of the columns (thread = TMEM lane = row)
+//   warps 8-11  elementwise, second half of the columns
 //
-// Tile shapes: B_c = 128 keys per CTA. B_r = 128 query rows for d = 64 and 64
-// for d = 128, so that the five accumulators fit the 512 TMEM columns:
-//   d=64:  S^T 0..127, dP^T 128..255, P^T 256..319, dV 320..383, dK 384..447, dQ 448..511
-//   d=128: S^T 0..63,  dP^T 64..127,  P^T 128..159, dV 160..287, dK 288..415, dQ^T 416..479
-// For d=128 dQ is produced transposed (dQ^T = K_j^T dS^T, M = d = 128), which
-// keeps every MMA at M = 128.
-//
-// MMA order per tile n (all tcgen05 MMAs of a CTA execute in issue order):
-//   wait elementwise(n) -> S^T, dP^T of n+1 -> dV(n), dK(n) -> dQ(n)
-// so the elementwise work of tile n+1 overlaps dV, dK, dQ of tile n.
+// TMEM (512 columns):
+//   key-stationary:   buffer b in {0,1}: S^T at 128b (64 columns), dP^T at 128b+64;
+//                     warpgroup h writes its P^T (16 columns) over its own S^T
+//                     columns at 128b+32h and its dS^T over dP^T at 128b+64+32h;
+//                     dV at 256, dK at 256+d.
+//   query-stationary: S buffers at 0 and 128, dP at 256 (warpgroup h writes its
+//                     dS, 32 columns, at 256+64h), dQ at 384.
 #pragma once
 
 #include <cuda_fp16.h>
@@ -43,41 +47,84 @@ namespace bwd {
 
 using namespace fa::sm100;
 
-constexpr int kBlockN = 128;  // keys per CTA
-constexpr int kThreads = 512;
-constexpr int kMaxSparseTiles = 4096;
+constexpr int kThreads = 384;
+constexpr int kBlockN = 128;  // keys per key-stationary CTA and per query-stationary step
+constexpr int kBlockQ = 128;  // queries per query-stationary CTA
+constexpr int kBR = 64;       // queries per key-stationary step
+constexpr int kRegsLaunch = 168;
+constexpr int kRegsLow = 88;
+constexpr int kRegsHigh = 208;
+static_assert(128 * kRegsLow + 256 * kRegsHigh <= kThreads * kRegsLaunch,
+              "register split exceeds the launch allocation");
 constexpr float kLog2e = 1.4426950408889634f;
 
 template <int D>
 struct Cfg {
-  static constexpr int BR = (D == 64) ? 128 : 64;  // query rows per step
-  static constexpr int kColS = 0;
-  static constexpr int kColDP = BR;
-  static constexpr int kColP = 2 * BR;
-  static constexpr int kColDV = 2 * BR + BR / 2;
-  static constexpr int kColDK = kColDV + D;
-  static constexpr int kColDQ = kColDK + D;
-  static_assert(kColDQ + (D == 64 ? D : BR) <= 512, "TMEM budget");
-
-  static constexpr int kKVBytes = kBlockN * D * 2;  // K_j or V_j
-  static constexpr int kQBytes = BR * D * 2;        // Q_i or dO_i
-  static constexpr int kDSBytes = kBlockN * BR * 2; // dS^T (bf16/fp16)
-  static constexpr int kStageVec = BR * 4;          // lse2 or D of one tile
-  static constexpr int kOffK = 0;
-  static constexpr int kOffV = kOffK + kKVBytes;
-  static constexpr int kOffQ = kOffV + kKVBytes;             // [2 stages]
-  static constexpr int kOffDO = kOffQ + 2 * kQBytes;         // [2 stages]
-  static constexpr int kOffDS = kOffDO + 2 * kQBytes;        // [2 buffers]
-  static constexpr int kOffDQ = kOffDS + 2 * kDSBytes;       // fp32 staging BR x D
-  static constexpr int kOffL = kOffDQ + BR * D * 4;          // lse2 [2][BR]
-  static constexpr int kOffDv = kOffL + 2 * kStageVec;       // D [2][BR]
-  static constexpr int kOffBar = kOffDv + 2 * kStageVec;
-  // bars: kv_full, qdo_full[2], qdo_empty[2], s_full, p_full, p_free, ds_empty[2], dq_full, dq_empty, all_done
-  static constexpr int kNumBars = 13;
-  static constexpr int kOffMisc = kOffBar + 8 * kNumBars;    // tmem slot, abort flag, list length
-  static constexpr int kOffList = kOffMisc + 16;
-  static constexpr int kBytes = kOffList + 4 * kMaxSparseTiles;
+  static constexpr int kKVBytes = kBlockN * D * 2;  // 128-row K or V tile
+  static constexpr int kQ1Bytes = kBR * D * 2;      // 64-row Q or dO tile
+  static constexpr int kQ2Bytes = kBlockQ * D * 2;  // 128-row Q or dO tile
+  // key-stationary layout: K_j, V_j, then a ring of (Q_i, dO_i, lse2_i, D_i)
+  static constexpr int kS1 = 4;
+  static constexpr int k1K = 0;
+  static constexpr int k1V = k1K + kKVBytes;
+  static constexpr int k1Q = k1V + kKVBytes;
+  static constexpr int k1DO = k1Q + kS1 * kQ1Bytes;
+  static constexpr int k1L = k1DO + kS1 * kQ1Bytes;
+  static constexpr int k1Dv = k1L + kS1 * kBR * 4;
+  static constexpr int k1End = k1Dv + kS1 * kBR * 4;
+  // query-stationary layout: Q_i, dO_i, then rings of K_j and V_j
+  static constexpr int kSK = 3;
+  static constexpr int kSV = (D == 128) ? 2 : 3;
+  static constexpr int k2Q = 0;
+  static constexpr int k2DO = k2Q + kQ2Bytes;
+  static constexpr int k2K = k2DO + kQ2Bytes;
+  static constexpr int k2V = k2K + kSK * kKVBytes;
+  static constexpr int k2End = k2V + kSV * kKVBytes;
+  static constexpr int kOffBar = ((k1End > k2End ? k1End : k2End) + 15) / 16 * 16;
+  static constexpr int kNumBars = 18;
+  static constexpr int kOffMisc = kOffBar + 8 * kNumBars;  // tmem slot, abort flag, list length
+  static constexpr int kBytes = kOffMisc + 16;
   static constexpr int kAlloc = kBytes + 1024;
+  static_assert(kAlloc <= 232448, "shared memory budget");
+  static_assert(256 + 2 * D <= 512 && 384 + D <= 512, "TMEM budget");
+};
+
+// Barrier slots of the two CTA kinds (they share the same shared-memory words).
+struct KeyBars {
+  static constexpr int kv_full = 0, qdo_full = 1, qdo_empty = 5, s_full = 9, p_full = 11, all_done = 13;
+};
+struct QueryBars {
+  static constexpr int q_full = 0, k_full = 1, k_empty = 4, v_full = 7, v_empty = 10, s_full = 13, dp_full = 15,
+                       ds_full = 16, all_done = 17;
+};
+
+// Walks the tiles one CTA visits, in ascending order. Dense and causal ranges
+// are arithmetic; a block mask is read from global memory (a few cached bytes
+// per step): key-stationary CTAs scan mask column j over 64-row query tiles
+// (mask row q*64/128), query-stationary CTAs scan mask row i over key tiles,
+// both with the causal valid-tile rule applied by AND.
+struct TileCursor {
+  const uint8_t* mask;
+  int kind;  // 0 key-stationary, 1 query-stationary
+  int tile, T, Tq1, causal, pos;
+  __device__ __forceinline__ bool allowed(int x) const {
+    if (kind == 0) {
+      if (causal && tile * kBlockN > x * kBR + kBR - 1) return false;
+      return mask[static_cast<size_t>((x * kBR) / 128) * T + tile] != 0;
+    }
+    if (causal && x > tile) return false;
+    return mask[static_cast<size_t>(tile) * T + x] != 0;
+  }
+  __device__ __forceinline__ int first() const {
+    if (mask != nullptr) return 0;
+    return (kind == 0 && causal) ? (tile * kBlockN) / kBR : 0;
+  }
+  // Next visited tile (call exactly `len` times).
+  __device__ __forceinline__ int next() {
+    if (mask == nullptr) return pos++;
+    while (!allowed(pos)) ++pos;
+    return pos++;
+  }
 };
 
 struct Params {
@@ -87,17 +134,16 @@ struct Params {
   void* dq;
   void* dk;
   void* dv;
-  float* dq_acc;   // [BH][N][d]
-  float* delta;    // [BH][Npad]
-  float* lse2;     // [BH][Npad]
+  float* delta;  // [BH][Npad]
+  float* lse2;   // [BH][Npad]
   const uint8_t* block_mask;
   int32_t* trace;
   int* status;
   int N;
   int Npad;
   int BH;
-  int Tq;  // query tiles of B_r rows
-  int Tc;  // key tiles of 128
+  int T;    // ceil(N / 128): key tiles, and 128-row query tiles
+  int Tq1;  // ceil(N / 64): 64-row query tiles
   int causal;
   float scale;
   float scale_log2;
@@ -110,7 +156,7 @@ template <int D, bool BF16>
 __global__ void __launch_bounds__(256) fa_bwd_prep_kernel(Params p) {
   constexpr int kTPR = D / 8;
   const long long gt = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const long long row = gt / kTPR;  // over BH * Npad
+  const long long row = gt / kTPR;  // over BH * Npad (Npad * kTPR is a multiple of 256)
   const int part = static_cast<int>(gt % kTPR);
   const long long total = static_cast<long long>(p.BH) * p.Npad;
   if (row >= total) return;
@@ -133,18 +179,16 @@ __global__ void __launch_bounds__(256) fa_bwd_prep_kernel(Params p) {
         b0 = __uint_as_float(bw[i] << 16);
         b1 = __uint_as_float(bw[i] & 0xFFFF0000u);
       } else {
-        const __half2 ha = *reinterpret_cast<const __half2*>(&aw[i]);
-        const __half2 hb = *reinterpret_cast<const __half2*>(&bw[i]);
-        const float2 fa = __half22float2(ha);
-        const float2 fb = __half22float2(hb);
-        a0 = fa.x; a1 = fa.y; b0 = fb.x; b1 = fb.y;
+        const float2 fa = __half22float2(*reinterpret_cast<const __half2*>(&aw[i]));
+        const float2 fb = __half22float2(*reinterpret_cast<const __half2*>(&bw[i]));
+        a0 = fa.x;
+        a1 = fa.y;
+        b0 = fb.x;
+        b1 = fb.y;
       }
       acc = fmaf(a0, b0, acc);
       acc = fmaf(a1, b1, acc);
     }
-    float4* z = reinterpret_cast<float4*>(p.dq_acc + off);
-    z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
-    z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
 #pragma unroll
   for (int m = kTPR / 2; m > 0; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
@@ -160,431 +204,522 @@ __global__ void __launch_bounds__(256) fa_bwd_prep_kernel(Params p) {
   }
 }
 
-// --------------------------------------------------------------------------- finish
+// --------------------------------------------------------------------------- shared state
+
+struct Ctx {
+  uint8_t* smem;
+  uint64_t* bars;
+  TileCursor cursor;  // positioned at the first candidate tile
+  int len;
+  uint32_t tmem;
+  WaitCtx wait;
+  int warp, lane, bh;
+  __device__ __forceinline__ uint32_t bar(int i) const { return smem_u32(&bars[i]); }
+};
+
+// Write `ncols` fp32 TMEM columns of this thread's lane, scaled by `mul`, to a
+// 16-bit row in global memory (zeros if `have` is false; nothing if !valid).
+template <bool BF16>
+__device__ __forceinline__ void store_row_from_tmem(uint32_t taddr, int ncols, float mul, bool have, bool valid,
+                                                    uint16_t* dst) {
+  for (int c = 0; c < ncols; c += 32) {
+    uint32_t v[32];
+    if (have) {
+      tmem_ld32(taddr + c, v);
+      tmem_ld_wait();
+    }
+    uint32_t w[16];
+#pragma unroll
+    for (int x = 0; x < 16; ++x)
+      w[x] = have ? pack2<BF16>(__uint_as_float(v[2 * x]) * mul, __uint_as_float(v[2 * x + 1]) * mul) : 0u;
+    if (valid) {
+      uint4* o4 = reinterpret_cast<uint4*>(dst + c);
+      o4[0] = make_uint4(w[0], w[1], w[2], w[3]);
+      o4[1] = make_uint4(w[4], w[5], w[6], w[7]);
+      o4[2] = make_uint4(w[8], w[9], w[10], w[11]);
+      o4[3] = make_uint4(w[12], w[13], w[14], w[15]);
+    }
+  }
+}
+
+// --------------------------------------------------------------------------- key-stationary CTA
 
 template <int D, bool BF16>
-__global__ void __launch_bounds__(256) fa_bwd_finish_kernel(Params p) {
-  const long long total4 = static_cast<long long>(p.BH) * p.N * D / 4;
-  for (long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; t < total4;
-       t += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const float4 a = reinterpret_cast<const float4*>(p.dq_acc)[t];
-    uint2 w;
-    w.x = pack2<BF16>(a.x * p.scale, a.y * p.scale);
-    w.y = pack2<BF16>(a.z * p.scale, a.w * p.scale);
-    reinterpret_cast<uint2*>(p.dq)[t] = w;
+__device__ __forceinline__ void key_cta(const Ctx& c, const Params& p, const CUtensorMap* tq, const CUtensorMap* tk,
+                                        const CUtensorMap* tv, const CUtensorMap* tdo, int j) {
+  using C = Cfg<D>;
+  using B = KeyBars;
+  constexpr int S = C::kS1;
+  uint8_t* sK = c.smem + C::k1K;
+  uint8_t* sV = c.smem + C::k1V;
+  uint8_t* sQ = c.smem + C::k1Q;
+  uint8_t* sDO = c.smem + C::k1DO;
+  float* sL = reinterpret_cast<float*>(c.smem + C::k1L);
+  float* sDv = reinterpret_cast<float*>(c.smem + C::k1Dv);
+  constexpr int kKVChunk = kBlockN * 128;  // 64 columns x 128 rows
+  constexpr int kQChunk = kBR * 128;       // 64 columns x 64 rows
+  const int len = c.len;
+
+  if (c.warp < 4) {
+    reg_dealloc<kRegsLow>();
+    if (c.warp == 0 && c.lane == 0) {
+      // ---------------------------------------------------------- producer
+      TileCursor cur = c.cursor;
+      int32_t* tr = p.trace ? p.trace + (static_cast<size_t>(c.bh) * p.T + j) * (p.Tq1 + 1) : nullptr;
+      if (tr) tr[0] = len;
+      if (len > 0) {
+        mbar_arrive_expect_tx(c.bar(B::kv_full), 2 * C::kKVBytes);
+        for (int ch = 0; ch < D / 64; ++ch) {
+          tma_load_3d(smem_u32(sK + ch * kKVChunk), tk, c.bar(B::kv_full), ch * 64, j * kBlockN, c.bh);
+          tma_load_3d(smem_u32(sV + ch * kKVChunk), tv, c.bar(B::kv_full), ch * 64, j * kBlockN, c.bh);
+        }
+      }
+      for (int n = 0; n < len; ++n) {
+        const int i = cur.next();
+        if (tr) tr[1 + n] = i | (1 << 16);
+        const int s = n % S;
+        if (!mbar_wait(c.bar(B::qdo_empty + s), ((n / S) & 1) ^ 1, c.wait)) break;
+        const uint32_t bar = c.bar(B::qdo_full + s);
+        mbar_arrive_expect_tx(bar, 2 * C::kQ1Bytes + 2 * kBR * 4);
+        for (int ch = 0; ch < D / 64; ++ch) {
+          tma_load_3d(smem_u32(sQ + s * C::kQ1Bytes + ch * kQChunk), tq, bar, ch * 64, i * kBR, c.bh);
+          tma_load_3d(smem_u32(sDO + s * C::kQ1Bytes + ch * kQChunk), tdo, bar, ch * 64, i * kBR, c.bh);
+        }
+        const size_t vo = static_cast<size_t>(c.bh) * p.Npad + static_cast<size_t>(i) * kBR;
+        bulk_load(smem_u32(sL + s * kBR), p.lse2 + vo, kBR * 4, bar);
+        bulk_load(smem_u32(sDv + s * kBR), p.delta + vo, kBR * 4, bar);
+      }
+    } else if (c.warp == 1 && c.lane == 0 && len > 0) {
+      // ---------------------------------------------------------- MMA issuer
+      constexpr uint32_t idesc_sp = idesc_f16(BF16, 128, kBR, false, false);  // S^T, dP^T
+      constexpr uint32_t idesc_kv = idesc_f16(BF16, 128, D, false, true);     // dV, dK
+      const uint32_t t = c.tmem;
+      // Base descriptors; every MMA below adds a compile-time offset to them.
+      const uint64_t dK = sdesc_sw128(smem_u32(sK), 16, 1024);          // K-major A of S^T
+      const uint64_t dV = sdesc_sw128(smem_u32(sV), 16, 1024);          // K-major A of dP^T
+      const uint64_t dQk = sdesc_sw128(smem_u32(sQ), 16, 1024);         // K-major B of S^T
+      const uint64_t dDOk = sdesc_sw128(smem_u32(sDO), 16, 1024);       // K-major B of dP^T
+      const uint64_t dQm = sdesc_sw128(smem_u32(sQ), kQChunk, 1024);    // MN-major B of dK
+      const uint64_t dDOm = sdesc_sw128(smem_u32(sDO), kQChunk, 1024);  // MN-major B of dV
+      auto issue_sdp = [&](int n) -> bool {  // S^T_n, dP^T_n into buffer n & 1
+        const int s = n % S;
+        const int b = n & 1;
+        if (!mbar_wait(c.bar(B::qdo_full + s), (n / S) & 1, c.wait)) return false;
+        tc_fence_after();
+        const uint32_t so = static_cast<uint32_t>(s) * C::kQ1Bytes;
+        const uint64_t bq = sdesc_add(dQk, so);
+        const uint64_t bdo = sdesc_add(dDOk, so);
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const int kk = k * 16;
+          const uint32_t okv = (kk / 64) * kKVChunk + (kk % 64) * 2;
+          const uint32_t oq = (kk / 64) * kQChunk + (kk % 64) * 2;
+          umma_ss(t + 128 * b, sdesc_add(dK, okv), sdesc_add(bq, oq), idesc_sp, k > 0);
+        }
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const int kk = k * 16;
+          const uint32_t okv = (kk / 64) * kKVChunk + (kk % 64) * 2;
+          const uint32_t oq = (kk / 64) * kQChunk + (kk % 64) * 2;
+          umma_ss(t + 128 * b + 64, sdesc_add(dV, okv), sdesc_add(bdo, oq), idesc_sp, k > 0);
+        }
+        umma_commit(c.bar(B::s_full + b));
+        return true;
+      };
+      bool ok = mbar_wait(c.bar(B::kv_full), 0, c.wait);
+      if (ok) ok = issue_sdp(0);
+      if (ok && len > 1) ok = issue_sdp(1);
+      for (int n = 0; ok && n < len; ++n) {
+        const int s = n % S;
+        const int b = n & 1;
+        if (!(ok = mbar_wait(c.bar(B::p_full + b), (n >> 1) & 1, c.wait))) break;
+        tc_fence_after();
+        const uint32_t acc = n > 0 ? 1u : 0u;
+        const uint32_t so = static_cast<uint32_t>(s) * C::kQ1Bytes;
+        const uint64_t bdo = sdesc_add(dDOm, so);
+        const uint64_t bq = sdesc_add(dQm, so);
+        const uint32_t tb = t + 128 * b;
+#pragma unroll
+        for (int k = 0; k < kBR / 16; ++k) {
+          // P^T columns of query rows 16k..16k+15 (warpgroup h = k/2 wrote them).
+          umma_ts(t + 256, tb + 32 * (k / 2) + 8 * (k % 2), sdesc_add(bdo, k * 16 * 128), idesc_kv,
+                  acc | static_cast<uint32_t>(k > 0));
+        }
+#pragma unroll
+        for (int k = 0; k < kBR / 16; ++k) {
+          umma_ts(t + 256 + D, tb + 64 + 32 * (k / 2) + 8 * (k % 2), sdesc_add(bq, k * 16 * 128), idesc_kv,
+                  acc | static_cast<uint32_t>(k > 0));
+        }
+        umma_commit(c.bar(B::qdo_empty + s));
+        if (n + 2 < len) ok = issue_sdp(n + 2);  // buffer b again: ordered after dV, dK above
+      }
+      if (ok) umma_commit(c.bar(B::all_done));
+    }
+  } else {
+    reg_alloc<kRegsHigh>();
+    // ------------------------------------------------------------ elementwise (thread = key row)
+    TileCursor cur = c.cursor;
+    const int h = (c.warp - 4) / 4;  // query columns [32h, 32h + 32) of each 64-row tile
+    const int wq = c.warp % 4;
+    const int r = wq * 32 + c.lane;
+    const int key = j * kBlockN + r;
+    const bool key_valid = key < p.N;
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const float sl2 = p.scale_log2;
+    const int qo = 32 * h;
+    bool ok = true;
+    for (int n = 0; n < len; ++n) {
+      const int i = cur.next();
+      const int s = n % S;
+      const int b = n & 1;
+      if (!(ok = mbar_wait_warp(c.bar(B::s_full + b), (n >> 1) & 1, c.wait))) break;
+      if (!(ok = mbar_wait_warp(c.bar(B::qdo_full + s), (n / S) & 1, c.wait))) break;  // lse2, D of tile i
+      tc_fence_after();
+      const uint32_t tS = c.tmem + lane_off + 128 * b;
+      uint32_t sr[32], dr[32];
+      tmem_ld32(tS + qo, sr);
+      tmem_ld32(tS + 64 + qo, dr);
+      tmem_ld_wait();
+      // Columns x < lim are masked (causal: key > query; or the key row lies past N).
+      int lim = 0;
+      if (!key_valid) {
+        lim = 32;
+      } else if (p.causal && j * kBlockN + kBlockN - 1 > i * kBR) {
+        lim = min(32, max(0, key - (i * kBR + qo)));
+      }
+      const uint32_t aL = smem_u32(sL + s * kBR + qo);
+      const uint32_t aD = smem_u32(sDv + s * kBR + qo);
+      uint32_t pk[16], dk[16];
+#pragma unroll
+      for (int x = 0; x < 32; x += 4) {
+        const float4 l4 = lds128(aL + x * 4);
+        const float4 d4 = lds128(aD + x * 4);
+        float p0 = ex2(fmaf(__uint_as_float(sr[x]), sl2, -l4.x));
+        float p1 = ex2(fmaf(__uint_as_float(sr[x + 1]), sl2, -l4.y));
+        float p2 = ex2(fmaf(__uint_as_float(sr[x + 2]), sl2, -l4.z));
+        float p3 = ex2(fmaf(__uint_as_float(sr[x + 3]), sl2, -l4.w));
+        if (lim > 0) {
+          if (x < lim) p0 = 0.0f;
+          if (x + 1 < lim) p1 = 0.0f;
+          if (x + 2 < lim) p2 = 0.0f;
+          if (x + 3 < lim) p3 = 0.0f;
+        }
+        pk[x / 2] = pack2<BF16>(p0, p1);
+        pk[x / 2 + 1] = pack2<BF16>(p2, p3);
+        dk[x / 2] = pack2<BF16>(p0 * (__uint_as_float(dr[x]) - d4.x), p1 * (__uint_as_float(dr[x + 1]) - d4.y));
+        dk[x / 2 + 1] =
+            pack2<BF16>(p2 * (__uint_as_float(dr[x + 2]) - d4.z), p3 * (__uint_as_float(dr[x + 3]) - d4.w));
+      }
+      tmem_st16(tS + 32 * h, pk);
+      tmem_st16(tS + 64 + 32 * h, dk);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(c.bar(B::p_full + b));
+    }
+    // Epilogue: warpgroup 0 writes dV_j, warpgroup 1 writes scale * dK_j.
+    bool have = false;
+    if (ok && len > 0) {
+      ok = mbar_wait_warp(c.bar(B::all_done), 0, c.wait);
+      have = ok;
+    }
+    tc_fence_after();
+    if (ok) {
+      uint16_t* dst = reinterpret_cast<uint16_t*>(h == 0 ? p.dv : p.dk) +
+                      (static_cast<size_t>(c.bh) * p.N + (key_valid ? key : 0)) * D;
+      store_row_from_tmem<BF16>(c.tmem + lane_off + 256 + h * D, D, h == 0 ? 1.0f : p.scale, have, key_valid, dst);
+    }
+  }
+}
+
+// --------------------------------------------------------------------------- query-stationary CTA
+
+template <int D, bool BF16>
+__device__ __forceinline__ void query_cta(const Ctx& c, const Params& p, const CUtensorMap* tq,
+                                          const CUtensorMap* tk, const CUtensorMap* tv, const CUtensorMap* tdo,
+                                          int i) {
+  using C = Cfg<D>;
+  using B = QueryBars;
+  constexpr int SK = C::kSK;
+  constexpr int SV = C::kSV;
+  uint8_t* sQ = c.smem + C::k2Q;
+  uint8_t* sDO = c.smem + C::k2DO;
+  uint8_t* sK = c.smem + C::k2K;
+  uint8_t* sV = c.smem + C::k2V;
+  constexpr int kChunk = 128 * 128;  // 64 columns x 128 rows
+  const int len = c.len;
+
+  if (c.warp < 4) {
+    reg_dealloc<kRegsLow>();
+    if (c.warp == 0 && c.lane == 0) {
+      // ---------------------------------------------------------- producer
+      TileCursor cur = c.cursor;
+      int32_t* tr = p.trace ? p.trace + static_cast<size_t>(p.BH) * p.T * (p.Tq1 + 1) +
+                                  (static_cast<size_t>(c.bh) * p.T + i) * (p.T + 1)
+                            : nullptr;
+      if (tr) tr[0] = len;
+      if (len > 0) {
+        mbar_arrive_expect_tx(c.bar(B::q_full), 2 * C::kQ2Bytes);
+        // The Q and dO maps have 64-row boxes: two boxes fill one 128-row chunk.
+        for (int ch = 0; ch < D / 64; ++ch) {
+          for (int hr = 0; hr < 2; ++hr) {
+            tma_load_3d(smem_u32(sQ + ch * kChunk + hr * 64 * 128), tq, c.bar(B::q_full), ch * 64,
+                        i * kBlockQ + hr * 64, c.bh);
+            tma_load_3d(smem_u32(sDO + ch * kChunk + hr * 64 * 128), tdo, c.bar(B::q_full), ch * 64,
+                        i * kBlockQ + hr * 64, c.bh);
+          }
+        }
+      }
+      for (int n = 0; n < len; ++n) {
+        const int jt = cur.next();
+        if (tr) tr[1 + n] = jt | (1 << 16);
+        const int sk = n % SK;
+        if (!mbar_wait(c.bar(B::k_empty + sk), ((n / SK) & 1) ^ 1, c.wait)) break;
+        mbar_arrive_expect_tx(c.bar(B::k_full + sk), C::kKVBytes);
+        for (int ch = 0; ch < D / 64; ++ch)
+          tma_load_3d(smem_u32(sK + sk * C::kKVBytes + ch * kChunk), tk, c.bar(B::k_full + sk), ch * 64,
+                      jt * kBlockN, c.bh);
+        const int sv = n % SV;
+        if (!mbar_wait(c.bar(B::v_empty + sv), ((n / SV) & 1) ^ 1, c.wait)) break;
+        mbar_arrive_expect_tx(c.bar(B::v_full + sv), C::kKVBytes);
+        for (int ch = 0; ch < D / 64; ++ch)
+          tma_load_3d(smem_u32(sV + sv * C::kKVBytes + ch * kChunk), tv, c.bar(B::v_full + sv), ch * 64,
+                      jt * kBlockN, c.bh);
+      }
+    } else if (c.warp == 1 && c.lane == 0 && len > 0) {
+      // ---------------------------------------------------------- MMA issuer
+      constexpr uint32_t idesc_sp = idesc_f16(BF16, 128, kBlockN, false, false);  // S, dP
+      constexpr uint32_t idesc_q = idesc_f16(BF16, 128, D, false, true);          // dQ
+      const uint32_t t = c.tmem;
+      // Base descriptors; every MMA below adds a compile-time offset to them.
+      const uint64_t dQ = sdesc_sw128(smem_u32(sQ), 16, 1024);        // K-major A of S
+      const uint64_t dDO = sdesc_sw128(smem_u32(sDO), 16, 1024);      // K-major A of dP
+      const uint64_t dKk = sdesc_sw128(smem_u32(sK), 16, 1024);       // K-major B of S
+      const uint64_t dVk = sdesc_sw128(smem_u32(sV), 16, 1024);       // K-major B of dP
+      const uint64_t dKm = sdesc_sw128(smem_u32(sK), kChunk, 1024);   // MN-major B of dQ
+      auto issue_s = [&](int n) -> bool {  // S_n into buffer n & 1
+        const int sk = n % SK;
+        if (!mbar_wait(c.bar(B::k_full + sk), (n / SK) & 1, c.wait)) return false;
+        tc_fence_after();
+        const uint64_t bk = sdesc_add(dKk, static_cast<uint32_t>(sk) * C::kKVBytes);
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const int kk = k * 16;
+          const uint32_t off = (kk / 64) * kChunk + (kk % 64) * 2;
+          umma_ss(t + 128 * (n & 1), sdesc_add(dQ, off), sdesc_add(bk, off), idesc_sp, k > 0);
+        }
+        umma_commit(c.bar(B::s_full + (n & 1)));
+        return true;
+      };
+      auto issue_dp = [&](int n) -> bool {  // dP_n; V_n is released as soon as it completes
+        const int sv = n % SV;
+        if (!mbar_wait(c.bar(B::v_full + sv), (n / SV) & 1, c.wait)) return false;
+        tc_fence_after();
+        const uint64_t bv = sdesc_add(dVk, static_cast<uint32_t>(sv) * C::kKVBytes);
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const int kk = k * 16;
+          const uint32_t off = (kk / 64) * kChunk + (kk % 64) * 2;
+          umma_ss(t + 256, sdesc_add(dDO, off), sdesc_add(bv, off), idesc_sp, k > 0);
+        }
+        umma_commit(c.bar(B::dp_full));
+        umma_commit(c.bar(B::v_empty + sv));
+        return true;
+      };
+      bool ok = mbar_wait(c.bar(B::q_full), 0, c.wait);
+      if (ok) ok = issue_s(0);
+      if (ok) ok = issue_dp(0);
+      if (ok && len > 1) ok = issue_s(1);
+      for (int n = 0; ok && n < len; ++n) {
+        const int sk = n % SK;
+        if (!(ok = mbar_wait(c.bar(B::ds_full), n & 1, c.wait))) break;  // dS_n written, S_n consumed
+        tc_fence_after();
+        const uint64_t bk = sdesc_add(dKm, static_cast<uint32_t>(sk) * C::kKVBytes);
+#pragma unroll
+        for (int k = 0; k < kBlockN / 16; ++k) {
+          // dS columns of keys 16k..16k+15 (warpgroup h = k/4 wrote them at 256 + 64h).
+          umma_ts(t + 384, t + 256 + 64 * (k / 4) + 8 * (k % 4), sdesc_add(bk, k * 16 * 128), idesc_q,
+                  (n > 0 || k > 0) ? 1u : 0u);
+        }
+        umma_commit(c.bar(B::k_empty + sk));              // K_n free once dQ_n is done
+        if (ok && n + 1 < len) ok = issue_dp(n + 1);      // dP region: ordered after dQ_n read dS_n
+        if (ok && n + 2 < len) ok = issue_s(n + 2);       // S buffer n & 1: consumed by elementwise n
+      }
+      if (ok) umma_commit(c.bar(B::all_done));
+    }
+  } else {
+    reg_alloc<kRegsHigh>();
+    // ------------------------------------------------------------ elementwise (thread = query row)
+    TileCursor cur = c.cursor;
+    const int h = (c.warp - 4) / 4;  // key columns [64h, 64h + 64) of each tile
+    const int wq = c.warp % 4;
+    const int r = wq * 32 + c.lane;
+    const int qrow = i * kBlockQ + r;
+    const bool row_valid = qrow < p.N;
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const float sl2 = p.scale_log2;
+    const size_t vo = static_cast<size_t>(c.bh) * p.Npad + static_cast<size_t>(i) * kBlockQ + r;
+    const float l2 = p.lse2[vo];  // +inf on padding rows: P = 0
+    const float dd = p.delta[vo];
+    bool ok = true;
+    for (int n = 0; n < len; ++n) {
+      const int jt = cur.next();
+      const int cb = n & 1;
+      if (!(ok = mbar_wait_warp(c.bar(B::s_full + cb), (n >> 1) & 1, c.wait))) break;
+      tc_fence_after();
+      uint32_t sr[64];
+      tmem_ld32(c.tmem + lane_off + 128 * cb + 64 * h, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tmem_ld32(c.tmem + lane_off + 128 * cb + 64 * h + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      tmem_ld_wait();
+      // Mask columns x > lim: causal (key > query) and keys past N.
+      int lim = 63;
+      if (p.causal && jt * kBlockN + 64 * h + 63 > qrow) lim = qrow - jt * kBlockN - 64 * h;
+      const int kv_left = p.N - jt * kBlockN - 64 * h - 1;
+      if (kv_left < lim) lim = kv_left;
+      float pv[64];
+#pragma unroll
+      for (int x = 0; x < 64; ++x) pv[x] = ex2(fmaf(__uint_as_float(sr[x]), sl2, -l2));
+      if (lim < 63) {
+#pragma unroll
+        for (int x = 0; x < 64; ++x)
+          if (x > lim) pv[x] = 0.0f;
+      }
+      if (!(ok = mbar_wait_warp(c.bar(B::dp_full), n & 1, c.wait))) break;  // dP_n
+      tc_fence_after();
+      uint32_t dr[64];
+      tmem_ld32(c.tmem + lane_off + 256 + 64 * h, *reinterpret_cast<uint32_t(*)[32]>(&dr[0]));
+      tmem_ld32(c.tmem + lane_off + 256 + 64 * h + 32, *reinterpret_cast<uint32_t(*)[32]>(&dr[32]));
+      tmem_ld_wait();
+      uint32_t dk[32];
+#pragma unroll
+      for (int x = 0; x < 32; ++x)
+        dk[x] = pack2<BF16>(pv[2 * x] * (__uint_as_float(dr[2 * x]) - dd),
+                            pv[2 * x + 1] * (__uint_as_float(dr[2 * x + 1]) - dd));
+      tmem_st32(c.tmem + lane_off + 256 + 64 * h, dk);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(c.bar(B::ds_full));
+    }
+    // Epilogue: warpgroup h writes columns [h*D/2, (h+1)*D/2) of scale * dQ_i.
+    bool have = false;
+    if (ok && len > 0) {
+      ok = mbar_wait_warp(c.bar(B::all_done), 0, c.wait);
+      have = ok;
+    }
+    tc_fence_after();
+    if (ok) {
+      uint16_t* dst = reinterpret_cast<uint16_t*>(p.dq) +
+                      (static_cast<size_t>(c.bh) * p.N + (row_valid ? qrow : 0)) * D + h * (D / 2);
+      store_row_from_tmem<BF16>(c.tmem + lane_off + 384 + h * (D / 2), D / 2, p.scale, have, row_valid, dst);
+    }
   }
 }
 
 // --------------------------------------------------------------------------- main
 
-__device__ __forceinline__ void named_barrier(int id, int threads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
-}
-
-// Query-tile iteration of one key tile: entry n is query tile i(n).
-struct QList {
-  int len;
-  int mode;  // 0 dense, 1 causal (range from start), 2 smem list
-  int start;
-  const uint32_t* list;
-  __device__ __forceinline__ int at(int n) const { return mode == 2 ? static_cast<int>(list[n]) : start + n; }
-};
-
+// grid = (batch*heads, 2*T). blockIdx.y = 2t: key-stationary CTA for key tile t;
+// blockIdx.y = 2t+1: query-stationary CTA for query tile T-1-t. Under a causal
+// mask small key tiles and large query tiles carry the most work, so the
+// heaviest CTAs of both kinds are dispatched first.
 template <int D, bool BF16>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_bwd_main_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                        const __grid_constant__ CUtensorMap tmap_v, const __grid_constant__ CUtensorMap tmap_do,
-                       const __grid_constant__ CUtensorMap tmap_dq, const Params p) {
+                       const Params p) {
   using C = Cfg<D>;
-  constexpr int BR = C::BR;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  Ctx c;
+  c.smem = smem;
+  c.bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
   int* list_len = reinterpret_cast<int*>(smem + C::kOffMisc + 8);
-  uint32_t* list = reinterpret_cast<uint32_t*>(smem + C::kOffList);
-  float* sL = reinterpret_cast<float*>(smem + C::kOffL);
-  float* sDv = reinterpret_cast<float*>(smem + C::kOffDv);
+  c.warp = threadIdx.x / 32;
+  c.lane = threadIdx.x % 32;
+  c.bh = blockIdx.x;
+  const bool keys = (blockIdx.y & 1) == 0;
+  const int tile = keys ? static_cast<int>(blockIdx.y >> 1) : p.T - 1 - static_cast<int>(blockIdx.y >> 1);
 
-  const uint32_t bar_kv_full = smem_u32(&bars[0]);
-  auto bar_qdo_full = [&](int s) { return smem_u32(&bars[1 + s]); };
-  auto bar_qdo_empty = [&](int s) { return smem_u32(&bars[3 + s]); };
-  const uint32_t bar_s_full = smem_u32(&bars[5]);
-  const uint32_t bar_p_full = smem_u32(&bars[6]);
-  const uint32_t bar_p_free = smem_u32(&bars[7]);
-  auto bar_ds_empty = [&](int b) { return smem_u32(&bars[8 + b]); };
-  const uint32_t bar_dq_full = smem_u32(&bars[10]);
-  const uint32_t bar_dq_empty = smem_u32(&bars[11]);
-  const uint32_t bar_all_done = smem_u32(&bars[12]);
-
-  const int warp = threadIdx.x / 32;
-  const int lane = threadIdx.x % 32;
-  // x runs over the key tiles of one head, so the CTAs that share a head's Q, dO
-  // and dQ accumulator in L2 run together; small j (most query tiles under a
-  // causal mask) goes first.
-  const int bh = blockIdx.y;
-  const int j = blockIdx.x;
-  const int cta = bh * p.Tc + j;
+  c.cursor.mask = p.block_mask;
+  c.cursor.kind = keys ? 0 : 1;
+  c.cursor.tile = tile;
+  c.cursor.T = p.T;
+  c.cursor.Tq1 = p.Tq1;
+  c.cursor.causal = p.causal;
+  c.cursor.pos = c.cursor.first();
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
-    mbar_init(bar_kv_full, 1);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(bar_qdo_full(s), 1);
-      mbar_init(bar_qdo_empty(s), 1);
-      mbar_init(bar_ds_empty(s), 1);
+    if (keys) {
+      using B = KeyBars;
+      mbar_init(c.bar(B::kv_full), 1);
+      for (int s = 0; s < C::kS1; ++s) {
+        mbar_init(c.bar(B::qdo_full + s), 1);
+        mbar_init(c.bar(B::qdo_empty + s), 1);
+      }
+      for (int b = 0; b < 2; ++b) {
+        mbar_init(c.bar(B::s_full + b), 1);
+        mbar_init(c.bar(B::p_full + b), 256);
+      }
+      mbar_init(c.bar(B::all_done), 1);
+    } else {
+      using B = QueryBars;
+      mbar_init(c.bar(B::q_full), 1);
+      for (int s = 0; s < 3; ++s) {
+        mbar_init(c.bar(B::k_full + s), 1);
+        mbar_init(c.bar(B::k_empty + s), 1);
+        mbar_init(c.bar(B::v_full + s), 1);
+        mbar_init(c.bar(B::v_empty + s), 1);
+      }
+      mbar_init(c.bar(B::s_full), 1);
+      mbar_init(c.bar(B::s_full + 1), 1);
+      mbar_init(c.bar(B::dp_full), 1);
+      mbar_init(c.bar(B::ds_full), 256);
+      mbar_init(c.bar(B::all_done), 1);
     }
-    mbar_init(bar_s_full, 1);
-    mbar_init(bar_p_full, 256);
-    mbar_init(bar_p_free, 1);
-    mbar_init(bar_dq_full, 1);
-    mbar_init(bar_dq_empty, 128);
-    mbar_init(bar_all_done, 1);
     fence_barrier_init();
   }
-  if (warp == 1) {
+  if (c.warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
   }
-  if (warp == 2 && p.block_mask != nullptr) {
-    // Query tiles i whose mask row (i*B_r/128) has column j set, with the causal
-    // valid-tile rule j*128 <= i*B_r + B_r - 1 applied by AND; ascending i.
+  if (c.warp == 2) {
+    // Number of tiles this CTA visits.
     int count = 0;
-    for (int base = 0; base < p.Tq; base += 32) {
-      const int i = base + lane;
-      bool use = false;
-      if (i < p.Tq) {
-        use = p.block_mask[static_cast<size_t>((i * BR) / 128) * p.Tc + j] != 0;
-        if (p.causal && j * kBlockN > i * BR + BR - 1) use = false;
+    if (p.block_mask != nullptr) {
+      const int range = keys ? p.Tq1 : p.T;
+      for (int base = 0; base < range; base += 32) {
+        const int x = base + c.lane;
+        const bool use = x < range && c.cursor.allowed(x);
+        count += __popc(__ballot_sync(0xffffffffu, use));
       }
-      const uint32_t ballot = __ballot_sync(0xffffffffu, use);
-      if (use) {
-        const int pos = count + __popc(ballot & ((1u << lane) - 1u));
-        if (pos < kMaxSparseTiles) list[pos] = static_cast<uint32_t>(i);
-      }
-      count += __popc(ballot);
+    } else if (keys) {
+      count = p.Tq1 - c.cursor.first();
+      if (count < 0) count = 0;
+    } else {
+      count = p.causal ? tile + 1 : p.T;
     }
-    if (lane == 0) *list_len = count < kMaxSparseTiles ? count : kMaxSparseTiles;
+    if (c.lane == 0) *list_len = count;
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  c.tmem = *tmem_slot;
+  c.len = *list_len;
+  c.wait = WaitCtx{abort_flag, p.status};
 
-  const uint32_t tmem = *tmem_slot;
-  WaitCtx ctx{abort_flag, p.status};
-
-  QList ql;
-  ql.list = list;
-  if (p.block_mask != nullptr) {
-    ql.mode = 2;
-    ql.start = 0;
-    ql.len = *list_len;
-  } else if (p.causal) {
-    ql.mode = 1;
-    ql.start = (j * kBlockN) / BR;
-    ql.len = p.Tq > ql.start ? p.Tq - ql.start : 0;
+  if (keys) {
+    key_cta<D, BF16>(c, p, &tmap_q, &tmap_k, &tmap_v, &tmap_do, tile);
   } else {
-    ql.mode = 0;
-    ql.start = 0;
-    ql.len = p.Tq;
-  }
-
-  uint8_t* sK = smem + C::kOffK;
-  uint8_t* sV = smem + C::kOffV;
-  uint8_t* sQ = smem + C::kOffQ;
-  uint8_t* sDO = smem + C::kOffDO;
-  uint8_t* sDS = smem + C::kOffDS;
-  float* sDQ = reinterpret_cast<float*>(smem + C::kOffDQ);
-  constexpr int kKVChunk = kBlockN * 128;  // 64 columns x 128 key rows
-  constexpr int kQChunk = BR * 128;        // 64 columns x B_r query rows
-
-  if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      if (p.trace) {
-        int32_t* t = p.trace + static_cast<size_t>(cta) * (p.Tq + 1);
-        t[0] = ql.len;
-        for (int n = 0; n < ql.len; ++n) t[1 + n] = ql.at(n) | (1 << 16);
-      }
-      if (ql.len > 0) {
-        prefetch_tmap(&tmap_q);
-        prefetch_tmap(&tmap_k);
-        prefetch_tmap(&tmap_v);
-        prefetch_tmap(&tmap_do);
-        mbar_arrive_expect_tx(bar_kv_full, 2 * C::kKVBytes);
-        for (int c = 0; c < D / 64; ++c) {
-          tma_load_3d(smem_u32(sK + c * kKVChunk), &tmap_k, bar_kv_full, c * 64, j * kBlockN, bh);
-          tma_load_3d(smem_u32(sV + c * kKVChunk), &tmap_v, bar_kv_full, c * 64, j * kBlockN, bh);
-        }
-        for (int n = 0; n < ql.len; ++n) {
-          const int i = ql.at(n);
-          const int s = n & 1;
-          if (!mbar_wait(bar_qdo_empty(s), ((n >> 1) & 1) ^ 1, ctx)) break;
-          const uint32_t bar = bar_qdo_full(s);
-          mbar_arrive_expect_tx(bar, 2 * C::kQBytes + 2 * C::kStageVec);
-          for (int c = 0; c < D / 64; ++c) {
-            tma_load_3d(smem_u32(sQ + s * C::kQBytes + c * kQChunk), &tmap_q, bar, c * 64, i * BR, bh);
-            tma_load_3d(smem_u32(sDO + s * C::kQBytes + c * kQChunk), &tmap_do, bar, c * 64, i * BR, bh);
-          }
-          const size_t vo = static_cast<size_t>(bh) * p.Npad + static_cast<size_t>(i) * BR;
-          bulk_load(smem_u32(sL + s * BR), p.lse2 + vo, C::kStageVec, bar);
-          bulk_load(smem_u32(sDv + s * BR), p.delta + vo, C::kStageVec, bar);
-        }
-      }
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && ql.len > 0) {
-      constexpr uint32_t idesc_sp = idesc_f16(BF16, 128, BR, false, false);  // S^T, dP^T
-      constexpr uint32_t idesc_kv = idesc_f16(BF16, 128, D, false, true);    // dV, dK
-      constexpr uint32_t idesc_q = idesc_f16(BF16, 128, D == 64 ? D : BR, true, true);  // dQ / dQ^T
-
-      auto issue_sdp = [&](int n) {
-        const int s = n & 1;
-#pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          const int kk = k * 16;
-          const uint32_t okv = (kk / 64) * kKVChunk + (kk % 64) * 2;
-          const uint32_t oq = (kk / 64) * kQChunk + (kk % 64) * 2;
-          umma_ss(tmem + C::kColS, sdesc_sw128(smem_u32(sK + okv), 16, 1024),
-                  sdesc_sw128(smem_u32(sQ + s * C::kQBytes + oq), 16, 1024), idesc_sp, k > 0);
-        }
-#pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          const int kk = k * 16;
-          const uint32_t okv = (kk / 64) * kKVChunk + (kk % 64) * 2;
-          const uint32_t oq = (kk / 64) * kQChunk + (kk % 64) * 2;
-          umma_ss(tmem + C::kColDP, sdesc_sw128(smem_u32(sV + okv), 16, 1024),
-                  sdesc_sw128(smem_u32(sDO + s * C::kQBytes + oq), 16, 1024), idesc_sp, k > 0);
-        }
-        umma_commit(bar_s_full);
-      };
-
-      bool ok = mbar_wait(bar_kv_full, 0, ctx) && mbar_wait(bar_qdo_full(0), 0, ctx);
-      if (ok) {
-        tc_fence_after();
-        issue_sdp(0);
-      }
-      for (int n = 0; ok && n < ql.len; ++n) {
-        const int s = n & 1;
-        const int b = n & 1;
-        if (!(ok = mbar_wait(bar_p_full, n & 1, ctx))) break;
-        tc_fence_after();
-        if (n + 1 < ql.len) {
-          if (!(ok = mbar_wait(bar_qdo_full((n + 1) & 1), ((n + 1) >> 1) & 1, ctx))) break;
-          tc_fence_after();
-          issue_sdp(n + 1);
-        }
-        const uint32_t acc = n > 0 ? 1u : 0u;
-        // dV += P^T dO_i   (A: P^T in TMEM; B: dO_i, d contiguous)
-#pragma unroll
-        for (int k = 0; k < BR / 16; ++k) {
-          const int kk = k * 16;
-          umma_ts(tmem + C::kColDV, tmem + C::kColP + kk / 2,
-                  sdesc_sw128(smem_u32(sDO + s * C::kQBytes + kk * 128), kQChunk, 1024), idesc_kv,
-                  acc | static_cast<uint32_t>(k > 0));
-        }
-        umma_commit(bar_p_free);
-        // dK += dS^T Q_i   (A: dS^T in smem, query columns contiguous; B: Q_i, d contiguous)
-#pragma unroll
-        for (int k = 0; k < BR / 16; ++k) {
-          const int kk = k * 16;
-          const uint32_t oa = (kk / 64) * (kBlockN * 128) + (kk % 64) * 2;
-          umma_ss(tmem + C::kColDK, sdesc_sw128(smem_u32(sDS + b * C::kDSBytes + oa), 16, 1024),
-                  sdesc_sw128(smem_u32(sQ + s * C::kQBytes + kk * 128), kQChunk, 1024), idesc_kv,
-                  acc | static_cast<uint32_t>(k > 0));
-        }
-        if (!(ok = mbar_wait(bar_dq_empty, (n & 1) ^ 1, ctx))) break;
-        tc_fence_after();
-#pragma unroll
-        for (int k = 0; k < kBlockN / 16; ++k) {
-          const int kk = k * 16;
-          if constexpr (D == 64) {
-            // dQ = dS K_j: A = dS (query rows contiguous in smem), B = K_j (d contiguous)
-            umma_ss(tmem + C::kColDQ, sdesc_sw128(smem_u32(sDS + b * C::kDSBytes + kk * 128), kBlockN * 128, 1024),
-                    sdesc_sw128(smem_u32(sK + kk * 128), kKVChunk, 1024), idesc_q, k > 0);
-          } else {
-            // dQ^T = K_j^T dS^T: A = K_j^T (d contiguous), B = dS^T (query columns contiguous)
-            umma_ss(tmem + C::kColDQ, sdesc_sw128(smem_u32(sK + kk * 128), kKVChunk, 1024),
-                    sdesc_sw128(smem_u32(sDS + b * C::kDSBytes + kk * 128), kBlockN * 128, 1024), idesc_q,
-                    k > 0);
-          }
-        }
-        umma_commit(bar_dq_full);
-        umma_commit(bar_ds_empty(b));
-        umma_commit(bar_qdo_empty(s));
-      }
-      if (ok) umma_commit(bar_all_done);
-    }
-  } else if (warp >= 4 && warp < 12) {
-    // ------------------------------------------------------------ elementwise (thread = key row)
-    const int half = (warp - 4) / 4;  // which half of the query columns
-    const int wq = warp % 4;
-    const int r = wq * 32 + lane;      // key row within the tile
-    const int key = j * kBlockN + r;
-    const bool key_valid = key < p.N;  // rows past N were zero-filled; keep their P at 0
-    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-    const float sl2 = p.scale_log2;
-    bool ok = true;
-    for (int n = 0; ok && n < ql.len; ++n) {
-      const int i = ql.at(n);
-      const int s = n & 1;
-      const int b = n & 1;
-      if (!(ok = mbar_wait_warp(bar_s_full, n & 1, ctx))) break;
-      // lse2 and D of this tile arrived with Q_i (same barrier phase as the S^T inputs).
-      if (!(ok = mbar_wait_warp(bar_qdo_full(s), (n >> 1) & 1, ctx))) break;
-      tc_fence_after();
-      const bool diag = p.causal && (j * kBlockN + kBlockN - 1 > i * BR);
-      const uint32_t aL = smem_u32(sL + s * BR);
-      const uint32_t aD = smem_u32(sDv + s * BR);
-#pragma unroll
-      for (int cc = 0; cc < BR / 64; ++cc) {
-        const int qo = half * (BR / 2) + cc * 32;  // first query column of this chunk
-        uint32_t sr[32], dr[32];
-        tmem_ld32(tmem + lane_off + C::kColS + qo, sr);
-        tmem_ld32(tmem + lane_off + C::kColDP + qo, dr);
-        tmem_ld_wait();
-        // Columns x < lim are masked (causal: key > query; or the key row is past N).
-        int lim = 0;
-        if (!key_valid) lim = 32;
-        else if (diag) lim = min(32, max(0, key - (i * BR + qo)));
-        uint32_t pk[16], dk[16];
-#pragma unroll
-        for (int x = 0; x < 32; x += 4) {
-          const float4 l4 = lds128(aL + (qo + x) * 4);
-          const float4 d4 = lds128(aD + (qo + x) * 4);
-          float p0 = ex2(fmaf(__uint_as_float(sr[x]), sl2, -l4.x));
-          float p1 = ex2(fmaf(__uint_as_float(sr[x + 1]), sl2, -l4.y));
-          float p2 = ex2(fmaf(__uint_as_float(sr[x + 2]), sl2, -l4.z));
-          float p3 = ex2(fmaf(__uint_as_float(sr[x + 3]), sl2, -l4.w));
-          if (lim > 0) {
-            if (x < lim) p0 = 0.0f;
-            if (x + 1 < lim) p1 = 0.0f;
-            if (x + 2 < lim) p2 = 0.0f;
-            if (x + 3 < lim) p3 = 0.0f;
-          }
-          pk[x / 2] = pack2<BF16>(p0, p1);
-          pk[x / 2 + 1] = pack2<BF16>(p2, p3);
-          dk[x / 2] = pack2<BF16>(p0 * (__uint_as_float(dr[x]) - d4.x), p1 * (__uint_as_float(dr[x + 1]) - d4.y));
-          dk[x / 2 + 1] = pack2<BF16>(p2 * (__uint_as_float(dr[x + 2]) - d4.z), p3 * (__uint_as_float(dr[x + 3]) - d4.w));
-        }
-        if (cc == 0 && n > 0) {
-          // P^T of the previous tile must have been consumed by its dV MMA.
-          if (!(ok = mbar_wait_warp(bar_p_free, (n - 1) & 1, ctx))) break;
-        }
-        tmem_st16(tmem + lane_off + C::kColP + qo / 2, pk);
-        if (cc == 0 && n >= 2) {
-          if (!(ok = mbar_wait_warp(bar_ds_empty(b), ((n - 2) >> 1) & 1, ctx))) break;
-        }
-        // dS^T row r, query columns qo..qo+31 -> four 16-byte pieces of the swizzled row.
-        const uint32_t rowa = smem_u32(sDS + b * C::kDSBytes + (qo / 64) * (kBlockN * 128) + r * 128);
-        const int p0i = (qo % 64) / 8;
-#pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          const int phys = (p0i + t) ^ (r & 7);
-          sts128(rowa + phys * 16, dk[4 * t], dk[4 * t + 1], dk[4 * t + 2], dk[4 * t + 3]);
-        }
-      }
-      if (!ok) break;
-      tmem_st_wait();
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(bar_p_full);
-    }
-    // Epilogue: half 0 writes dV_j, half 1 writes scale * dK_j.
-    bool have = false;
-    if (ok && ql.len > 0) {
-      ok = mbar_wait_warp(bar_all_done, 0, ctx);
-      have = ok;
-    }
-    tc_fence_after();
-    if (ok) {
-      const uint32_t col = half == 0 ? C::kColDV : C::kColDK;
-      const float mul = half == 0 ? 1.0f : p.scale;
-      uint16_t* dst = reinterpret_cast<uint16_t*>(half == 0 ? p.dv : p.dk);
-      const bool valid = key < p.N;
-      uint16_t* rowp = dst + (static_cast<size_t>(bh) * p.N + (valid ? key : 0)) * D;
-#pragma unroll
-      for (int c = 0; c < D; c += 32) {
-        uint32_t v[32];
-        if (have) {
-          tmem_ld32(tmem + lane_off + col + c, v);
-          tmem_ld_wait();
-        }
-        uint32_t w[16];
-#pragma unroll
-        for (int x = 0; x < 16; ++x)
-          w[x] = have ? pack2<BF16>(__uint_as_float(v[2 * x]) * mul, __uint_as_float(v[2 * x + 1]) * mul) : 0u;
-        if (valid) {
-          uint4* o4 = reinterpret_cast<uint4*>(rowp + c);
-          o4[0] = make_uint4(w[0], w[1], w[2], w[3]);
-          o4[1] = make_uint4(w[4], w[5], w[6], w[7]);
-          o4[2] = make_uint4(w[8], w[9], w[10], w[11]);
-          o4[3] = make_uint4(w[12], w[13], w[14], w[15]);
-        }
-      }
-    }
-  } else if (warp >= 12) {
-    // ------------------------------------------------------------ dQ drain
-    const int wq = warp % 4;
-    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-    const bool leader = (warp == 12 && lane == 0);
-    bool ok = true;
-    for (int n = 0; ok && n < ql.len; ++n) {
-      const int i = ql.at(n);
-      if (!(ok = mbar_wait_warp(bar_dq_full, n & 1, ctx))) break;
-      tc_fence_after();
-      uint32_t v0[32], v1[32];
-      tmem_ld32(tmem + lane_off + C::kColDQ, v0);
-      tmem_ld32(tmem + lane_off + C::kColDQ + 32, v1);
-      tmem_ld_wait();
-      tc_fence_before();
-      mbar_arrive(bar_dq_empty);
-      if (leader) bulk_wait_group_read<0>();  // the previous reduce has read the staging tile
-      named_barrier(1, 128);
-      const int t = wq * 32 + lane;  // TMEM lane
-      if constexpr (D == 64) {
-        // lane = query row. Staging is two [128 rows][32] fp32 boxes in the TMA
-        // 128-byte swizzle: 16-byte piece x of row t sits at piece x ^ (t & 7).
-        const uint32_t row0 = smem_u32(sDQ) + t * 128;
-        const uint32_t row1 = row0 + 128 * 128;
-#pragma unroll
-        for (int x = 0; x < 8; ++x) {
-          const int phys = (x ^ (t & 7)) * 16;
-          sts128(row0 + phys, v0[4 * x], v0[4 * x + 1], v0[4 * x + 2], v0[4 * x + 3]);
-          sts128(row1 + phys, v1[4 * x], v1[4 * x + 1], v1[4 * x + 2], v1[4 * x + 3]);
-        }
-      } else {
-        // lane = d index; columns are the 64 query rows; staging is [64 rows][128] fp32.
-        const uint32_t base = smem_u32(sDQ) + t * 4;
-#pragma unroll
-        for (int x = 0; x < 32; ++x) {
-          sts32(base + x * D * 4, v0[x]);
-          sts32(base + (x + 32) * D * 4, v1[x]);
-        }
-      }
-      fence_proxy_async_smem();
-      named_barrier(1, 128);
-      if (leader) {
-        if constexpr (D == 64) {
-          tma_reduce_add_3d(&tmap_dq, smem_u32(sDQ), 0, i * BR, bh);
-          tma_reduce_add_3d(&tmap_dq, smem_u32(sDQ) + 128 * 128, 32, i * BR, bh);
-        } else {
-          tma_reduce_add_3d(&tmap_dq, smem_u32(sDQ), 0, i * BR, bh);
-        }
-        bulk_commit_group();
-      }
-    }
-    if (leader) bulk_wait_group<0>();
+    query_cta<D, BF16>(c, p, &tmap_q, &tmap_k, &tmap_v, &tmap_do, tile);
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (c.warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(c.tmem, 512);
   }
 }
 

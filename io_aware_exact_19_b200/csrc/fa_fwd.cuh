@@ -43,8 +43,8 @@ constexpr int kThreads = 384;
 constexpr int kMaxSparseTiles = 2048;
 constexpr float kRescaleThreshold = 8.0f;
 constexpr int kRegsLaunch = 168;  // 65536 / 384, rounded down to a multiple of 8
-constexpr int kRegsLow = 56;
-constexpr int kRegsHigh = 224;
+constexpr int kRegsLow = 64;
+constexpr int kRegsHigh = 216;
 static_assert(128 * kRegsLow + 256 * kRegsHigh <= kThreads * kRegsLaunch, "register split exceeds the launch allocation");
 
 struct Params {
@@ -250,16 +250,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t started[2] = {0, 0};
       bool ok = mbar_wait(bar_q_full, 0, ctx);
 
+      // Base descriptors; every MMA below adds a compile-time offset to them.
+      const uint64_t dQ = sdesc_sw128(smem_u32(sQ), 16, 1024);             // K-major A of S
+      const uint64_t dK = sdesc_sw128(smem_u32(sK), 16, 1024);             // K-major B of S
+      const uint64_t dV = sdesc_sw128(smem_u32(sV), kChunkBytes, 1024);    // MN-major B of P V
       auto issue_s = [&](int q, int n) {
         const int s = n % S;
         const uint32_t d_tmem = tmem + q * 128;
+        const uint64_t bq = sdesc_add(dQ, static_cast<uint32_t>(q) * L::kTileBytes);
+        const uint64_t bk = sdesc_add(dK, static_cast<uint32_t>(s) * L::kTileBytes);
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
           const int kk = k * 16;
           const uint32_t off = (kk / 64) * kChunkBytes + (kk % 64) * 2;
-          const uint64_t a = sdesc_sw128(smem_u32(sQ + q * L::kTileBytes + off), 16, 1024);
-          const uint64_t b = sdesc_sw128(smem_u32(sK + s * L::kTileBytes + off), 16, 1024);
-          umma_ss(d_tmem, a, b, idesc_s, k > 0);
+          umma_ss(d_tmem, sdesc_add(bq, off), sdesc_add(bk, off), idesc_s, k > 0);
         }
         umma_commit(bar_s_full(q));
       };
@@ -267,11 +271,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int s = n % S;
         const uint32_t d_tmem = tmem + 256 + q * D;
         const uint32_t a_tmem = tmem + q * 128;
+        const uint64_t bv = sdesc_add(dV, static_cast<uint32_t>(s) * L::kTileBytes);
 #pragma unroll
         for (int k = 0; k < kBlockN / 16; ++k) {
-          const int kk = k * 16;
-          const uint64_t b = sdesc_sw128(smem_u32(sV + s * L::kTileBytes + kk * 128), kChunkBytes, 1024);
-          umma_ts(d_tmem, a_tmem + kk / 2, b, idesc_pv, (started[q] | static_cast<uint32_t>(k > 0)));
+          umma_ts(d_tmem, a_tmem + 8 * k, sdesc_add(bv, k * 16 * 128), idesc_pv,
+                  (started[q] | static_cast<uint32_t>(k > 0)));
         }
         started[q] = 1;
       };

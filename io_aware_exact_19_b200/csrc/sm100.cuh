@@ -279,6 +279,13 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_byt
   return d;
 }
 
+// Advance a descriptor's start address by `byte_off` bytes (a multiple of 16).
+// The start-address field holds address >> 4 in bits 0-13; for addresses inside
+// the CTA's shared memory the sum never carries out of the field.
+__device__ __forceinline__ uint64_t sdesc_add(uint64_t desc, uint32_t byte_off) {
+  return desc + static_cast<uint64_t>(byte_off >> 4);
+}
+
 // Instruction descriptor for kind::f16 with fp32 accumulation.
 //   bits 4-5 D format (1 = f32), 7-9 A format, 10-12 B format (0 = f16, 1 = bf16),
 //   15 A major, 16 B major (0 = K, 1 = MN), 17-22 N >> 3, 24-28 M >> 4.

@@ -142,11 +142,20 @@ def test_tile_trace_matches_oracle_enumeration(N, causal, use_mask, d):
     trace = torch.full((fa.fa_bwd_trace_size(B, H, N, d),), -1, dtype=torch.int32, device="cuda")
     fa.fa_debug_bwd_trace(q, k, v, o, lse, do, dq, dk, dv, ws, trace, causal=causal, block_mask=mdev)
     torch.cuda.synchronize()
+    got = trace.cpu().numpy().astype(np.int64)
     br = fa.fa_bwd_row_tile(d)
-    lists = oracle.backward_tile_lists(N, causal, mask, br=br, bc=128)
+    t = -(-N // 128)
     tq = -(-N // br)
-    got = trace.cpu().numpy().astype(np.int64).reshape(B * H, len(lists), tq + 1)
+    # key-stationary CTAs: the query tiles (br rows) that reach each key tile
+    key_lists = oracle.backward_tile_lists(N, causal, mask, br=br, bc=128)
+    key_part = got[:B * H * t * (tq + 1)].reshape(B * H, t, tq + 1)
+    # query-stationary CTAs: the key tiles each 128-row query tile reaches
+    query_lists = oracle.forward_tile_lists(N, causal, mask, br=128, bc=128)
+    query_part = got[B * H * t * (tq + 1):].reshape(B * H, t, t + 1)
     for bh in range(B * H):
-        for j, exp in enumerate(lists):
-            assert got[bh, j, 0] == len(exp)
-            assert list(got[bh, j, 1:1 + len(exp)]) == [i | (1 << 16) for i in exp], (bh, j)
+        for j, exp in enumerate(key_lists):
+            assert key_part[bh, j, 0] == len(exp)
+            assert list(key_part[bh, j, 1:1 + len(exp)]) == [i | (1 << 16) for i in exp], (bh, j)
+        for i, exp in enumerate(query_lists):
+            assert query_part[bh, i, 0] == len(exp)
+            assert list(query_part[bh, i, 1:1 + len(exp)]) == [j | (1 << 16) for j in exp], (bh, i)
