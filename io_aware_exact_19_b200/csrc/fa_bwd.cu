@@ -30,6 +30,7 @@ int launch_bwd_t(const AttnArgs& a, cudaStream_t stream) {
   uint8_t* base = static_cast<uint8_t*>(a.workspace);
 
   bwd::Params p;
+  p.q = a.q;
   p.o = a.o;
   p.dout = a.dout;
   p.lse = a.lse;
@@ -45,7 +46,6 @@ int launch_bwd_t(const AttnArgs& a, cudaStream_t stream) {
   p.Npad = (a.N + 127) / 128 * 128;
   p.BH = BH;
   p.T = (a.N + 127) / 128;
-  p.Tq1 = (a.N + bwd::kBR - 1) / bwd::kBR;
   p.causal = a.causal;
   p.scale = a.scale;
   p.scale_log2 = a.scale * 1.4426950408889634f;
@@ -61,8 +61,8 @@ int launch_bwd_t(const AttnArgs& a, cudaStream_t stream) {
   // main
   if (a.phases & 2) {
     CUtensorMap tq, tk, tv, tdo;
-    // Q and dO are read in 64-row tiles by key-stationary CTAs and in 128-row
-    // tiles by query-stationary CTAs: two 64-row boxes make one 128-row tile.
+    // Q and dO are read by key-stationary CTAs in 128-row tiles, loaded as two
+    // 64-row boxes per 64-column chunk.
     bool ok = host::make_map_3d(&tq, dt, 2, a.q, D, a.N, BH, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B) &&
               host::make_map_3d(&tdo, dt, 2, a.dout, D, a.N, BH, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B) &&
               host::make_map_3d(&tk, dt, 2, a.k, D, a.N, BH, 64, bwd::kBlockN, CU_TENSOR_MAP_SWIZZLE_128B) &&

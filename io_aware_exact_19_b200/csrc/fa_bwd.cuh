@@ -7,35 +7,42 @@
 //          rows and rows without keys, so their P is 0).
 //   main   one launch with two kinds of CTA, interleaved heaviest first:
 //     key-stationary (one 128-key tile j of one head; dK_j and dV_j stay in TMEM)
-//       for each 64-row query tile i that reaches j:
-//         S^T  = K_j Q_i^T,  dP^T = V_j dO_i^T                (shared-memory operands)
+//       for each 128-row query tile i that reaches j:
+//         S^T  = K_j Q_i^T,  dP^T = V_j dO_i^T
 //         P^T  = exp2(S^T * scale*log2e - lse2_i),  dS^T = P^T o (dP^T - D_i)
-//         dV_j += P^T dO_i,  dK_j += dS^T Q_i                 (P^T, dS^T read from TMEM)
+//         dV_j += P^T dO_i,  dK_j += dS^T Q_i         (P^T, dS^T read from TMEM)
 //       then dV_j and scale * dK_j are written once.
 //     query-stationary (one 128-row query tile i of one head; dQ_i stays in TMEM)
 //       for each 128-key tile j that i reaches:
-//         S = Q_i K_j^T,  dP = dO_i V_j^T,  P = exp2(S*scale*log2e - lse2),  dS = P o (dP - D)
-//         dQ_i += dS K_j                                        (dS read from TMEM)
+//         S = Q_i K_j^T,  dP = dO_i V_j^T               (Q_i, dO_i read from TMEM)
+//         P = exp2(S*scale*log2e - lse2),  dS = P o (dP - D)
+//         dQ_i += dS K_j                                (dS read from TMEM)
 //       then scale * dQ_i is written once.
 // dQ is thus produced without atomics or an fp32 accumulator in global memory,
 // at the price of recomputing S and dP once more (7 MMAs per 128x128 block of
-// scores instead of 5). The P^T, dS^T and dS operands live in TMEM, so no MMA
-// reads more than one operand tile from shared memory per 16-wide K step, which
-// keeps the shared-memory port (128 B/clock) from throttling the tensor core.
+// scores instead of 5). Every MMA is 128 x 128 (x d) or 128 x d (x 128), and
+// operands that would be re-read from shared memory every step (Q_i, dO_i in
+// the query-stationary CTA; P^T, dS^T, dS) are kept in TMEM, which keeps the
+// shared-memory port (128 bytes per clock) below the tensor core's demand.
+//
+// In both kinds the elementwise warps signal as soon as they have copied S^T
+// (or S) into registers, so the MMA for the next tile's S^T (S) overlaps their
+// work on the current tile; dP^T (dP) shares its TMEM columns with the P^T and
+// dS^T (dS) written back from it, so the next dP^T waits for the dV/dK (dQ)
+// MMAs that read them, which run in issue order.
 //
 // Roles (384 threads, one CTA per SM, both kinds):
 //   warp 0      TMA producer          warp 1      MMA issuer, TMEM owner
 //   warp 2      counts the tiles of a block-sparse CTA
-//   warps 4-7   elementwise, first half of the columns (thread = TMEM lane = row)
-//   warps 8-11  elementwise, second half of the columns
+//   warps 4-7   elementwise, columns [0, 64) of each tile (thread = TMEM lane = row)
+//   warps 8-11  elementwise, columns [64, 128)
 //
 // TMEM (512 columns):
-//   key-stationary:   buffer b in {0,1}: S^T at 128b (64 columns), dP^T at 128b+64;
-//                     warpgroup h writes its P^T (16 columns) over its own S^T
-//                     columns at 128b+32h and its dS^T over dP^T at 128b+64+32h;
+//   key-stationary:   S^T at 0; dP^T at 128, where warpgroup h later writes its
+//                     P^T (32 columns) at 128+64h and dS^T at 128+64h+32;
 //                     dV at 256, dK at 256+d.
-//   query-stationary: S buffers at 0 and 128, dP at 256 (warpgroup h writes its
-//                     dS, 32 columns, at 256+64h), dQ at 384.
+//   query-stationary: Q_i at 0 and dO_i at d/2 (bf16 pairs), S at d, dP at
+//                     d+128 (warpgroup h writes its dS at d+128+64h), dQ at d+256.
 #pragma once
 
 #include <cuda_fp16.h>
@@ -50,7 +57,7 @@ using namespace fa::sm100;
 constexpr int kThreads = 384;
 constexpr int kBlockN = 128;  // keys per key-stationary CTA and per query-stationary step
 constexpr int kBlockQ = 128;  // queries per query-stationary CTA
-constexpr int kBR = 64;       // queries per key-stationary step
+constexpr int kBR = 128;      // queries per key-stationary step
 constexpr int kRegsLaunch = 168;
 constexpr int kRegsLow = 88;
 constexpr int kRegsHigh = 208;
@@ -60,64 +67,62 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 template <int D>
 struct Cfg {
-  static constexpr int kKVBytes = kBlockN * D * 2;  // 128-row K or V tile
-  static constexpr int kQ1Bytes = kBR * D * 2;      // 64-row Q or dO tile
-  static constexpr int kQ2Bytes = kBlockQ * D * 2;  // 128-row Q or dO tile
+  static constexpr int kTile = 128 * D * 2;  // one 128-row tile of Q, dO, K or V
+  static constexpr int kChunk = 128 * 128;   // 64 columns x 128 rows, 128-byte swizzle
   // key-stationary layout: K_j, V_j, then a ring of (Q_i, dO_i, lse2_i, D_i)
-  static constexpr int kS1 = 4;
+  static constexpr int kS1 = (D == 128) ? 2 : 3;
   static constexpr int k1K = 0;
-  static constexpr int k1V = k1K + kKVBytes;
-  static constexpr int k1Q = k1V + kKVBytes;
-  static constexpr int k1DO = k1Q + kS1 * kQ1Bytes;
-  static constexpr int k1L = k1DO + kS1 * kQ1Bytes;
+  static constexpr int k1V = k1K + kTile;
+  static constexpr int k1Q = k1V + kTile;
+  static constexpr int k1DO = k1Q + kS1 * kTile;
+  static constexpr int k1L = k1DO + kS1 * kTile;
   static constexpr int k1Dv = k1L + kS1 * kBR * 4;
   static constexpr int k1End = k1Dv + kS1 * kBR * 4;
-  // query-stationary layout: Q_i, dO_i, then rings of K_j and V_j
-  static constexpr int kSK = 3;
-  static constexpr int kSV = (D == 128) ? 2 : 3;
-  static constexpr int k2Q = 0;
-  static constexpr int k2DO = k2Q + kQ2Bytes;
-  static constexpr int k2K = k2DO + kQ2Bytes;
-  static constexpr int k2V = k2K + kSK * kKVBytes;
-  static constexpr int k2End = k2V + kSV * kKVBytes;
+  // query-stationary layout: rings of K_j and V_j (Q_i, dO_i live in TMEM)
+  static constexpr int kS2 = 3;
+  static constexpr int k2K = 0;
+  static constexpr int k2V = k2K + kS2 * kTile;
+  static constexpr int k2End = k2V + kS2 * kTile;
   static constexpr int kOffBar = ((k1End > k2End ? k1End : k2End) + 15) / 16 * 16;
-  static constexpr int kNumBars = 18;
-  static constexpr int kOffMisc = kOffBar + 8 * kNumBars;  // tmem slot, abort flag, list length
+  static constexpr int kNumBars = 20;
+  static constexpr int kOffMisc = kOffBar + 8 * kNumBars;  // tmem slot, abort flag, tile count
   static constexpr int kBytes = kOffMisc + 16;
   static constexpr int kAlloc = kBytes + 1024;
   static_assert(kAlloc <= 232448, "shared memory budget");
-  static_assert(256 + 2 * D <= 512 && 384 + D <= 512, "TMEM budget");
+  static_assert(256 + 2 * D <= 512 && 2 * D + 256 <= 512, "TMEM budget");
+  // TMEM columns
+  static constexpr int kColQ = 0, kColDO = D / 2, kColS2 = D, kColDP2 = D + 128, kColDQ = D + 256;
 };
 
 // Barrier slots of the two CTA kinds (they share the same shared-memory words).
 struct KeyBars {
-  static constexpr int kv_full = 0, qdo_full = 1, qdo_empty = 5, s_full = 9, p_full = 11, all_done = 13;
+  static constexpr int kv_full = 0, qdo_full = 1, qdo_empty = 4, s_full = 7, s_free = 8, dp_full = 9,
+                       p_full = 10, all_done = 11;
 };
 struct QueryBars {
-  static constexpr int q_full = 0, k_full = 1, k_empty = 4, v_full = 7, v_empty = 10, s_full = 13, dp_full = 15,
-                       ds_full = 16, all_done = 17;
+  static constexpr int q_ready = 0, k_full = 1, k_empty = 4, v_full = 7, v_empty = 10, s_full = 13,
+                       s_free = 14, dp_full = 15, ds_full = 16, all_done = 17;
 };
 
 // Walks the tiles one CTA visits, in ascending order. Dense and causal ranges
 // are arithmetic; a block mask is read from global memory (a few cached bytes
-// per step): key-stationary CTAs scan mask column j over 64-row query tiles
-// (mask row q*64/128), query-stationary CTAs scan mask row i over key tiles,
-// both with the causal valid-tile rule applied by AND.
+// per step): key-stationary CTAs scan mask column j, query-stationary CTAs scan
+// mask row i, both with the causal valid-tile rule applied by AND.
 struct TileCursor {
   const uint8_t* mask;
   int kind;  // 0 key-stationary, 1 query-stationary
-  int tile, T, Tq1, causal, pos;
+  int tile, T, causal, pos;
   __device__ __forceinline__ bool allowed(int x) const {
     if (kind == 0) {
-      if (causal && tile * kBlockN > x * kBR + kBR - 1) return false;
-      return mask[static_cast<size_t>((x * kBR) / 128) * T + tile] != 0;
+      if (causal && x < tile) return false;
+      return mask[static_cast<size_t>(x) * T + tile] != 0;
     }
     if (causal && x > tile) return false;
     return mask[static_cast<size_t>(tile) * T + x] != 0;
   }
   __device__ __forceinline__ int first() const {
     if (mask != nullptr) return 0;
-    return (kind == 0 && causal) ? (tile * kBlockN) / kBR : 0;
+    return (kind == 0 && causal) ? tile : 0;
   }
   // Next visited tile (call exactly `len` times).
   __device__ __forceinline__ int next() {
@@ -128,6 +133,7 @@ struct TileCursor {
 };
 
 struct Params {
+  const void* q;
   const void* o;
   const void* dout;
   const float* lse;
@@ -142,8 +148,7 @@ struct Params {
   int N;
   int Npad;
   int BH;
-  int T;    // ceil(N / 128): key tiles, and 128-row query tiles
-  int Tq1;  // ceil(N / 64): 64-row query tiles
+  int T;  // ceil(N / 128): key tiles, and query tiles
   int causal;
   float scale;
   float scale_log2;
@@ -250,14 +255,13 @@ __device__ __forceinline__ void key_cta(const Ctx& c, const Params& p, const CUt
   using C = Cfg<D>;
   using B = KeyBars;
   constexpr int S = C::kS1;
+  constexpr int kChunk = C::kChunk;
   uint8_t* sK = c.smem + C::k1K;
   uint8_t* sV = c.smem + C::k1V;
   uint8_t* sQ = c.smem + C::k1Q;
   uint8_t* sDO = c.smem + C::k1DO;
   float* sL = reinterpret_cast<float*>(c.smem + C::k1L);
   float* sDv = reinterpret_cast<float*>(c.smem + C::k1Dv);
-  constexpr int kKVChunk = kBlockN * 128;  // 64 columns x 128 rows
-  constexpr int kQChunk = kBR * 128;       // 64 columns x 64 rows
   const int len = c.len;
 
   if (c.warp < 4) {
@@ -265,13 +269,13 @@ __device__ __forceinline__ void key_cta(const Ctx& c, const Params& p, const CUt
     if (c.warp == 0 && c.lane == 0) {
       // ---------------------------------------------------------- producer
       TileCursor cur = c.cursor;
-      int32_t* tr = p.trace ? p.trace + (static_cast<size_t>(c.bh) * p.T + j) * (p.Tq1 + 1) : nullptr;
+      int32_t* tr = p.trace ? p.trace + (static_cast<size_t>(c.bh) * p.T + j) * (p.T + 1) : nullptr;
       if (tr) tr[0] = len;
       if (len > 0) {
-        mbar_arrive_expect_tx(c.bar(B::kv_full), 2 * C::kKVBytes);
+        mbar_arrive_expect_tx(c.bar(B::kv_full), 2 * C::kTile);
         for (int ch = 0; ch < D / 64; ++ch) {
-          tma_load_3d(smem_u32(sK + ch * kKVChunk), tk, c.bar(B::kv_full), ch * 64, j * kBlockN, c.bh);
-          tma_load_3d(smem_u32(sV + ch * kKVChunk), tv, c.bar(B::kv_full), ch * 64, j * kBlockN, c.bh);
+          tma_load_3d(smem_u32(sK + ch * kChunk), tk, c.bar(B::kv_full), ch * 64, j * kBlockN, c.bh);
+          tma_load_3d(smem_u32(sV + ch * kChunk), tv, c.bar(B::kv_full), ch * 64, j * kBlockN, c.bh);
         }
       }
       for (int n = 0; n < len; ++n) {
@@ -280,10 +284,14 @@ __device__ __forceinline__ void key_cta(const Ctx& c, const Params& p, const CUt
         const int s = n % S;
         if (!mbar_wait(c.bar(B::qdo_empty + s), ((n / S) & 1) ^ 1, c.wait)) break;
         const uint32_t bar = c.bar(B::qdo_full + s);
-        mbar_arrive_expect_tx(bar, 2 * C::kQ1Bytes + 2 * kBR * 4);
+        mbar_arrive_expect_tx(bar, 2 * C::kTile + 2 * kBR * 4);
+        // The Q and dO maps have 64-row boxes: two boxes fill one 128-row chunk.
         for (int ch = 0; ch < D / 64; ++ch) {
-          tma_load_3d(smem_u32(sQ + s * C::kQ1Bytes + ch * kQChunk), tq, bar, ch * 64, i * kBR, c.bh);
-          tma_load_3d(smem_u32(sDO + s * C::kQ1Bytes + ch * kQChunk), tdo, bar, ch * 64, i * kBR, c.bh);
+          for (int hr = 0; hr < 2; ++hr) {
+            const uint32_t off = s * C::kTile + ch * kChunk + hr * 64 * 128;
+            tma_load_3d(smem_u32(sQ + off), tq, bar, ch * 64, i * kBR + hr * 64, c.bh);
+            tma_load_3d(smem_u32(sDO + off), tdo, bar, ch * 64, i * kBR + hr * 64, c.bh);
+          }
         }
         const size_t vo = static_cast<size_t>(c.bh) * p.Npad + static_cast<size_t>(i) * kBR;
         bulk_load(smem_u32(sL + s * kBR), p.lse2 + vo, kBR * 4, bar);
@@ -299,59 +307,59 @@ __device__ __forceinline__ void key_cta(const Ctx& c, const Params& p, const CUt
       const uint64_t dV = sdesc_sw128(smem_u32(sV), 16, 1024);          // K-major A of dP^T
       const uint64_t dQk = sdesc_sw128(smem_u32(sQ), 16, 1024);         // K-major B of S^T
       const uint64_t dDOk = sdesc_sw128(smem_u32(sDO), 16, 1024);       // K-major B of dP^T
-      const uint64_t dQm = sdesc_sw128(smem_u32(sQ), kQChunk, 1024);    // MN-major B of dK
-      const uint64_t dDOm = sdesc_sw128(smem_u32(sDO), kQChunk, 1024);  // MN-major B of dV
-      auto issue_sdp = [&](int n) -> bool {  // S^T_n, dP^T_n into buffer n & 1
-        const int s = n % S;
-        const int b = n & 1;
-        if (!mbar_wait(c.bar(B::qdo_full + s), (n / S) & 1, c.wait)) return false;
-        tc_fence_after();
-        const uint32_t so = static_cast<uint32_t>(s) * C::kQ1Bytes;
-        const uint64_t bq = sdesc_add(dQk, so);
-        const uint64_t bdo = sdesc_add(dDOk, so);
+      const uint64_t dQm = sdesc_sw128(smem_u32(sQ), kChunk, 1024);     // MN-major B of dK
+      const uint64_t dDOm = sdesc_sw128(smem_u32(sDO), kChunk, 1024);   // MN-major B of dV
+      auto issue_s = [&](int n) {  // S^T_n (stage resident)
+        const uint64_t bq = sdesc_add(dQk, static_cast<uint32_t>(n % S) * C::kTile);
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
-          const int kk = k * 16;
-          const uint32_t okv = (kk / 64) * kKVChunk + (kk % 64) * 2;
-          const uint32_t oq = (kk / 64) * kQChunk + (kk % 64) * 2;
-          umma_ss(t + 128 * b, sdesc_add(dK, okv), sdesc_add(bq, oq), idesc_sp, k > 0);
+          const uint32_t off = ((k * 16) / 64) * kChunk + ((k * 16) % 64) * 2;
+          umma_ss(t, sdesc_add(dK, off), sdesc_add(bq, off), idesc_sp, k > 0);
         }
-#pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          const int kk = k * 16;
-          const uint32_t okv = (kk / 64) * kKVChunk + (kk % 64) * 2;
-          const uint32_t oq = (kk / 64) * kQChunk + (kk % 64) * 2;
-          umma_ss(t + 128 * b + 64, sdesc_add(dV, okv), sdesc_add(bdo, oq), idesc_sp, k > 0);
-        }
-        umma_commit(c.bar(B::s_full + b));
-        return true;
+        umma_commit(c.bar(B::s_full));
       };
-      bool ok = mbar_wait(c.bar(B::kv_full), 0, c.wait);
-      if (ok) ok = issue_sdp(0);
-      if (ok && len > 1) ok = issue_sdp(1);
+      auto issue_dp = [&](int n) {  // dP^T_n (stage resident)
+        const uint64_t bdo = sdesc_add(dDOk, static_cast<uint32_t>(n % S) * C::kTile);
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t off = ((k * 16) / 64) * kChunk + ((k * 16) % 64) * 2;
+          umma_ss(t + 128, sdesc_add(dV, off), sdesc_add(bdo, off), idesc_sp, k > 0);
+        }
+        umma_commit(c.bar(B::dp_full));
+      };
+      bool ok = mbar_wait(c.bar(B::kv_full), 0, c.wait) && mbar_wait(c.bar(B::qdo_full), 0, c.wait);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0);
+        issue_dp(0);
+      }
       for (int n = 0; ok && n < len; ++n) {
         const int s = n % S;
-        const int b = n & 1;
-        if (!(ok = mbar_wait(c.bar(B::p_full + b), (n >> 1) & 1, c.wait))) break;
+        if (n + 1 < len) {
+          // S^T_{n+1} overwrites S^T_n once the elementwise warps hold it in registers.
+          if (!(ok = mbar_wait(c.bar(B::s_free), n & 1, c.wait))) break;
+          if (!(ok = mbar_wait(c.bar(B::qdo_full + (n + 1) % S), ((n + 1) / S) & 1, c.wait))) break;
+          tc_fence_after();
+          issue_s(n + 1);
+        }
+        if (!(ok = mbar_wait(c.bar(B::p_full), n & 1, c.wait))) break;
         tc_fence_after();
         const uint32_t acc = n > 0 ? 1u : 0u;
-        const uint32_t so = static_cast<uint32_t>(s) * C::kQ1Bytes;
-        const uint64_t bdo = sdesc_add(dDOm, so);
-        const uint64_t bq = sdesc_add(dQm, so);
-        const uint32_t tb = t + 128 * b;
+        const uint64_t bdo = sdesc_add(dDOm, static_cast<uint32_t>(s) * C::kTile);
+        const uint64_t bq = sdesc_add(dQm, static_cast<uint32_t>(s) * C::kTile);
 #pragma unroll
         for (int k = 0; k < kBR / 16; ++k) {
-          // P^T columns of query rows 16k..16k+15 (warpgroup h = k/2 wrote them).
-          umma_ts(t + 256, tb + 32 * (k / 2) + 8 * (k % 2), sdesc_add(bdo, k * 16 * 128), idesc_kv,
+          // P^T columns of query rows 16k..16k+15: warpgroup h = k/4 wrote them at 128 + 64h.
+          umma_ts(t + 256, t + 128 + 64 * (k / 4) + 8 * (k % 4), sdesc_add(bdo, k * 16 * 128), idesc_kv,
                   acc | static_cast<uint32_t>(k > 0));
         }
 #pragma unroll
         for (int k = 0; k < kBR / 16; ++k) {
-          umma_ts(t + 256 + D, tb + 64 + 32 * (k / 2) + 8 * (k % 2), sdesc_add(bq, k * 16 * 128), idesc_kv,
+          umma_ts(t + 256 + D, t + 128 + 64 * (k / 4) + 32 + 8 * (k % 4), sdesc_add(bq, k * 16 * 128), idesc_kv,
                   acc | static_cast<uint32_t>(k > 0));
         }
         umma_commit(c.bar(B::qdo_empty + s));
-        if (n + 2 < len) ok = issue_sdp(n + 2);  // buffer b again: ordered after dV, dK above
+        if (n + 1 < len) issue_dp(n + 1);  // dP^T columns: ordered after dV, dK read P^T, dS^T
       }
       if (ok) umma_commit(c.bar(B::all_done));
     }
@@ -359,62 +367,71 @@ __device__ __forceinline__ void key_cta(const Ctx& c, const Params& p, const CUt
     reg_alloc<kRegsHigh>();
     // ------------------------------------------------------------ elementwise (thread = key row)
     TileCursor cur = c.cursor;
-    const int h = (c.warp - 4) / 4;  // query columns [32h, 32h + 32) of each 64-row tile
+    const int h = (c.warp - 4) / 4;  // query columns [64h, 64h + 64) of each tile
     const int wq = c.warp % 4;
     const int r = wq * 32 + c.lane;
     const int key = j * kBlockN + r;
     const bool key_valid = key < p.N;
-    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t tl = c.tmem + (static_cast<uint32_t>(wq * 32) << 16);
     const float sl2 = p.scale_log2;
-    const int qo = 32 * h;
+    const int qo = 64 * h;
     bool ok = true;
     for (int n = 0; n < len; ++n) {
       const int i = cur.next();
       const int s = n % S;
-      const int b = n & 1;
-      if (!(ok = mbar_wait_warp(c.bar(B::s_full + b), (n >> 1) & 1, c.wait))) break;
-      if (!(ok = mbar_wait_warp(c.bar(B::qdo_full + s), (n / S) & 1, c.wait))) break;  // lse2, D of tile i
+      if (!(ok = mbar_wait_warp(c.bar(B::s_full), n & 1, c.wait))) break;
       tc_fence_after();
-      const uint32_t tS = c.tmem + lane_off + 128 * b;
-      uint32_t sr[32], dr[32];
-      tmem_ld32(tS + qo, sr);
-      tmem_ld32(tS + 64 + qo, dr);
+      uint32_t sr[64];
+      tmem_ld32(tl + qo, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tmem_ld32(tl + qo + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
       tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(c.bar(B::s_free));
+      if (!(ok = mbar_wait_warp(c.bar(B::qdo_full + s), (n / S) & 1, c.wait))) break;  // lse2, D of tile i
       // Columns x < lim are masked (causal: key > query; or the key row lies past N).
       int lim = 0;
       if (!key_valid) {
-        lim = 32;
+        lim = 64;
       } else if (p.causal && j * kBlockN + kBlockN - 1 > i * kBR) {
-        lim = min(32, max(0, key - (i * kBR + qo)));
+        lim = min(64, max(0, key - (i * kBR + qo)));
       }
       const uint32_t aL = smem_u32(sL + s * kBR + qo);
-      const uint32_t aD = smem_u32(sDv + s * kBR + qo);
-      uint32_t pk[16], dk[16];
+      float pv[64];
 #pragma unroll
-      for (int x = 0; x < 32; x += 4) {
+      for (int x = 0; x < 64; x += 4) {
         const float4 l4 = lds128(aL + x * 4);
-        const float4 d4 = lds128(aD + x * 4);
-        float p0 = ex2(fmaf(__uint_as_float(sr[x]), sl2, -l4.x));
-        float p1 = ex2(fmaf(__uint_as_float(sr[x + 1]), sl2, -l4.y));
-        float p2 = ex2(fmaf(__uint_as_float(sr[x + 2]), sl2, -l4.z));
-        float p3 = ex2(fmaf(__uint_as_float(sr[x + 3]), sl2, -l4.w));
-        if (lim > 0) {
-          if (x < lim) p0 = 0.0f;
-          if (x + 1 < lim) p1 = 0.0f;
-          if (x + 2 < lim) p2 = 0.0f;
-          if (x + 3 < lim) p3 = 0.0f;
-        }
-        pk[x / 2] = pack2<BF16>(p0, p1);
-        pk[x / 2 + 1] = pack2<BF16>(p2, p3);
-        dk[x / 2] = pack2<BF16>(p0 * (__uint_as_float(dr[x]) - d4.x), p1 * (__uint_as_float(dr[x + 1]) - d4.y));
-        dk[x / 2 + 1] =
-            pack2<BF16>(p2 * (__uint_as_float(dr[x + 2]) - d4.z), p3 * (__uint_as_float(dr[x + 3]) - d4.w));
+        pv[x] = ex2(fmaf(__uint_as_float(sr[x]), sl2, -l4.x));
+        pv[x + 1] = ex2(fmaf(__uint_as_float(sr[x + 1]), sl2, -l4.y));
+        pv[x + 2] = ex2(fmaf(__uint_as_float(sr[x + 2]), sl2, -l4.z));
+        pv[x + 3] = ex2(fmaf(__uint_as_float(sr[x + 3]), sl2, -l4.w));
       }
-      tmem_st16(tS + 32 * h, pk);
-      tmem_st16(tS + 64 + 32 * h, dk);
+      if (lim > 0) {
+#pragma unroll
+        for (int x = 0; x < 64; ++x)
+          if (x < lim) pv[x] = 0.0f;
+      }
+      if (!(ok = mbar_wait_warp(c.bar(B::dp_full), n & 1, c.wait))) break;
+      tc_fence_after();
+      uint32_t dr[64];
+      tmem_ld32(tl + 128 + qo, *reinterpret_cast<uint32_t(*)[32]>(&dr[0]));
+      tmem_ld32(tl + 128 + qo + 32, *reinterpret_cast<uint32_t(*)[32]>(&dr[32]));
+      tmem_ld_wait();
+      const uint32_t aD = smem_u32(sDv + s * kBR + qo);
+      uint32_t pk[32], dk[32];
+#pragma unroll
+      for (int x = 0; x < 64; x += 4) {
+        const float4 d4 = lds128(aD + x * 4);
+        pk[x / 2] = pack2<BF16>(pv[x], pv[x + 1]);
+        pk[x / 2 + 1] = pack2<BF16>(pv[x + 2], pv[x + 3]);
+        dk[x / 2] = pack2<BF16>(pv[x] * (__uint_as_float(dr[x]) - d4.x), pv[x + 1] * (__uint_as_float(dr[x + 1]) - d4.y));
+        dk[x / 2 + 1] =
+            pack2<BF16>(pv[x + 2] * (__uint_as_float(dr[x + 2]) - d4.z), pv[x + 3] * (__uint_as_float(dr[x + 3]) - d4.w));
+      }
+      tmem_st32(tl + 128 + qo, pk);
+      tmem_st32(tl + 128 + qo + 32, dk);
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(c.bar(B::p_full + b));
+      mbar_arrive(c.bar(B::p_full));
     }
     // Epilogue: warpgroup 0 writes dV_j, warpgroup 1 writes scale * dK_j.
     bool have = false;
@@ -426,7 +443,7 @@ __device__ __forceinline__ void key_cta(const Ctx& c, const Params& p, const CUt
     if (ok) {
       uint16_t* dst = reinterpret_cast<uint16_t*>(h == 0 ? p.dv : p.dk) +
                       (static_cast<size_t>(c.bh) * p.N + (key_valid ? key : 0)) * D;
-      store_row_from_tmem<BF16>(c.tmem + lane_off + 256 + h * D, D, h == 0 ? 1.0f : p.scale, have, key_valid, dst);
+      store_row_from_tmem<BF16>(tl + 256 + h * D, D, h == 0 ? 1.0f : p.scale, have, key_valid, dst);
     }
   }
 }
@@ -434,18 +451,14 @@ __device__ __forceinline__ void key_cta(const Ctx& c, const Params& p, const CUt
 // --------------------------------------------------------------------------- query-stationary CTA
 
 template <int D, bool BF16>
-__device__ __forceinline__ void query_cta(const Ctx& c, const Params& p, const CUtensorMap* tq,
-                                          const CUtensorMap* tk, const CUtensorMap* tv, const CUtensorMap* tdo,
-                                          int i) {
+__device__ __forceinline__ void query_cta(const Ctx& c, const Params& p, const CUtensorMap* tk,
+                                          const CUtensorMap* tv, int i) {
   using C = Cfg<D>;
   using B = QueryBars;
-  constexpr int SK = C::kSK;
-  constexpr int SV = C::kSV;
-  uint8_t* sQ = c.smem + C::k2Q;
-  uint8_t* sDO = c.smem + C::k2DO;
+  constexpr int S = C::kS2;
+  constexpr int kChunk = C::kChunk;
   uint8_t* sK = c.smem + C::k2K;
   uint8_t* sV = c.smem + C::k2V;
-  constexpr int kChunk = 128 * 128;  // 64 columns x 128 rows
   const int len = c.len;
 
   if (c.warp < 4) {
@@ -453,36 +466,23 @@ __device__ __forceinline__ void query_cta(const Ctx& c, const Params& p, const C
     if (c.warp == 0 && c.lane == 0) {
       // ---------------------------------------------------------- producer
       TileCursor cur = c.cursor;
-      int32_t* tr = p.trace ? p.trace + static_cast<size_t>(p.BH) * p.T * (p.Tq1 + 1) +
+      int32_t* tr = p.trace ? p.trace + static_cast<size_t>(p.BH) * p.T * (p.T + 1) +
                                   (static_cast<size_t>(c.bh) * p.T + i) * (p.T + 1)
                             : nullptr;
       if (tr) tr[0] = len;
-      if (len > 0) {
-        mbar_arrive_expect_tx(c.bar(B::q_full), 2 * C::kQ2Bytes);
-        // The Q and dO maps have 64-row boxes: two boxes fill one 128-row chunk.
-        for (int ch = 0; ch < D / 64; ++ch) {
-          for (int hr = 0; hr < 2; ++hr) {
-            tma_load_3d(smem_u32(sQ + ch * kChunk + hr * 64 * 128), tq, c.bar(B::q_full), ch * 64,
-                        i * kBlockQ + hr * 64, c.bh);
-            tma_load_3d(smem_u32(sDO + ch * kChunk + hr * 64 * 128), tdo, c.bar(B::q_full), ch * 64,
-                        i * kBlockQ + hr * 64, c.bh);
-          }
-        }
-      }
       for (int n = 0; n < len; ++n) {
         const int jt = cur.next();
         if (tr) tr[1 + n] = jt | (1 << 16);
-        const int sk = n % SK;
-        if (!mbar_wait(c.bar(B::k_empty + sk), ((n / SK) & 1) ^ 1, c.wait)) break;
-        mbar_arrive_expect_tx(c.bar(B::k_full + sk), C::kKVBytes);
+        const int s = n % S;
+        if (!mbar_wait(c.bar(B::k_empty + s), ((n / S) & 1) ^ 1, c.wait)) break;
+        mbar_arrive_expect_tx(c.bar(B::k_full + s), C::kTile);
         for (int ch = 0; ch < D / 64; ++ch)
-          tma_load_3d(smem_u32(sK + sk * C::kKVBytes + ch * kChunk), tk, c.bar(B::k_full + sk), ch * 64,
+          tma_load_3d(smem_u32(sK + s * C::kTile + ch * kChunk), tk, c.bar(B::k_full + s), ch * 64,
                       jt * kBlockN, c.bh);
-        const int sv = n % SV;
-        if (!mbar_wait(c.bar(B::v_empty + sv), ((n / SV) & 1) ^ 1, c.wait)) break;
-        mbar_arrive_expect_tx(c.bar(B::v_full + sv), C::kKVBytes);
+        if (!mbar_wait(c.bar(B::v_empty + s), ((n / S) & 1) ^ 1, c.wait)) break;
+        mbar_arrive_expect_tx(c.bar(B::v_full + s), C::kTile);
         for (int ch = 0; ch < D / 64; ++ch)
-          tma_load_3d(smem_u32(sV + sv * C::kKVBytes + ch * kChunk), tv, c.bar(B::v_full + sv), ch * 64,
+          tma_load_3d(smem_u32(sV + s * C::kTile + ch * kChunk), tv, c.bar(B::v_full + s), ch * 64,
                       jt * kBlockN, c.bh);
       }
     } else if (c.warp == 1 && c.lane == 0 && len > 0) {
@@ -490,59 +490,59 @@ __device__ __forceinline__ void query_cta(const Ctx& c, const Params& p, const C
       constexpr uint32_t idesc_sp = idesc_f16(BF16, 128, kBlockN, false, false);  // S, dP
       constexpr uint32_t idesc_q = idesc_f16(BF16, 128, D, false, true);          // dQ
       const uint32_t t = c.tmem;
-      // Base descriptors; every MMA below adds a compile-time offset to them.
-      const uint64_t dQ = sdesc_sw128(smem_u32(sQ), 16, 1024);        // K-major A of S
-      const uint64_t dDO = sdesc_sw128(smem_u32(sDO), 16, 1024);      // K-major A of dP
       const uint64_t dKk = sdesc_sw128(smem_u32(sK), 16, 1024);       // K-major B of S
       const uint64_t dVk = sdesc_sw128(smem_u32(sV), 16, 1024);       // K-major B of dP
       const uint64_t dKm = sdesc_sw128(smem_u32(sK), kChunk, 1024);   // MN-major B of dQ
-      auto issue_s = [&](int n) -> bool {  // S_n into buffer n & 1
-        const int sk = n % SK;
-        if (!mbar_wait(c.bar(B::k_full + sk), (n / SK) & 1, c.wait)) return false;
+      auto issue_s = [&](int n) -> bool {  // S_n = Q K_n^T (A: Q in TMEM)
+        const int s = n % S;
+        if (!mbar_wait(c.bar(B::k_full + s), (n / S) & 1, c.wait)) return false;
         tc_fence_after();
-        const uint64_t bk = sdesc_add(dKk, static_cast<uint32_t>(sk) * C::kKVBytes);
+        const uint64_t bk = sdesc_add(dKk, static_cast<uint32_t>(s) * C::kTile);
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
-          const int kk = k * 16;
-          const uint32_t off = (kk / 64) * kChunk + (kk % 64) * 2;
-          umma_ss(t + 128 * (n & 1), sdesc_add(dQ, off), sdesc_add(bk, off), idesc_sp, k > 0);
+          const uint32_t off = ((k * 16) / 64) * kChunk + ((k * 16) % 64) * 2;
+          umma_ts(t + C::kColS2, t + C::kColQ + 8 * k, sdesc_add(bk, off), idesc_sp, k > 0);
         }
-        umma_commit(c.bar(B::s_full + (n & 1)));
+        umma_commit(c.bar(B::s_full));
         return true;
       };
-      auto issue_dp = [&](int n) -> bool {  // dP_n; V_n is released as soon as it completes
-        const int sv = n % SV;
-        if (!mbar_wait(c.bar(B::v_full + sv), (n / SV) & 1, c.wait)) return false;
+      auto issue_dp = [&](int n) -> bool {  // dP_n = dO V_n^T (A: dO in TMEM); V_n released after
+        const int s = n % S;
+        if (!mbar_wait(c.bar(B::v_full + s), (n / S) & 1, c.wait)) return false;
         tc_fence_after();
-        const uint64_t bv = sdesc_add(dVk, static_cast<uint32_t>(sv) * C::kKVBytes);
+        const uint64_t bv = sdesc_add(dVk, static_cast<uint32_t>(s) * C::kTile);
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
-          const int kk = k * 16;
-          const uint32_t off = (kk / 64) * kChunk + (kk % 64) * 2;
-          umma_ss(t + 256, sdesc_add(dDO, off), sdesc_add(bv, off), idesc_sp, k > 0);
+          const uint32_t off = ((k * 16) / 64) * kChunk + ((k * 16) % 64) * 2;
+          umma_ts(t + C::kColDP2, t + C::kColDO + 8 * k, sdesc_add(bv, off), idesc_sp, k > 0);
         }
         umma_commit(c.bar(B::dp_full));
-        umma_commit(c.bar(B::v_empty + sv));
+        umma_commit(c.bar(B::v_empty + s));
         return true;
       };
-      bool ok = mbar_wait(c.bar(B::q_full), 0, c.wait);
-      if (ok) ok = issue_s(0);
-      if (ok) ok = issue_dp(0);
-      if (ok && len > 1) ok = issue_s(1);
-      for (int n = 0; ok && n < len; ++n) {
-        const int sk = n % SK;
-        if (!(ok = mbar_wait(c.bar(B::ds_full), n & 1, c.wait))) break;  // dS_n written, S_n consumed
+      bool ok = mbar_wait(c.bar(B::q_ready), 0, c.wait);
+      if (ok) {
         tc_fence_after();
-        const uint64_t bk = sdesc_add(dKm, static_cast<uint32_t>(sk) * C::kKVBytes);
+        ok = issue_s(0) && issue_dp(0);
+      }
+      for (int n = 0; ok && n < len; ++n) {
+        const int s = n % S;
+        if (n + 1 < len) {
+          // S_{n+1} overwrites S_n once the elementwise warps hold it in registers.
+          if (!(ok = mbar_wait(c.bar(B::s_free), n & 1, c.wait))) break;
+          if (!(ok = issue_s(n + 1))) break;
+        }
+        if (!(ok = mbar_wait(c.bar(B::ds_full), n & 1, c.wait))) break;  // dS_n written over dP_n
+        tc_fence_after();
+        const uint64_t bk = sdesc_add(dKm, static_cast<uint32_t>(s) * C::kTile);
 #pragma unroll
         for (int k = 0; k < kBlockN / 16; ++k) {
-          // dS columns of keys 16k..16k+15 (warpgroup h = k/4 wrote them at 256 + 64h).
-          umma_ts(t + 384, t + 256 + 64 * (k / 4) + 8 * (k % 4), sdesc_add(bk, k * 16 * 128), idesc_q,
-                  (n > 0 || k > 0) ? 1u : 0u);
+          // dS columns of keys 16k..16k+15: warpgroup h = k/4 wrote them at dP + 64h.
+          umma_ts(t + C::kColDQ, t + C::kColDP2 + 64 * (k / 4) + 8 * (k % 4), sdesc_add(bk, k * 16 * 128),
+                  idesc_q, (n > 0 || k > 0) ? 1u : 0u);
         }
-        umma_commit(c.bar(B::k_empty + sk));              // K_n free once dQ_n is done
-        if (ok && n + 1 < len) ok = issue_dp(n + 1);      // dP region: ordered after dQ_n read dS_n
-        if (ok && n + 2 < len) ok = issue_s(n + 2);       // S buffer n & 1: consumed by elementwise n
+        umma_commit(c.bar(B::k_empty + s));               // K_n free once dQ_n is done
+        if (n + 1 < len && !(ok = issue_dp(n + 1))) break;  // dP columns: ordered after dQ_n read dS_n
       }
       if (ok) umma_commit(c.bar(B::all_done));
     }
@@ -555,21 +555,46 @@ __device__ __forceinline__ void query_cta(const Ctx& c, const Params& p, const C
     const int r = wq * 32 + c.lane;
     const int qrow = i * kBlockQ + r;
     const bool row_valid = qrow < p.N;
-    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t tl = c.tmem + (static_cast<uint32_t>(wq * 32) << 16);
     const float sl2 = p.scale_log2;
     const size_t vo = static_cast<size_t>(c.bh) * p.Npad + static_cast<size_t>(i) * kBlockQ + r;
     const float l2 = p.lse2[vo];  // +inf on padding rows: P = 0
     const float dd = p.delta[vo];
+    // Q_i and dO_i rows into TMEM as the A operands of S and dP: warpgroup h
+    // copies its half of the 32-bit words (pairs of 16-bit values) of this row.
+    {
+      const size_t roff = (static_cast<size_t>(c.bh) * p.N + (row_valid ? qrow : 0)) * D;
+      const uint4* gq = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(p.q) + roff);
+      const uint4* gdo = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(p.dout) + roff);
+      constexpr int kWords = D / 4;  // this warpgroup's 32-bit words per row
+#pragma unroll
+      for (int w0 = 0; w0 < kWords; w0 += 16) {
+        uint32_t a[16], b[16];
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const uint4 x = row_valid ? gq[(h * kWords + w0) / 4 + v] : make_uint4(0, 0, 0, 0);
+          const uint4 y = row_valid ? gdo[(h * kWords + w0) / 4 + v] : make_uint4(0, 0, 0, 0);
+          a[4 * v] = x.x; a[4 * v + 1] = x.y; a[4 * v + 2] = x.z; a[4 * v + 3] = x.w;
+          b[4 * v] = y.x; b[4 * v + 1] = y.y; b[4 * v + 2] = y.z; b[4 * v + 3] = y.w;
+        }
+        tmem_st16(tl + C::kColQ + h * kWords + w0, a);
+        tmem_st16(tl + C::kColDO + h * kWords + w0, b);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(c.bar(B::q_ready));
+    }
     bool ok = true;
     for (int n = 0; n < len; ++n) {
       const int jt = cur.next();
-      const int cb = n & 1;
-      if (!(ok = mbar_wait_warp(c.bar(B::s_full + cb), (n >> 1) & 1, c.wait))) break;
+      if (!(ok = mbar_wait_warp(c.bar(B::s_full), n & 1, c.wait))) break;
       tc_fence_after();
       uint32_t sr[64];
-      tmem_ld32(c.tmem + lane_off + 128 * cb + 64 * h, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-      tmem_ld32(c.tmem + lane_off + 128 * cb + 64 * h + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      tmem_ld32(tl + C::kColS2 + 64 * h, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tmem_ld32(tl + C::kColS2 + 64 * h + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
       tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(c.bar(B::s_free));
       // Mask columns x > lim: causal (key > query) and keys past N.
       int lim = 63;
       if (p.causal && jt * kBlockN + 64 * h + 63 > qrow) lim = qrow - jt * kBlockN - 64 * h;
@@ -586,15 +611,15 @@ __device__ __forceinline__ void query_cta(const Ctx& c, const Params& p, const C
       if (!(ok = mbar_wait_warp(c.bar(B::dp_full), n & 1, c.wait))) break;  // dP_n
       tc_fence_after();
       uint32_t dr[64];
-      tmem_ld32(c.tmem + lane_off + 256 + 64 * h, *reinterpret_cast<uint32_t(*)[32]>(&dr[0]));
-      tmem_ld32(c.tmem + lane_off + 256 + 64 * h + 32, *reinterpret_cast<uint32_t(*)[32]>(&dr[32]));
+      tmem_ld32(tl + C::kColDP2 + 64 * h, *reinterpret_cast<uint32_t(*)[32]>(&dr[0]));
+      tmem_ld32(tl + C::kColDP2 + 64 * h + 32, *reinterpret_cast<uint32_t(*)[32]>(&dr[32]));
       tmem_ld_wait();
       uint32_t dk[32];
 #pragma unroll
       for (int x = 0; x < 32; ++x)
         dk[x] = pack2<BF16>(pv[2 * x] * (__uint_as_float(dr[2 * x]) - dd),
                             pv[2 * x + 1] * (__uint_as_float(dr[2 * x + 1]) - dd));
-      tmem_st32(c.tmem + lane_off + 256 + 64 * h, dk);
+      tmem_st32(tl + C::kColDP2 + 64 * h, dk);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(c.bar(B::ds_full));
@@ -609,7 +634,7 @@ __device__ __forceinline__ void query_cta(const Ctx& c, const Params& p, const C
     if (ok) {
       uint16_t* dst = reinterpret_cast<uint16_t*>(p.dq) +
                       (static_cast<size_t>(c.bh) * p.N + (row_valid ? qrow : 0)) * D + h * (D / 2);
-      store_row_from_tmem<BF16>(c.tmem + lane_off + 384 + h * (D / 2), D / 2, p.scale, have, row_valid, dst);
+      store_row_from_tmem<BF16>(tl + C::kColDQ + h * (D / 2), D / 2, p.scale, have, row_valid, dst);
     }
   }
 }
@@ -633,7 +658,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   c.bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
-  int* list_len = reinterpret_cast<int*>(smem + C::kOffMisc + 8);
+  int* tile_count = reinterpret_cast<int*>(smem + C::kOffMisc + 8);
   c.warp = threadIdx.x / 32;
   c.lane = threadIdx.x % 32;
   c.bh = blockIdx.x;
@@ -644,7 +669,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   c.cursor.kind = keys ? 0 : 1;
   c.cursor.tile = tile;
   c.cursor.T = p.T;
-  c.cursor.Tq1 = p.Tq1;
   c.cursor.causal = p.causal;
   c.cursor.pos = c.cursor.first();
 
@@ -653,18 +677,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (keys) {
       using B = KeyBars;
       mbar_init(c.bar(B::kv_full), 1);
-      for (int s = 0; s < C::kS1; ++s) {
+      for (int s = 0; s < 3; ++s) {
         mbar_init(c.bar(B::qdo_full + s), 1);
         mbar_init(c.bar(B::qdo_empty + s), 1);
       }
-      for (int b = 0; b < 2; ++b) {
-        mbar_init(c.bar(B::s_full + b), 1);
-        mbar_init(c.bar(B::p_full + b), 256);
-      }
+      mbar_init(c.bar(B::s_full), 1);
+      mbar_init(c.bar(B::s_free), 256);
+      mbar_init(c.bar(B::dp_full), 1);
+      mbar_init(c.bar(B::p_full), 256);
       mbar_init(c.bar(B::all_done), 1);
     } else {
       using B = QueryBars;
-      mbar_init(c.bar(B::q_full), 1);
+      mbar_init(c.bar(B::q_ready), 256);
       for (int s = 0; s < 3; ++s) {
         mbar_init(c.bar(B::k_full + s), 1);
         mbar_init(c.bar(B::k_empty + s), 1);
@@ -672,7 +696,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(c.bar(B::v_empty + s), 1);
       }
       mbar_init(c.bar(B::s_full), 1);
-      mbar_init(c.bar(B::s_full + 1), 1);
+      mbar_init(c.bar(B::s_free), 256);
       mbar_init(c.bar(B::dp_full), 1);
       mbar_init(c.bar(B::ds_full), 256);
       mbar_init(c.bar(B::all_done), 1);
@@ -687,31 +711,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Number of tiles this CTA visits.
     int count = 0;
     if (p.block_mask != nullptr) {
-      const int range = keys ? p.Tq1 : p.T;
-      for (int base = 0; base < range; base += 32) {
+      for (int base = 0; base < p.T; base += 32) {
         const int x = base + c.lane;
-        const bool use = x < range && c.cursor.allowed(x);
+        const bool use = x < p.T && c.cursor.allowed(x);
         count += __popc(__ballot_sync(0xffffffffu, use));
       }
     } else if (keys) {
-      count = p.Tq1 - c.cursor.first();
-      if (count < 0) count = 0;
+      count = p.T - c.cursor.first();
     } else {
       count = p.causal ? tile + 1 : p.T;
     }
-    if (c.lane == 0) *list_len = count;
+    if (c.lane == 0) *tile_count = count;
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   c.tmem = *tmem_slot;
-  c.len = *list_len;
+  c.len = *tile_count;
   c.wait = WaitCtx{abort_flag, p.status};
 
   if (keys) {
     key_cta<D, BF16>(c, p, &tmap_q, &tmap_k, &tmap_v, &tmap_do, tile);
   } else {
-    query_cta<D, BF16>(c, p, &tmap_q, &tmap_k, &tmap_v, &tmap_do, tile);
+    query_cta<D, BF16>(c, p, &tmap_k, &tmap_v, tile);
   }
 
   tc_fence_before();

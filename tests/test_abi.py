@@ -78,5 +78,5 @@ def test_host_argument_errors_return_before_launch(lib):
 
 def test_trace_sizes(lib):
     assert lib.fa_fwd_trace_size(2, 3, 1000) == 2 * 3 * 4 * (8 + 1)
-    assert lib.fa_bwd_row_tile(64) == 64 and lib.fa_bwd_row_tile(128) == 64
-    assert lib.fa_bwd_trace_size(2, 3, 1000, 128) == 2 * 3 * 8 * ((16 + 1) + (8 + 1))
+    assert lib.fa_bwd_row_tile(64) == 128 and lib.fa_bwd_row_tile(128) == 128
+    assert lib.fa_bwd_trace_size(2, 3, 1000, 128) == 2 * 3 * 8 * ((8 + 1) + (8 + 1))
