@@ -52,9 +52,8 @@ fa_status check_common(fa_dtype dtype, int B, int H, int N, int d) {
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
   const long long bh = static_cast<long long>(B) * H;
   const long long tiles = (static_cast<long long>(N) + 127) / 128;
-  // Grids put batch*heads on one axis and tiles on the other (both <= 65535
-  // here); key-tile indices fit 16 bits.
-  if (bh > 65535 || tiles > 65535) return FA_ERR_UNSUPPORTED;
+  // Grids are 1-D over batch*heads*(2*tiles) CTAs (< 2^31); key-tile indices fit 16 bits.
+  if (bh > 65535 || tiles > 32767 || bh * 2 * tiles > 0x7FFFFFFFLL) return FA_ERR_UNSUPPORTED;
   return FA_OK;
 }
 

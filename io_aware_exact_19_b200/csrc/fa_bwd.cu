@@ -48,6 +48,12 @@ int launch_bwd_t(const AttnArgs& a, cudaStream_t stream) {
   p.T = (a.N + 127) / 128;
   p.causal = a.causal;
   p.scale = a.scale;
+  // Heads per CTA-order group: their Q, dO, K, V (N*d*2 bytes each) fit ~48 MB of L2.
+  {
+    const long long per_head = 8LL * a.N * D;
+    long long g = (48LL << 20) / (per_head > 0 ? per_head : 1);
+    p.head_group = static_cast<int>(g < 1 ? 1 : (g > BH ? BH : g));
+  }
   p.scale_log2 = a.scale * 1.4426950408889634f;
 
   // prep: D/8 threads per padded row.
@@ -71,7 +77,7 @@ int launch_bwd_t(const AttnArgs& a, cudaStream_t stream) {
     auto kern = bwd::fa_bwd_main_kernel<D, BF16>;
     cudaError_t e = host::ensure_dynamic_smem(reinterpret_cast<const void*>(kern), C::kAlloc);
     if (e != cudaSuccess) return static_cast<int>(e);
-    dim3 grid(BH, 2 * p.T);
+    dim3 grid(static_cast<unsigned>(BH) * 2u * static_cast<unsigned>(p.T));
     kern<<<grid, bwd::kThreads, C::kAlloc, stream>>>(tq, tk, tv, tdo, p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return static_cast<int>(e);

@@ -149,6 +149,7 @@ struct Params {
   int Npad;
   int BH;
   int T;  // ceil(N / 128): key tiles, and query tiles
+  int head_group;  // heads walked together (CTA order)
   int causal;
   float scale;
   float scale_log2;
@@ -641,10 +642,10 @@ __device__ __forceinline__ void query_cta(const Ctx& c, const Params& p, const C
 
 // --------------------------------------------------------------------------- main
 
-// grid = (batch*heads, 2*T). blockIdx.y = 2t: key-stationary CTA for key tile t;
-// blockIdx.y = 2t+1: query-stationary CTA for query tile T-1-t. Under a causal
-// mask small key tiles and large query tiles carry the most work, so the
-// heaviest CTAs of both kinds are dispatched first.
+// 1-D grid of batch*heads*2T CTAs walked in groups of heads (grouped_order).
+// Rank 2t: key-stationary CTA for key tile t; rank 2t+1: query-stationary CTA
+// for query tile T-1-t. Under a causal mask small key tiles and large query
+// tiles carry the most work, so the heaviest CTAs of both kinds start first.
 template <int D, bool BF16>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_bwd_main_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
@@ -661,9 +662,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   int* tile_count = reinterpret_cast<int*>(smem + C::kOffMisc + 8);
   c.warp = threadIdx.x / 32;
   c.lane = threadIdx.x % 32;
-  c.bh = blockIdx.x;
-  const bool keys = (blockIdx.y & 1) == 0;
-  const int tile = keys ? static_cast<int>(blockIdx.y >> 1) : p.T - 1 - static_cast<int>(blockIdx.y >> 1);
+  int rank = 0;
+  grouped_order(static_cast<int>(blockIdx.x), p.BH, 2 * p.T, p.head_group, c.bh, rank);
+  const bool keys = (rank & 1) == 0;
+  const int tile = keys ? (rank >> 1) : p.T - 1 - (rank >> 1);
 
   c.cursor.mask = p.block_mask;
   c.cursor.kind = keys ? 0 : 1;

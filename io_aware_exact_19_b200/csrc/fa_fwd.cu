@@ -29,11 +29,17 @@ int launch_fwd_t(const AttnArgs& a, cudaStream_t stream) {
   p.n_pairs = (Tq + 1) / 2;
   p.Tc = (a.N + fwd::kBlockN - 1) / fwd::kBlockN;
   p.causal = a.causal;
+  // Heads per CTA-order group: their K and V (2*N*d*2 bytes each) fit ~48 MB of L2.
+  {
+    const long long per_head = 4LL * a.N * D;
+    long long g = (48LL << 20) / (per_head > 0 ? per_head : 1);
+    p.head_group = static_cast<int>(g < 1 ? 1 : (g > BH ? BH : g));
+  }
   p.scale_log2 = a.scale * 1.4426950408889634f;
   auto kern = fwd::fa_fwd_kernel<D, BF16>;
   cudaError_t e = host::ensure_dynamic_smem(reinterpret_cast<const void*>(kern), L::kAlloc);
   if (e != cudaSuccess) return static_cast<int>(e);
-  dim3 grid(BH, p.n_pairs);
+  dim3 grid(BH * p.n_pairs);
   kern<<<grid, fwd::kThreads, L::kAlloc, stream>>>(tq, tk, tv, p);
   return static_cast<int>(cudaGetLastError());
 }

@@ -57,6 +57,7 @@ struct Params {
   int BH;
   int n_pairs;  // ceil(T_q / 2)
   int Tc;       // ceil(N / 128)
+  int head_group;  // heads walked together (CTA order)
   int causal;
   float scale_log2;  // softmax scale * log2(e)
 };
@@ -122,11 +123,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
-  // Blocks are dispatched x-fastest and x runs over heads, so every head's
-  // heaviest query-tile pair (the last one, under a causal mask) starts first
-  // and the light pairs fill the tail.
-  const int bh = blockIdx.x;
-  const int pair = p.n_pairs - 1 - static_cast<int>(blockIdx.y);
+  // Heads in groups of p.head_group (their K/V stay in L2); inside a group the
+  // heaviest query-tile pairs (the last ones, under a causal mask) start first.
+  int bh, rank;
+  grouped_order(static_cast<int>(blockIdx.x), p.BH, p.n_pairs, p.head_group, bh, rank);
+  const int pair = p.n_pairs - 1 - rank;
   const int q0 = 2 * pair;
   const int Tq = (p.N + kBlockM - 1) / kBlockM;
   const int q1_active = (q0 + 1) < Tq;

@@ -355,6 +355,29 @@ __device__ __forceinline__ void reg_dealloc() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
+// ------------------------------------------------------------------ CTA order
+
+// A 1-D grid of BH * R CTAs (R work items per head, rank 0 the heaviest) is
+// walked in groups of G heads: all ranks of group 0 (rank-major, heads inside),
+// then group 1, and so on. Blocks are dispatched roughly in index order, so the
+// CTAs in flight touch only about G heads' tensors, which stay in L2, while the
+// heaviest items of each group still start first.
+__device__ __forceinline__ void grouped_order(int L, int BH, int R, int G, int& head, int& rank) {
+  const int nfull = BH / G;
+  const long long span = static_cast<long long>(G) * R;
+  if (static_cast<long long>(L) < nfull * span) {
+    const int g = static_cast<int>(L / span);
+    const int rem = static_cast<int>(L - g * span);
+    rank = rem / G;
+    head = g * G + rem % G;
+  } else {
+    const int glast = BH - nfull * G;
+    const int rem = static_cast<int>(L - nfull * span);
+    rank = rem / glast;
+    head = nfull * G + rem % glast;
+  }
+}
+
 // ------------------------------------------------------------------ numerics
 
 __device__ __forceinline__ float ex2(float x) {
