@@ -37,6 +37,8 @@ L2_BYTES = 126 * 1024 * 1024
 WORKLOADS = {
     "long_causal_d128": dict(B=4, H=16, N=4096, d=128, causal=True, fmt="bf16", mask=False,
                              desc="long-context causal attention B=4 H=16 N=4096 d=128 bf16, fwd+bwd"),
+    "tiny_exact": dict(B=1, H=1, N=128, d=64, causal=False, fmt="fp16", mask=False,
+                       desc="tiny exact check B=1 H=1 N=128 d=64 fp16, fwd+bwd (one CTA; latency bound)"),
     "gpt2_small": dict(B=8, H=12, N=1024, d=64, causal=False, fmt="bf16", mask=False,
                        desc="GPT-2-small-shaped attention B=8 H=12 N=1024 d=64 bf16, fwd+bwd"),
     "gpt2_small_causal": dict(B=8, H=12, N=1024, d=64, causal=True, fmt="bf16", mask=False,
@@ -200,6 +202,32 @@ def cpu_rate(w, vals, n_rows, budget_s, min_steps=1, max_steps=None):
     return per_row * n_rows * steps / el / 1e12, steps, el
 
 
+# ----------------------------------------------------------------------------- multi-rank plumbing
+
+def max_over_ranks(values, device=None, world=1):
+    """Element-wise max of a list of floats over all ranks of the default process
+    group (device times are reported as the slowest rank's)."""
+    vals = [float(x) for x in values]
+    if world == 1:
+        return vals
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(vals, dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def whole_job_tflops(flops_per_rank_step, steps, world, ms_max):
+    """Throughput of the whole job: every rank processes its own batch of the same
+    size (weak scaling), so total work over the slowest rank's time."""
+    return world * flops_per_rank_step * steps / (ms_max * 1e-3) / 1e12
+
+
+def rank_seed(rank):
+    """Seed of a rank's synthetic batch: each rank draws an independent batch."""
+    return rank
+
+
 # ----------------------------------------------------------------------------- reference arm
 
 def run_reference(args, w, rank, world):
@@ -208,13 +236,13 @@ def run_reference(args, w, rank, world):
     vals = oracle_inputs(w, list(range(min(4, w["B"] * w["H"]))))
     f_fwd, f_bwd = step_flops(w)
     per_row = (f_fwd + f_bwd) / (w["B"] * w["H"] * w["N"])
-    # Size the per-step sample so warm-up plus timed steps stay within about two minutes.
+    # Size the per-step sample so warm-up plus timed steps stay within the budget.
     rows = sample_rows_for(w, 64)
     t0 = time.perf_counter()
     oracle_sample_step(vals, w, rows, 0)
     t_probe = max(time.perf_counter() - t0, 1e-4)
     n_rows = 64
-    target = 120.0 / max(1, args.steps + args.warmup)
+    target = args.reference_seconds / max(1, args.steps + args.warmup)
     while n_rows < min(w["N"], 2048) and t_probe * (2 * n_rows) / 64 <= target:
         n_rows *= 2
     rows = sample_rows_for(w, n_rows)
@@ -239,11 +267,21 @@ def run_reference(args, w, rank, world):
     return 0
 
 
+def input_bytes(w):
+    return 4 * w["B"] * w["H"] * w["N"] * w["d"] * 2
+
+
+def needs_l2_flush(w):
+    """Inputs under twice the L2 size could stay cached between steps: flush instead."""
+    return input_bytes(w) < 2 * L2_BYTES
+
+
 def config_block(w, name):
+    l2 = (f"L2 flushed between steps ({2 * L2_BYTES >> 20} MiB write outside the timed events); "
+          if needs_l2_flush(w) else "inputs larger than L2 (no flush): ")
     return {"workload": w["desc"], "name": name, "B": w["B"], "H": w["H"], "N": w["N"], "d": w["d"],
             "causal": w["causal"], "block_sparse": w["mask"], "dtype": w["fmt"],
-            "l2": "inputs larger than L2 (no flush): " + str(
-                round(4 * w["B"] * w["H"] * w["N"] * w["d"] * 2 / 2 ** 20)) + " MiB of Q/K/V/dO per step",
+            "l2": l2 + str(round(input_bytes(w) / 2 ** 20)) + " MiB of Q/K/V/dO per step",
             "parallelism": "one independent batch per GPU"}
 
 
@@ -263,7 +301,7 @@ def run_gpu(args, w, rank, world, local_rank):
     causal = w["causal"]
     tdt = torch.bfloat16 if w["fmt"] == "bf16" else torch.float16
 
-    bits = fa_synth.attention_input_bits(B, H, N, d, w["fmt"], seed=rank)
+    bits = fa_synth.attention_input_bits(B, H, N, d, w["fmt"], seed=rank_seed(rank))
     host = {n: torch.from_numpy(b.view(np.int16)).view(tdt) for n, b in bits.items()}
     q, k, v, do = (host[n].to(dev) for n in ("q", "k", "v", "do"))
     mask = None
@@ -312,7 +350,10 @@ def run_gpu(args, w, rank, world, local_rank):
         dist.barrier()
     torch.cuda.synchronize()
     t_wall0 = time.time()
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev) if needs_l2_flush(w) else None
     for s in range(args.steps):
+        if flush is not None:
+            flush.fill_(s & 0xFF)
         step(events[s])
     torch.cuda.synchronize()
     t_wall1 = time.time()
@@ -323,19 +364,16 @@ def run_gpu(args, w, rank, world, local_rank):
     clocks = sampler.summary(t_wall0, t_wall1)
     status = fa.fa_device_status()
 
-    ms_total = events[0][0].elapsed_time(events[-1][3])
+    # Sum of the per-step spans (first to last launch of each step): the L2 flush
+    # between steps, where there is one, stays outside.
+    ms_total = sum(e[0].elapsed_time(e[3]) for e in events)
     fwd_ms = [e[0].elapsed_time(e[1]) for e in events]
     prep_ms = [e[1].elapsed_time(e[2]) for e in events]
     main_ms = [e[2].elapsed_time(e[3]) for e in events]
-    if world > 1:
-        t = torch.tensor([ms_total, sum(main_ms), sum(fwd_ms)], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total, main_sum, fwd_sum = (float(x) for x in t.tolist())
-    else:
-        main_sum, fwd_sum = sum(main_ms), sum(fwd_ms)
+    ms_total, main_sum, fwd_sum = max_over_ranks([ms_total, sum(main_ms), sum(fwd_ms)], dev, world)
 
     f_fwd, f_bwd = step_flops(w)
-    value = world * (f_fwd + f_bwd) * args.steps / (ms_total * 1e-3) / 1e12
+    value = whole_job_tflops(f_fwd + f_bwd, args.steps, world, ms_total)
     peaks = load_peaks()
     main_avg = main_sum / args.steps
     fwd_avg = fwd_sum / args.steps
@@ -373,14 +411,10 @@ def run_gpu(args, w, rank, world, local_rank):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks([e0.elapsed_time(e1)], dev, world)[0]
     h2d = sum(t.numel() * t.element_size() for t in pin.values())
     d2h = sum(t.numel() * t.element_size() for t in out_host.values())
-    e2e_value = world * (f_fwd + f_bwd) * e2e_steps / (e2e_ms * 1e-3) / 1e12
+    e2e_value = whole_job_tflops(f_fwd + f_bwd, e2e_steps, world, e2e_ms)
 
     if rank != 0:
         return 0
@@ -401,7 +435,9 @@ def run_gpu(args, w, rank, world, local_rank):
         "config": config_block(w, args.workload),
         "roofline": {"kernel": kernel_key, "bound": "tensor", "achieved": achieved, "peak": peaks["bf16"],
                      "unit": UNIT, "frac": achieved / peaks["bf16"],
-                     "peak_source": f"{peaks['source']} bf16 dense burst", "traffic": load_traffic(kernel_key),
+                     "peak_source": f"{peaks['source']} bf16 dense burst" + (
+                         "; fp16 MMAs run at the bf16 rate (nominal ratio 1)" if w["fmt"] == "fp16" else ""),
+                     "traffic": load_traffic(kernel_key),
                      "flops_per_launch": f_bwd},
         "breakdown": {
             "fwd_ms": fwd_avg, "fwd_tflops": f_fwd / (fwd_avg * 1e-3) / 1e12,
@@ -430,11 +466,13 @@ def run_gpu(args, w, rank, world, local_rank):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--reference-seconds", type=float, default=120.0,
+                    help="approximate CPU time budget of the reference arm (warm-up plus timed steps)")
     args = ap.parse_args(argv)
     w = WORKLOADS[args.workload]
     rank = int(os.environ.get("RANK", "0"))
