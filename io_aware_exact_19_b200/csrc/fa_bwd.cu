@@ -66,19 +66,26 @@ int launch_bwd_t(const AttnArgs& a, cudaStream_t stream) {
   }
   // main
   if (a.phases & 2) {
-    CUtensorMap tq, tk, tv, tdo;
+    CUtensorMap tq, tk, tv, tdo, tdq, tdk, tdv;
     // Q and dO are read by key-stationary CTAs in 128-row tiles, loaded as two
-    // 64-row boxes per 64-column chunk.
+    // 64-row boxes per 64-column chunk. dK, dV and dQ are written by each warp in
+    // 32-row boxes: 64 columns with the 128-byte swizzle, or (dQ at d = 64, where
+    // a warpgroup owns 32 columns) 32 columns unswizzled.
+    const bool dq64 = D / 2 >= 64;
     bool ok = host::make_map_3d(&tq, dt, 2, a.q, D, a.N, BH, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B) &&
               host::make_map_3d(&tdo, dt, 2, a.dout, D, a.N, BH, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B) &&
               host::make_map_3d(&tk, dt, 2, a.k, D, a.N, BH, 64, bwd::kBlockN, CU_TENSOR_MAP_SWIZZLE_128B) &&
-              host::make_map_3d(&tv, dt, 2, a.v, D, a.N, BH, 64, bwd::kBlockN, CU_TENSOR_MAP_SWIZZLE_128B);
+              host::make_map_3d(&tv, dt, 2, a.v, D, a.N, BH, 64, bwd::kBlockN, CU_TENSOR_MAP_SWIZZLE_128B) &&
+              host::make_map_3d(&tdk, dt, 2, a.dk, D, a.N, BH, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B) &&
+              host::make_map_3d(&tdv, dt, 2, a.dv, D, a.N, BH, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B) &&
+              host::make_map_3d(&tdq, dt, 2, a.dq, D, a.N, BH, dq64 ? 64 : 32, 32,
+                                dq64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE);
     if (!ok) return static_cast<int>(cudaErrorInvalidValue);
     auto kern = bwd::fa_bwd_main_kernel<D, BF16>;
     cudaError_t e = host::ensure_dynamic_smem(reinterpret_cast<const void*>(kern), C::kAlloc);
     if (e != cudaSuccess) return static_cast<int>(e);
     dim3 grid(static_cast<unsigned>(BH) * 2u * static_cast<unsigned>(p.T));
-    kern<<<grid, bwd::kThreads, C::kAlloc, stream>>>(tq, tk, tv, tdo, p);
+    kern<<<grid, bwd::kThreads, C::kAlloc, stream>>>(tq, tk, tv, tdo, tdq, tdk, tdv, p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return static_cast<int>(e);
   }

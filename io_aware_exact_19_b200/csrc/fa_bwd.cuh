@@ -223,12 +223,24 @@ struct Ctx {
   __device__ __forceinline__ uint32_t bar(int i) const { return smem_u32(&bars[i]); }
 };
 
-// Write `ncols` fp32 TMEM columns of this thread's lane, scaled by `mul`, to a
-// 16-bit row in global memory (zeros if `have` is false; nothing if !valid).
-template <bool BF16>
-__device__ __forceinline__ void store_row_from_tmem(uint32_t taddr, int ncols, float mul, bool have, bool valid,
-                                                    uint16_t* dst) {
-  for (int c = 0; c < ncols; c += 32) {
+// Round NCOLS fp32 TMEM columns of this thread's lane, times `mul`, to 16-bit
+// values (zeros if `have` is false) and write the warp's 32 rows with TMA through
+// shared memory: boxes of 64 columns x 32 rows in the 128-byte-swizzled layout
+// (NCOLS = 64 or 128), or one unswizzled box of 32 columns (NCOLS = 32). `stage`
+// is the warp's own staging area (32 * NCOLS * 2 bytes, 1024-byte aligned). The
+// rows go to columns [col0, col0 + NCOLS) of rows [row0, row0 + 32) of head
+// `bh`; the store clips rows past N. Lane 0 commits one bulk group, which the
+// caller waits for before the CTA exits.
+template <bool BF16, int NCOLS>
+__device__ __forceinline__ void store_rows_tma(uint32_t taddr, float mul, bool have, uint32_t stage,
+                                               const CUtensorMap* map, int col0, int row0, int bh, int N) {
+  const uint32_t lane = threadIdx.x & 31u;
+  constexpr int kBoxCols = NCOLS >= 64 ? 64 : NCOLS;
+  constexpr uint32_t kRowBytes = kBoxCols * 2;
+  constexpr uint32_t kBoxBytes = 32 * kRowBytes;
+  constexpr bool kSwizzle = kBoxCols == 64;
+#pragma unroll
+  for (int c = 0; c < NCOLS; c += 32) {
     uint32_t v[32];
     if (have) {
       tmem_ld32(taddr + c, v);
@@ -238,13 +250,21 @@ __device__ __forceinline__ void store_row_from_tmem(uint32_t taddr, int ncols, f
 #pragma unroll
     for (int x = 0; x < 16; ++x)
       w[x] = have ? pack2<BF16>(__uint_as_float(v[2 * x]) * mul, __uint_as_float(v[2 * x + 1]) * mul) : 0u;
-    if (valid) {
-      uint4* o4 = reinterpret_cast<uint4*>(dst + c);
-      o4[0] = make_uint4(w[0], w[1], w[2], w[3]);
-      o4[1] = make_uint4(w[4], w[5], w[6], w[7]);
-      o4[2] = make_uint4(w[8], w[9], w[10], w[11]);
-      o4[3] = make_uint4(w[12], w[13], w[14], w[15]);
+    const uint32_t row_addr = stage + static_cast<uint32_t>(c / kBoxCols) * kBoxBytes + lane * kRowBytes;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      uint32_t chunk = static_cast<uint32_t>((c % kBoxCols) / 8 + k);
+      if (kSwizzle) chunk ^= lane & 7u;
+      sts128(row_addr + chunk * 16, w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
     }
+  }
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0 && row0 < N) {
+#pragma unroll
+    for (int b = 0; b < NCOLS / kBoxCols; ++b)
+      tma_store_3d(map, stage + static_cast<uint32_t>(b) * kBoxBytes, col0 + b * kBoxCols, row0, bh);
+    bulk_commit_group();
   }
 }
 
@@ -252,7 +272,8 @@ __device__ __forceinline__ void store_row_from_tmem(uint32_t taddr, int ncols, f
 
 template <int D, bool BF16>
 __device__ __forceinline__ void key_cta(const Ctx& c, const Params& p, const CUtensorMap* tq, const CUtensorMap* tk,
-                                        const CUtensorMap* tv, const CUtensorMap* tdo, int j) {
+                                        const CUtensorMap* tv, const CUtensorMap* tdo, const CUtensorMap* tdk,
+                                        const CUtensorMap* tdv, int j) {
   using C = Cfg<D>;
   using B = KeyBars;
   constexpr int S = C::kS1;
@@ -434,7 +455,8 @@ __device__ __forceinline__ void key_cta(const Ctx& c, const Params& p, const CUt
       tc_fence_before();
       mbar_arrive(c.bar(B::p_full));
     }
-    // Epilogue: warpgroup 0 writes dV_j, warpgroup 1 writes scale * dK_j.
+    // Epilogue: warpgroup 0 writes dV_j, warpgroup 1 writes scale * dK_j, staged in
+    // the Q/dO ring (free once the last MMA, which read the last stage, completed).
     bool have = false;
     if (ok && len > 0) {
       ok = mbar_wait_warp(c.bar(B::all_done), 0, c.wait);
@@ -442,10 +464,11 @@ __device__ __forceinline__ void key_cta(const Ctx& c, const Params& p, const CUt
     }
     tc_fence_after();
     if (ok) {
-      uint16_t* dst = reinterpret_cast<uint16_t*>(h == 0 ? p.dv : p.dk) +
-                      (static_cast<size_t>(c.bh) * p.N + (key_valid ? key : 0)) * D;
-      store_row_from_tmem<BF16>(tl + 256 + h * D, D, h == 0 ? 1.0f : p.scale, have, key_valid, dst);
+      const uint32_t stage = smem_u32(sQ) + static_cast<uint32_t>(c.warp - 4) * (32 * D * 2);
+      store_rows_tma<BF16, D>(tl + 256 + h * D, h == 0 ? 1.0f : p.scale, have, stage, h == 0 ? tdv : tdk, 0,
+                              j * kBlockN + wq * 32, c.bh, p.N);
     }
+    if (c.lane == 0) bulk_wait_group<0>();
   }
 }
 
@@ -453,7 +476,7 @@ __device__ __forceinline__ void key_cta(const Ctx& c, const Params& p, const CUt
 
 template <int D, bool BF16>
 __device__ __forceinline__ void query_cta(const Ctx& c, const Params& p, const CUtensorMap* tk,
-                                          const CUtensorMap* tv, int i) {
+                                          const CUtensorMap* tv, const CUtensorMap* tdq, int i) {
   using C = Cfg<D>;
   using B = QueryBars;
   constexpr int S = C::kS2;
@@ -625,7 +648,8 @@ __device__ __forceinline__ void query_cta(const Ctx& c, const Params& p, const C
       tc_fence_before();
       mbar_arrive(c.bar(B::ds_full));
     }
-    // Epilogue: warpgroup h writes columns [h*D/2, (h+1)*D/2) of scale * dQ_i.
+    // Epilogue: warpgroup h writes columns [h*D/2, (h+1)*D/2) of scale * dQ_i,
+    // staged in the K ring (free once the last dQ MMA, which read it, completed).
     bool have = false;
     if (ok && len > 0) {
       ok = mbar_wait_warp(c.bar(B::all_done), 0, c.wait);
@@ -633,10 +657,11 @@ __device__ __forceinline__ void query_cta(const Ctx& c, const Params& p, const C
     }
     tc_fence_after();
     if (ok) {
-      uint16_t* dst = reinterpret_cast<uint16_t*>(p.dq) +
-                      (static_cast<size_t>(c.bh) * p.N + (row_valid ? qrow : 0)) * D + h * (D / 2);
-      store_row_from_tmem<BF16>(tl + C::kColDQ + h * (D / 2), D / 2, p.scale, have, row_valid, dst);
+      const uint32_t stage = smem_u32(sK) + static_cast<uint32_t>(c.warp - 4) * (32 * (D / 2) * 2);
+      store_rows_tma<BF16, D / 2>(tl + C::kColDQ + h * (D / 2), p.scale, have, stage, tdq, h * (D / 2),
+                                  i * kBlockQ + wq * 32, c.bh, p.N);
     }
+    if (c.lane == 0) bulk_wait_group<0>();
   }
 }
 
@@ -650,7 +675,8 @@ template <int D, bool BF16>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_bwd_main_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                        const __grid_constant__ CUtensorMap tmap_v, const __grid_constant__ CUtensorMap tmap_do,
-                       const Params p) {
+                       const __grid_constant__ CUtensorMap tmap_dq, const __grid_constant__ CUtensorMap tmap_dk,
+                       const __grid_constant__ CUtensorMap tmap_dv, const Params p) {
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -733,9 +759,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   c.wait = WaitCtx{abort_flag, p.status};
 
   if (keys) {
-    key_cta<D, BF16>(c, p, &tmap_q, &tmap_k, &tmap_v, &tmap_do, tile);
+    key_cta<D, BF16>(c, p, &tmap_q, &tmap_k, &tmap_v, &tmap_do, &tmap_dk, &tmap_dv, tile);
   } else {
-    query_cta<D, BF16>(c, p, &tmap_k, &tmap_v, tile);
+    query_cta<D, BF16>(c, p, &tmap_k, &tmap_v, &tmap_dq, tile);
   }
 
   tc_fence_before();

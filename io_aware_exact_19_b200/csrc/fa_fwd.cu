@@ -12,10 +12,12 @@ int launch_fwd_t(const AttnArgs& a, cudaStream_t stream) {
   using L = fwd::Smem<D>;
   const int BH = a.B * a.H;
   const CUtensorMapDataType dt = BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
+  // O is written by 64-column x 32-row boxes, one per warp and 64 columns.
   bool ok = host::make_map_3d(&tq, dt, 2, a.q, D, a.N, BH, 64, fwd::kBlockM, CU_TENSOR_MAP_SWIZZLE_128B) &&
             host::make_map_3d(&tk, dt, 2, a.k, D, a.N, BH, 64, fwd::kBlockN, CU_TENSOR_MAP_SWIZZLE_128B) &&
-            host::make_map_3d(&tv, dt, 2, a.v, D, a.N, BH, 64, fwd::kBlockN, CU_TENSOR_MAP_SWIZZLE_128B);
+            host::make_map_3d(&tv, dt, 2, a.v, D, a.N, BH, 64, fwd::kBlockN, CU_TENSOR_MAP_SWIZZLE_128B) &&
+            host::make_map_3d(&to, dt, 2, a.o, D, a.N, BH, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B);
   if (!ok) return static_cast<int>(cudaErrorInvalidValue);
   fwd::Params p;
   p.o = const_cast<void*>(a.o);
@@ -40,7 +42,7 @@ int launch_fwd_t(const AttnArgs& a, cudaStream_t stream) {
   cudaError_t e = host::ensure_dynamic_smem(reinterpret_cast<const void*>(kern), L::kAlloc);
   if (e != cudaSuccess) return static_cast<int>(e);
   dim3 grid(BH * p.n_pairs);
-  kern<<<grid, fwd::kThreads, L::kAlloc, stream>>>(tq, tk, tv, p);
+  kern<<<grid, fwd::kThreads, L::kAlloc, stream>>>(tq, tk, tv, to, p);
   return static_cast<int>(cudaGetLastError());
 }
 

@@ -101,7 +101,8 @@ struct TileList {
 template <int D, bool BF16>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
-                  const __grid_constant__ CUtensorMap tmap_v, const Params p) {
+                  const __grid_constant__ CUtensorMap tmap_v, const __grid_constant__ CUtensorMap tmap_o,
+                  const Params p) {
   using L = Smem<D>;
   constexpr int S = L::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -422,18 +423,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++count;
       }
 
-      // Epilogue: O / l and lse for the rows of this tile that exist.
+      // Epilogue: O / l and lse for the rows of this tile that exist. Each warp
+      // rounds its 32 rows into shared memory, in the 128-byte-swizzled layout of a
+      // 64-column x 32-row TMA box, and writes them with one TMA store per box;
+      // rows past N are clipped by the store. The K/V ring is free by now: every
+      // load has landed and the last P V MMA, which read the last V, has completed.
       bool have_o = false;
       if (ok && count > 0) {
         ok = mbar_wait_warp(bar_o_full(q), 0, ctx);
         have_o = ok;
+      } else if (ok && tl.len > 0) {
+        // No key tile for this query tile (block-sparse): the other tile used them
+        // all; its completion frees the K/V ring used for staging.
+        ok = mbar_wait_warp(bar_o_full(1 - q), 0, ctx);
       }
       tc_fence_after();
       const size_t row_base = static_cast<size_t>(bh) * p.N;
       const bool row_valid = row < p.N;
       const float inv_l = (l_sum > 0.0f) ? 1.0f / l_sum : 0.0f;
-      uint16_t* orow = reinterpret_cast<uint16_t*>(p.o) + (row_base + (row_valid ? row : 0)) * D;
       if (ok) {
+        constexpr uint32_t kBoxBytes = 32 * 128;  // 32 rows x 64 columns x 2 bytes
+        const uint32_t stage = smem_u32(sK) + static_cast<uint32_t>(warp - 4) * (D / 64) * kBoxBytes;
 #pragma unroll
         for (int c = 0; c < D; c += 32) {
           uint32_t o[32];
@@ -448,13 +458,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float b = have_o ? __uint_as_float(o[2 * i + 1]) * inv_l : 0.0f;
             w[i] = pack2<BF16>(a, b);
           }
-          if (row_valid) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + c);
-            dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-            dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-            dst[2] = make_uint4(w[8], w[9], w[10], w[11]);
-            dst[3] = make_uint4(w[12], w[13], w[14], w[15]);
+          // Columns c..c+31 are 16-byte chunks 4*((c/32)%2) .. +3 of the row in box c/64.
+          const uint32_t row_addr = stage + static_cast<uint32_t>(c / 64) * kBoxBytes + lane * 128;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint32_t chunk = static_cast<uint32_t>(((c % 64) / 8 + k) ^ (lane & 7));
+            sts128(row_addr + chunk * 16, w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
           }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        const int row0 = qt * kBlockM + wq * 32;
+        if (lane == 0 && row0 < p.N) {
+#pragma unroll
+          for (int b = 0; b < D / 64; ++b)
+            tma_store_3d(&tmap_o, stage + b * kBoxBytes, b * 64, row0, bh);
+          bulk_commit_group();
         }
         if (row_valid) {
           const float lse = (l_sum > 0.0f) ? (m_ref + lg2(l_sum)) * 0.6931471805599453f : -INFINITY;
@@ -462,6 +481,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
+    // The stores read shared memory asynchronously: let them finish before exit.
+    if (lane == 0) bulk_wait_group<0>();
   }
 
   tc_fence_before();
