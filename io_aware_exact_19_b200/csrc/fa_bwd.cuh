@@ -591,18 +591,19 @@ __device__ __forceinline__ void query_cta(const Ctx& c, const Params& p, const C
       const uint4* gq = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(p.q) + roff);
       const uint4* gdo = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(p.dout) + roff);
       constexpr int kWords = D / 4;  // this warpgroup's 32-bit words per row
+      // All loads first, then the TMEM stores: one memory round trip.
+      uint32_t a[kWords], b[kWords];
+#pragma unroll
+      for (int v = 0; v < kWords / 4; ++v) {
+        const uint4 x = row_valid ? gq[h * kWords / 4 + v] : make_uint4(0, 0, 0, 0);
+        const uint4 y = row_valid ? gdo[h * kWords / 4 + v] : make_uint4(0, 0, 0, 0);
+        a[4 * v] = x.x; a[4 * v + 1] = x.y; a[4 * v + 2] = x.z; a[4 * v + 3] = x.w;
+        b[4 * v] = y.x; b[4 * v + 1] = y.y; b[4 * v + 2] = y.z; b[4 * v + 3] = y.w;
+      }
 #pragma unroll
       for (int w0 = 0; w0 < kWords; w0 += 16) {
-        uint32_t a[16], b[16];
-#pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          const uint4 x = row_valid ? gq[(h * kWords + w0) / 4 + v] : make_uint4(0, 0, 0, 0);
-          const uint4 y = row_valid ? gdo[(h * kWords + w0) / 4 + v] : make_uint4(0, 0, 0, 0);
-          a[4 * v] = x.x; a[4 * v + 1] = x.y; a[4 * v + 2] = x.z; a[4 * v + 3] = x.w;
-          b[4 * v] = y.x; b[4 * v + 1] = y.y; b[4 * v + 2] = y.z; b[4 * v + 3] = y.w;
-        }
-        tmem_st16(tl + C::kColQ + h * kWords + w0, a);
-        tmem_st16(tl + C::kColDO + h * kWords + w0, b);
+        tmem_st16(tl + C::kColQ + h * kWords + w0, *reinterpret_cast<uint32_t(*)[16]>(&a[w0]));
+        tmem_st16(tl + C::kColDO + h * kWords + w0, *reinterpret_cast<uint32_t(*)[16]>(&b[w0]));
       }
       tmem_st_wait();
       tc_fence_before();
