@@ -101,7 +101,7 @@ struct KeyBars {
 };
 struct QueryBars {
   static constexpr int q_ready = 0, k_full = 1, k_empty = 4, v_full = 7, v_empty = 10, s_full = 13,
-                       s_free = 14, dp_full = 15, ds_full = 16, all_done = 17;
+                       s_free = 14, dp_full = 15, ds_full = 16, all_done = 17, qdo_in = 18;
 };
 
 // Walks the tiles one CTA visits, in ascending order. Dense and causal ranges
@@ -475,8 +475,9 @@ __device__ __forceinline__ void key_cta(const Ctx& c, const Params& p, const CUt
 // --------------------------------------------------------------------------- query-stationary CTA
 
 template <int D, bool BF16>
-__device__ __forceinline__ void query_cta(const Ctx& c, const Params& p, const CUtensorMap* tk,
-                                          const CUtensorMap* tv, const CUtensorMap* tdq, int i) {
+__device__ __forceinline__ void query_cta(const Ctx& c, const Params& p, const CUtensorMap* tq,
+                                          const CUtensorMap* tk, const CUtensorMap* tv, const CUtensorMap* tdo,
+                                          const CUtensorMap* tdq, int i) {
   using C = Cfg<D>;
   using B = QueryBars;
   constexpr int S = C::kS2;
@@ -484,6 +485,10 @@ __device__ __forceinline__ void query_cta(const Ctx& c, const Params& p, const C
   uint8_t* sK = c.smem + C::k2K;
   uint8_t* sV = c.smem + C::k2V;
   const int len = c.len;
+  // At d = 128, Q_i and dO_i (256-byte rows) are staged through shared memory by
+  // TMA: per-thread row loads from global memory would touch 32 rows per warp
+  // instruction. At d = 64 the rows are read directly (measured faster there).
+  constexpr bool kStageQdo = D == 128;
 
   if (c.warp < 4) {
     reg_dealloc<kRegsLow>();
@@ -494,10 +499,22 @@ __device__ __forceinline__ void query_cta(const Ctx& c, const Params& p, const C
                                   (static_cast<size_t>(c.bh) * p.T + i) * (p.T + 1)
                             : nullptr;
       if (tr) tr[0] = len;
+      if constexpr (kStageQdo) {
+        // Q_i and dO_i land in the last K and V stages, which the elementwise warps
+        // copy into TMEM before those stages first take K and V.
+        mbar_arrive_expect_tx(c.bar(B::qdo_in), 2 * C::kTile);
+        for (int ch = 0; ch < D / 64; ++ch)
+          for (int hr = 0; hr < 2; ++hr) {
+            const uint32_t off = (S - 1) * C::kTile + ch * kChunk + hr * 64 * 128;
+            tma_load_3d(smem_u32(sK + off), tq, c.bar(B::qdo_in), ch * 64, i * kBlockQ + hr * 64, c.bh);
+            tma_load_3d(smem_u32(sV + off), tdo, c.bar(B::qdo_in), ch * 64, i * kBlockQ + hr * 64, c.bh);
+          }
+      }
       for (int n = 0; n < len; ++n) {
         const int jt = cur.next();
         if (tr) tr[1 + n] = jt | (1 << 16);
         const int s = n % S;
+        if (kStageQdo && n == S - 1 && !mbar_wait(c.bar(B::q_ready), 0, c.wait)) break;
         if (!mbar_wait(c.bar(B::k_empty + s), ((n / S) & 1) ^ 1, c.wait)) break;
         mbar_arrive_expect_tx(c.bar(B::k_full + s), C::kTile);
         for (int ch = 0; ch < D / 64; ++ch)
@@ -587,18 +604,38 @@ __device__ __forceinline__ void query_cta(const Ctx& c, const Params& p, const C
     // Q_i and dO_i rows into TMEM as the A operands of S and dP: warpgroup h
     // copies its half of the 32-bit words (pairs of 16-bit values) of this row.
     {
-      const size_t roff = (static_cast<size_t>(c.bh) * p.N + (row_valid ? qrow : 0)) * D;
-      const uint4* gq = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(p.q) + roff);
-      const uint4* gdo = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(p.dout) + roff);
       constexpr int kWords = D / 4;  // this warpgroup's 32-bit words per row
-      // All loads first, then the TMEM stores: one memory round trip.
       uint32_t a[kWords], b[kWords];
+      if constexpr (kStageQdo) {
+        // From the staged tiles (128-byte swizzle: 16-byte piece x of row r sits at
+        // x ^ (r % 8)); rows past N arrive as zeros.
+        const bool ok_in = mbar_wait_warp(c.bar(B::qdo_in), 0, c.wait);
+        const uint32_t q_base = smem_u32(sK) + (S - 1) * C::kTile;
+        const uint32_t do_base = smem_u32(sV) + (S - 1) * C::kTile;
 #pragma unroll
-      for (int v = 0; v < kWords / 4; ++v) {
-        const uint4 x = row_valid ? gq[h * kWords / 4 + v] : make_uint4(0, 0, 0, 0);
-        const uint4 y = row_valid ? gdo[h * kWords / 4 + v] : make_uint4(0, 0, 0, 0);
-        a[4 * v] = x.x; a[4 * v + 1] = x.y; a[4 * v + 2] = x.z; a[4 * v + 3] = x.w;
-        b[4 * v] = y.x; b[4 * v + 1] = y.y; b[4 * v + 2] = y.z; b[4 * v + 3] = y.w;
+        for (int v = 0; v < kWords / 4; ++v) {
+          const int col = h * (D / 2) + 8 * v;  // first of the 8 columns of this 16-byte piece
+          const uint32_t off = static_cast<uint32_t>((col / 64) * kChunk + r * 128 +
+                                                     ((((col % 64) / 8) ^ (r & 7)) * 16));
+          const float4 x = ok_in ? lds128(q_base + off) : make_float4(0.f, 0.f, 0.f, 0.f);
+          const float4 y = ok_in ? lds128(do_base + off) : make_float4(0.f, 0.f, 0.f, 0.f);
+          a[4 * v] = __float_as_uint(x.x); a[4 * v + 1] = __float_as_uint(x.y);
+          a[4 * v + 2] = __float_as_uint(x.z); a[4 * v + 3] = __float_as_uint(x.w);
+          b[4 * v] = __float_as_uint(y.x); b[4 * v + 1] = __float_as_uint(y.y);
+          b[4 * v + 2] = __float_as_uint(y.z); b[4 * v + 3] = __float_as_uint(y.w);
+        }
+      } else {
+        // Straight from global memory; all loads first, then the TMEM stores.
+        const size_t roff = (static_cast<size_t>(c.bh) * p.N + (row_valid ? qrow : 0)) * D;
+        const uint4* gq = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(p.q) + roff);
+        const uint4* gdo = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(p.dout) + roff);
+#pragma unroll
+        for (int v = 0; v < kWords / 4; ++v) {
+          const uint4 x = row_valid ? gq[h * kWords / 4 + v] : make_uint4(0, 0, 0, 0);
+          const uint4 y = row_valid ? gdo[h * kWords / 4 + v] : make_uint4(0, 0, 0, 0);
+          a[4 * v] = x.x; a[4 * v + 1] = x.y; a[4 * v + 2] = x.z; a[4 * v + 3] = x.w;
+          b[4 * v] = y.x; b[4 * v + 1] = y.y; b[4 * v + 2] = y.z; b[4 * v + 3] = y.w;
+        }
       }
 #pragma unroll
       for (int w0 = 0; w0 < kWords; w0 += 16) {
@@ -729,6 +766,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(c.bar(B::dp_full), 1);
       mbar_init(c.bar(B::ds_full), 256);
       mbar_init(c.bar(B::all_done), 1);
+      mbar_init(c.bar(B::qdo_in), 1);
     }
     fence_barrier_init();
   }
@@ -762,7 +800,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (keys) {
     key_cta<D, BF16>(c, p, &tmap_q, &tmap_k, &tmap_v, &tmap_do, &tmap_dk, &tmap_dv, tile);
   } else {
-    query_cta<D, BF16>(c, p, &tmap_k, &tmap_v, &tmap_dq, tile);
+    query_cta<D, BF16>(c, p, &tmap_q, &tmap_k, &tmap_v, &tmap_do, &tmap_dq, tile);
   }
 
   tc_fence_before();
