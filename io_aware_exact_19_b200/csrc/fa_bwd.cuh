@@ -468,7 +468,7 @@ __device__ __forceinline__ void key_cta(const Ctx& c, const Params& p, const CUt
       store_rows_tma<BF16, D>(tl + 256 + h * D, h == 0 ? 1.0f : p.scale, have, stage, h == 0 ? tdv : tdk, 0,
                               j * kBlockN + wq * 32, c.bh, p.N);
     }
-    if (c.lane == 0) bulk_wait_group<0>();
+    if (c.lane == 0) bulk_wait_group_read<0>();  // shared memory read; the writes complete on their own
   }
 }
 
@@ -699,7 +699,7 @@ __device__ __forceinline__ void query_cta(const Ctx& c, const Params& p, const C
       store_rows_tma<BF16, D / 2>(tl + C::kColDQ + h * (D / 2), p.scale, have, stage, tdq, h * (D / 2),
                                   i * kBlockQ + wq * 32, c.bh, p.N);
     }
-    if (c.lane == 0) bulk_wait_group<0>();
+    if (c.lane == 0) bulk_wait_group_read<0>();  // shared memory read; the writes complete on their own
   }
 }
 

@@ -481,8 +481,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-    // The stores read shared memory asynchronously: let them finish before exit.
-    if (lane == 0) bulk_wait_group<0>();
+    // The stores read shared memory asynchronously: the CTA may exit once they have
+    // read it; their global writes complete by themselves before the grid does.
+    if (lane == 0) bulk_wait_group_read<0>();
   }
 
   tc_fence_before();
