@@ -19,7 +19,10 @@ Readings of points the pages leave open:
   * softmax gradient: dS = P∘(dP − rowsum(P∘dP)) with dP = dO·Vᵀ (textbook
     softmax Jacobian); the formula printed in [explainer] "梯度计算优化" is not
     dimensionally consistent and is not used.
-  * causal: top-left aligned, query i sees keys j ≤ i ([essay] 三.1), N_q = N_k.
+  * causal: query i sees keys j ≤ i ([essay] 三.1) when N_q = N_k. With
+    N_q ≠ N_k (pages silent) the mask is bottom-right aligned: query i sees keys
+    j ≤ i + (N_k − N_q), i.e. the queries are the last N_q positions of the key
+    sequence; with N_q = N_k it is the rule above.
   * block mask: one uint8 entry per 128×128 tile of S, shared by every batch
     and head, composed with the causal mask by AND ([card] Block-Sparse).
   * a row with no allowed key: O = 0, lse = −inf, zero gradient (pages silent).
@@ -39,13 +42,14 @@ TILE = 128  # one block-mask entry covers a TILE x TILE tile of S
 def allowed_mask(nq: int, nk: int, causal: bool = False, block_mask=None, tile: int = TILE) -> np.ndarray:
     """Boolean [nq, nk]: True where query i may attend to key j.
 
-    Causal ([essay] 三.1): P_ij = 0 for j > i. Block mask ([card] Block-Sparse):
-    entry (I, J) = 0 removes every pair (i, j) with i // tile == I and
-    j // tile == J. The two compose by AND.
+    Causal ([essay] 三.1): P_ij = 0 for j > i + (nk − nq) (bottom-right aligned;
+    j > i when nq = nk). Block mask ([card] Block-Sparse): entry (I, J) = 0
+    removes every pair (i, j) with i // tile == I and j // tile == J. The two
+    compose by AND.
     """
     a = np.ones((nq, nk), dtype=bool)
     if causal:
-        a &= np.arange(nk)[None, :] <= np.arange(nq)[:, None]
+        a &= np.arange(nk)[None, :] <= np.arange(nq)[:, None] + (nk - nq)
     if block_mask is not None:
         bm = np.asarray(block_mask).astype(bool)
         a &= bm[np.arange(nq)[:, None] // tile, np.arange(nk)[None, :] // tile]
@@ -113,7 +117,7 @@ def forward_rows(q, k, v, scale: float, rows, causal: bool = False, block_mask=N
     rows = np.asarray(rows)
     lead = q.shape[:-2]
     n = k.shape[-2]
-    allowed = _allowed_pairs(rows, np.arange(n), causal, block_mask, tile)
+    allowed = _allowed_pairs(rows, np.arange(n), causal, block_mask, tile, n - q.shape[-2])
     O = np.empty(lead + (rows.size, v.shape[-1]))
     lse = np.empty(lead + (rows.size,))
     for idx in np.ndindex(*lead):
@@ -168,7 +172,7 @@ def backward_rows(q, k, v, do, scale: float, rows, causal: bool = False, block_m
     """
     q, k, v, do = (np.asarray(t, dtype=np.float64) for t in (q, k, v, do))
     rows = np.asarray(rows)
-    allowed = _allowed_pairs(rows, np.arange(k.shape[0]), causal, block_mask, tile)
+    allowed = _allowed_pairs(rows, np.arange(k.shape[0]), causal, block_mask, tile, k.shape[0] - q.shape[0])
     S = scale * (q[rows] @ k.T)
     S = np.where(allowed, S, -np.inf)
     P, lse = _softmax_rows(S)
@@ -232,22 +236,27 @@ def online_forward(q, k, v, scale: float, bounds, causal: bool = False, block_ma
 
 # --------------------------------------------------------------------------- tile enumeration
 
-def causal_tile_set(n: int, br: int, bc: int):
+def causal_tile_set(n: int, br: int, bc: int, nk: int | None = None):
     """The valid-tile set of [essay] 三.1: {(i, j) | j·B_c ≤ i·B_r + B_r − 1}.
 
     i ranges over the ⌈n/B_r⌉ query tiles and j over the ⌈n/B_c⌉ key tiles.
-    Returned as a sorted list of (i, j) pairs.
+    With ``nk`` keys (N_q = n ≠ N_k) the diagonal is shifted by N_k − N_q and
+    the last row of tile i is the last real query row: j·B_c ≤
+    min(i·B_r + B_r − 1, n − 1) + N_k − N_q. Returned as a sorted list of (i, j) pairs.
     """
-    tr, tc = -(-n // br), -(-n // bc)
-    return [(i, j) for i in range(tr) for j in range(tc) if j * bc <= i * br + br - 1]
+    nk = n if nk is None else nk
+    tr, tc = -(-n // br), -(-nk // bc)
+    return [(i, j) for i in range(tr) for j in range(tc)
+            if j * bc <= min(i * br + br - 1, n - 1) + (nk - n)]
 
 
-def _visited(n, causal, block_mask, br, bc, mask_tile=TILE):
+def _visited(n, causal, block_mask, br, bc, mask_tile=TILE, nk=None):
     """Set of (i, j) tile pairs the method processes: the causal valid-tile set
     (or all pairs) intersected with the non-zero entries of the block mask.
     A query tile of B_r rows inside mask row I = i·B_r // mask_tile (B_r divides mask_tile)."""
-    tr, tc = -(-n // br), -(-n // bc)
-    pairs = set(causal_tile_set(n, br, bc)) if causal else {(i, j) for i in range(tr) for j in range(tc)}
+    nk = n if nk is None else nk
+    tr, tc = -(-n // br), -(-nk // bc)
+    pairs = set(causal_tile_set(n, br, bc, nk)) if causal else {(i, j) for i in range(tr) for j in range(tc)}
     if block_mask is not None:
         bm = np.asarray(block_mask)
         pairs = {(i, j) for (i, j) in pairs
@@ -255,18 +264,18 @@ def _visited(n, causal, block_mask, br, bc, mask_tile=TILE):
     return pairs
 
 
-def forward_tile_lists(n: int, causal: bool, block_mask=None, br: int = 128, bc: int = 128):
+def forward_tile_lists(n: int, causal: bool, block_mask=None, br: int = 128, bc: int = 128, nk: int | None = None):
     """For each query tile i, the sorted key tiles j it streams ([essay] 三.1; [card] Block-Sparse:
-    zero tiles skipped)."""
+    zero tiles skipped). ``n`` queries, ``nk`` keys (default ``n``)."""
     tr = -(-n // br)
-    pairs = _visited(n, causal, block_mask, br, bc)
+    pairs = _visited(n, causal, block_mask, br, bc, nk=nk)
     return [sorted(j for (ii, j) in pairs if ii == i) for i in range(tr)]
 
 
-def backward_tile_lists(n: int, causal: bool, block_mask=None, br: int = 128, bc: int = 128):
+def backward_tile_lists(n: int, causal: bool, block_mask=None, br: int = 128, bc: int = 128, nk: int | None = None):
     """For each key tile j, the sorted query tiles i that reach it (the transpose of the forward lists)."""
-    tc = -(-n // bc)
-    pairs = _visited(n, causal, block_mask, br, bc)
+    tc = -(-(n if nk is None else nk) // bc)
+    pairs = _visited(n, causal, block_mask, br, bc, nk=nk)
     return [sorted(i for (i, jj) in pairs if jj == j) for j in range(tc)]
 
 
@@ -305,10 +314,12 @@ def _head_sampled(q, k, v, do, scale, causal, block_mask, tile, rows_q, rows_k, 
     return out
 
 
-def _allowed_pairs(rows, cols, causal, block_mask, tile):
+def _allowed_pairs(rows, cols, causal, block_mask, tile, offset=0):
+    """allowed_mask restricted to query rows ``rows`` and key columns ``cols``;
+    ``offset`` = N_k − N_q (the causal diagonal's shift)."""
     a = np.ones((rows.size, cols.size), dtype=bool)
     if causal:
-        a &= cols[None, :] <= rows[:, None]
+        a &= cols[None, :] <= rows[:, None] + offset
     if block_mask is not None:
         bm = np.asarray(block_mask).astype(bool)
         a &= bm[rows[:, None] // tile, cols[None, :] // tile]
@@ -328,6 +339,8 @@ def sampled_forward_backward(q, k, v, do, scale: float, causal: bool, rows_q, ro
     Returns a dict of arrays with leading dims [..., len(rows)].
     """
     q, k, v, do = (np.asarray(t, dtype=np.float64) for t in (q, k, v, do))
+    if q.shape[-2] != k.shape[-2]:
+        raise ValueError("the long-sequence mode covers N_q = N_k only")
     rows_q, rows_k = np.asarray(rows_q), np.asarray(rows_k)
     lead = q.shape[:-2]
     heads = list(np.ndindex(*lead))

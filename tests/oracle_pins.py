@@ -226,13 +226,20 @@ def check_blocksparse_reductions(forward, backward):
 # ----------------------------------------------------------------------------- brute force
 
 def brute_forward(q, k, v, scale, causal):
-    """Loop-level reading of the definition, for tiny inputs."""
+    """Loop-level reading of the definition, for tiny inputs. With len(q) = n_q
+    queries and len(k) = n_k keys, the causal rule lets query i see key j when
+    j <= i + n_k - n_q (the queries are the last n_q positions); a query with no
+    key gets O = 0 and lse = -inf."""
     n, d = len(q), len(q[0])
+    nk = len(k)
     dv = len(v[0])
     O = [[0.0] * dv for _ in range(n)]
     lse = [0.0] * n
     for i in range(n):
-        keys = [j for j in range(len(k)) if (not causal or j <= i)]
+        keys = [j for j in range(nk) if (not causal or j <= i + nk - n)]
+        if not keys:
+            lse[i] = -math.inf
+            continue
         s = {j: scale * sum(q[i][t] * k[j][t] for t in range(d)) for j in keys}
         mx = max(s.values())
         e = {j: math.exp(s[j] - mx) for j in keys}
@@ -245,16 +252,44 @@ def brute_forward(q, k, v, scale, causal):
 
 def check_bruteforce(forward):
     r = _rng(11)
-    for n, d, causal in ((1, 1, False), (3, 2, False), (5, 3, True), (6, 4, False), (4, 4, True)):
-        q, k, v = (r.standard_normal((n, d)) for _ in range(3))
-        v2 = r.standard_normal((n, d + 1))
+    for n, nk, d, causal in ((1, 1, 1, False), (3, 3, 2, False), (5, 5, 3, True), (6, 6, 4, False), (4, 4, 4, True),
+                             (2, 5, 3, True), (5, 2, 3, True), (1, 6, 2, True), (3, 7, 2, False)):
+        q = r.standard_normal((n, d))
+        k = r.standard_normal((nk, d))
+        v2 = r.standard_normal((nk, d + 1))
         Ob, lseb = brute_forward(q.tolist(), k.tolist(), v2.tolist(), 0.9, causal)
         O, lse = forward(q, k, v2, 0.9, causal=causal)
-        _close(O, Ob, 1e-13, f"brute force O n={n} d={d}")
-        _close(lse, lseb, 1e-13, f"brute force lse n={n} d={d}")
+        _close(O, Ob, 1e-13, f"brute force O n={n} nk={nk} d={d}")
+        _close(lse, lseb, 1e-13, f"brute force lse n={n} nk={nk} d={d}")
+
+
+def check_causal_suffix_alignment(forward):
+    """N_q < N_k: causal attention of the queries against all keys equals the
+    last N_q rows of square causal attention over the key positions (queries
+    are the suffix of the sequence). N_q > N_k: the first N_q - N_k rows see no
+    key (O = 0, lse = -inf) and the rest equal square causal attention of the
+    last N_k queries."""
+    r = _rng(12)
+    for nq, nk in ((1, 5), (3, 7), (4, 4), (7, 3), (6, 1)):
+        d = 3
+        q = r.standard_normal((nq, d))
+        k = r.standard_normal((nk, d))
+        v = r.standard_normal((nk, d))
+        O, lse = forward(q, k, v, 0.7, causal=True)
+        if nq <= nk:
+            qfull = np.concatenate([r.standard_normal((nk - nq, d)), q])
+            Of, lsef = forward(qfull, k, v, 0.7, causal=True)
+            _close(O, Of[nk - nq:], 1e-13, f"suffix alignment O nq={nq} nk={nk}")
+            _close(lse, lsef[nk - nq:], 1e-13, f"suffix alignment lse nq={nq} nk={nk}")
+        else:
+            e = nq - nk
+            assert np.all(O[:e] == 0.0) and np.all(lse[:e] == -np.inf), f"rows without keys nq={nq} nk={nk}"
+            Of, lsef = forward(q[e:], k, v, 0.7, causal=True)
+            _close(O[e:], Of, 1e-13, f"short keys O nq={nq} nk={nk}")
+            _close(lse[e:], lsef, 1e-13, f"short keys lse nq={nq} nk={nk}")
 
 
 ALL_FORWARD_CHECKS = (
     check_rows_sum_to_one, check_equal_keys, check_single_key, check_causal_first_row,
-    check_constant_value_column, check_key_shift, check_bruteforce,
+    check_constant_value_column, check_key_shift, check_bruteforce, check_causal_suffix_alignment,
 )

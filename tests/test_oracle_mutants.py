@@ -28,6 +28,7 @@ MUTANTS = {
                               "a &= bm.T[np.arange(nq)[:, None] // tile, np.arange(nk)[None, :] // tile]"),
     "online rescale of l dropped": ("l = a_old * l + a_new * l_t", "l = l + a_new * l_t"),
     "online rescale of O dropped": ("O = a_old[:, None] * O + a_new[:, None] * O_t", "O = O + a_new[:, None] * O_t"),
+    "causal diagonal not shifted for N_q != N_k": ("<= np.arange(nq)[:, None] + (nk - nq)", "<= np.arange(nq)[:, None]"),
 }
 
 

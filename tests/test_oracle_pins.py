@@ -65,9 +65,10 @@ def test_sampled_mode_matches_full():
 
 # ------------------------------------------------------------------ tile enumeration
 
-def _tiles_with_allowed_pair(n, br, bc, causal, block_mask):
-    a = A.allowed_mask(n, n, causal, block_mask)
-    tr, tc = -(-n // br), -(-n // bc)
+def _tiles_with_allowed_pair(n, br, bc, causal, block_mask, nk=None):
+    nk = n if nk is None else nk
+    a = A.allowed_mask(n, nk, causal, block_mask)
+    tr, tc = -(-n // br), -(-nk // bc)
     return {(i, j) for i in range(tr) for j in range(tc)
             if a[i * br:(i + 1) * br, j * bc:(j + 1) * bc].any()}
 
@@ -76,6 +77,18 @@ def _tiles_with_allowed_pair(n, br, bc, causal, block_mask):
 @pytest.mark.parametrize("br,bc", [(128, 128), (64, 128)])
 def test_causal_tile_set_is_exactly_the_tiles_with_an_unmasked_entry(n, br, bc):
     assert set(A.causal_tile_set(n, br, bc)) == _tiles_with_allowed_pair(n, br, bc, True, None)
+
+
+@pytest.mark.parametrize("nq,nk", [(1, 1000), (128, 384), (384, 128), (300, 129), (129, 300), (1000, 777),
+                                   (640, 1), (5, 7)])
+def test_causal_tile_set_with_unequal_lengths(nq, nk):
+    # Bottom-right alignment: still exactly the tiles holding an allowed pair, and
+    # the transpose lists agree with the forward lists.
+    assert set(A.causal_tile_set(nq, 128, 128, nk)) == _tiles_with_allowed_pair(nq, 128, 128, True, None, nk)
+    fwd = A.forward_tile_lists(nq, True, nk=nk)
+    bwd = A.backward_tile_lists(nq, True, nk=nk)
+    assert {(i, j) for i, js in enumerate(fwd) for j in js} == {(i, j) for j, is_ in enumerate(bwd) for i in is_}
+    assert len(fwd) == -(-nq // 128) and len(bwd) == -(-nk // 128)
 
 
 @pytest.mark.parametrize("causal", [False, True])
