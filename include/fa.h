@@ -123,6 +123,31 @@ fa_status fa_blocksparse_bwd(fa_dtype dtype, const void* q, const void* k, const
                              const uint8_t* block_mask, cudaStream_t stream);
 
 /*
+ * Forward with Nq query rows and Nk key/value rows (a query block that is the
+ * last Nq positions of a longer key sequence, cross-attention, decoding). The
+ * pages treat the square case; this generalises the same computation:
+ * q, o [B,H,Nq,d]; k, v [B,H,Nk,d]; lse [B,H,Nq]. The causal mask is
+ * bottom-right aligned: query i attends to key j iff j <= i + Nk - Nq (for
+ * Nq = Nk the rule j <= i). A query row with no key gets O = 0, lse = -inf.
+ * block_mask may be NULL; otherwise it is a DEVICE uint8 [Nq/128][Nk/128] as
+ * in fa_blocksparse_fwd and needs Nq, Nk multiples of 128 (at most 2048 tiles
+ * each). With Nq = Nk this computes exactly what fa_fwd / fa_blocksparse_fwd do.
+ * Errors, ownership and stream semantics as fa_fwd.
+ */
+fa_status fa_fwd_qk(fa_dtype dtype, const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                    int Nq, int Nk, int d, float softmax_scale, int causal, const uint8_t* block_mask,
+                    cudaStream_t stream);
+
+/*
+ * Backward of fa_fwd_qk: dq [B,H,Nq,d]; dk, dv [B,H,Nk,d]; o, dout [B,H,Nq,d];
+ * workspace of at least fa_bwd_workspace_size(B, H, Nq, d) bytes (256-byte
+ * aligned). Rows without keys contribute nothing. Otherwise as fa_bwd.
+ */
+fa_status fa_bwd_qk(fa_dtype dtype, const void* q, const void* k, const void* v, const void* o, const float* lse,
+                    const void* dout, void* dq, void* dk, void* dv, void* workspace, int B, int H, int Nq, int Nk,
+                    int d, float softmax_scale, int causal, const uint8_t* block_mask, cudaStream_t stream);
+
+/*
  * Debug: the forward / backward with a record of the tiles each CTA loaded.
  * trace: DEVICE int32 buffer of fa_*_trace_size() entries; each record is a
  * count followed by entries (tile index) | (flags << 16).

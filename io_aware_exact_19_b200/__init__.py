@@ -6,9 +6,9 @@ memory and streams. There is no fallback: if ``libfa.so`` is missing or no CUDA
 device is present, the calls raise.
 
 Functions keep the C names: :func:`fa_fwd`, :func:`fa_bwd`,
-:func:`fa_blocksparse_fwd`, :func:`fa_blocksparse_bwd`,
-:func:`fa_bwd_workspace_size`, plus debug entry points for tile traces and the
-device status word.
+:func:`fa_blocksparse_fwd`, :func:`fa_blocksparse_bwd`, :func:`fa_fwd_qk`,
+:func:`fa_bwd_qk` (N_q query rows, N_k key rows), :func:`fa_bwd_workspace_size`,
+plus debug entry points for tile traces and the device status word.
 """
 from __future__ import annotations
 
@@ -25,7 +25,7 @@ EXPORTED = (
     "fa_status_string", "fa_fwd", "fa_bwd", "fa_blocksparse_fwd", "fa_blocksparse_bwd",
     "fa_bwd_workspace_size", "fa_fwd_trace_size", "fa_bwd_trace_size", "fa_bwd_row_tile",
     "fa_debug_fwd_trace", "fa_debug_bwd_trace", "fa_debug_bwd_phase", "fa_device_status",
-    "fa_debug_timeout_probe", "fa_bwd_noalloc",
+    "fa_debug_timeout_probe", "fa_bwd_noalloc", "fa_fwd_qk", "fa_bwd_qk",
 )
 
 
@@ -65,6 +65,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "fa_device_status": ([vp], i),
         "fa_debug_timeout_probe": ([i, vp], i),
         "fa_bwd_noalloc": (bwd_args[:10] + bwd_args[11:] + [vp], i),
+        # N_q, N_k in place of N
+        "fa_fwd_qk": (fwd_args[:8] + [i] + fwd_args[8:] + [vp, vp], i),
+        "fa_bwd_qk": (bwd_args[:13] + [i] + bwd_args[13:] + [vp, vp], i),
     }
     for name, (argtypes, restype) in sigs.items():
         fn = getattr(lib, name)
@@ -236,6 +239,33 @@ def fa_debug_timeout_probe(timeout_ms: int, stream=None) -> None:
 
 
 # ----------------------------------------------------------------------------- conveniences
+
+def fa_fwd_qk(q, k, v, o, lse, causal: bool = False, block_mask=None, scale: float | None = None,
+              stream=None) -> None:
+    """Forward with q, o [B, H, N_q, d] and k, v [B, H, N_k, d]; the causal mask is
+    bottom-right aligned (query i sees key j <= i + N_k - N_q)."""
+    B, H, Nq, d = _shape(q)
+    Nk = _shape(k)[2]
+    _check_tensors(q, k, v, o, lse, block_mask)
+    st = load_library().fa_fwd_qk(_dtype_code(q), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Nq, Nk, d,
+                                  _scale(scale, d), int(bool(causal)),
+                                  _ptr(block_mask) if block_mask is not None else None, _stream(stream))
+    _check(st, "fa_fwd_qk")
+
+
+def fa_bwd_qk(q, k, v, o, lse, dout, dq, dk, dv, workspace, causal: bool = False, block_mask=None,
+              scale: float | None = None, stream=None) -> None:
+    """Backward of :func:`fa_fwd_qk`; ``workspace`` holds at least
+    ``fa_bwd_workspace_size(B, H, N_q, d)`` bytes."""
+    B, H, Nq, d = _shape(q)
+    Nk = _shape(k)[2]
+    _check_tensors(q, k, v, o, lse, dout, dq, dk, dv, workspace, block_mask)
+    st = load_library().fa_bwd_qk(_dtype_code(q), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout),
+                                  _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace), B, H, Nq, Nk, d,
+                                  _scale(scale, d), int(bool(causal)),
+                                  _ptr(block_mask) if block_mask is not None else None, _stream(stream))
+    _check(st, "fa_bwd_qk")
+
 
 def attention_forward(q, k, v, causal: bool = False, block_mask=None, scale=None, stream=None):
     """Allocate O and lse with torch and run the forward; returns (o, lse)."""

@@ -57,6 +57,24 @@ fa_status check_common(fa_dtype dtype, int B, int H, int N, int d) {
   return FA_OK;
 }
 
+// The same limits for a problem with Nq query rows and Nk key rows (the
+// backward grid holds batch*heads*(Tq + Tk) CTAs).
+fa_status check_qk(fa_dtype dtype, int B, int H, int Nq, int Nk, int d) {
+  fa_status s = check_common(dtype, B, H, Nq, d);
+  if (s != FA_OK) return s;
+  s = check_common(dtype, B, H, Nk, d);
+  if (s != FA_OK) return s;
+  const long long bh = static_cast<long long>(B) * H;
+  const long long tiles = (static_cast<long long>(Nq) + 127) / 128 + (static_cast<long long>(Nk) + 127) / 128;
+  if (bh * tiles > 0x7FFFFFFFLL) return FA_ERR_UNSUPPORTED;
+  return FA_OK;
+}
+
+fa_status check_mask_qk(int Nq, int Nk) {
+  if (Nq % 128 != 0 || Nk % 128 != 0 || Nq / 128 > 2048 || Nk / 128 > 2048) return FA_ERR_UNSUPPORTED;
+  return FA_OK;
+}
+
 fa_status check_mask(int N, int d, const uint8_t* block_mask) {
   (void)d;
   if (block_mask == nullptr) return FA_ERR_INVALID_ARG;
@@ -66,8 +84,8 @@ fa_status check_mask(int N, int d, const uint8_t* block_mask) {
 
 fa_status fwd_impl(fa_dtype dtype, const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
                    int N, int d, float scale, int causal, const uint8_t* mask, int32_t* trace,
-                   cudaStream_t stream) {
-  fa_status s = check_common(dtype, B, H, N, d);
+                   cudaStream_t stream, int Nk = 0) {
+  fa_status s = Nk > 0 ? check_qk(dtype, B, H, N, Nk, d) : check_common(dtype, B, H, N, d);
   if (s != FA_OK) return s;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
     return FA_ERR_INVALID_ARG;
@@ -81,6 +99,7 @@ fa_status fwd_impl(fa_dtype dtype, const void* q, const void* k, const void* v, 
   a.B = B;
   a.H = H;
   a.N = N;
+  a.Nk = Nk;
   a.d = d;
   a.scale = scale;
   a.causal = causal ? 1 : 0;
@@ -94,8 +113,8 @@ fa_status fwd_impl(fa_dtype dtype, const void* q, const void* k, const void* v, 
 fa_status bwd_impl(fa_dtype dtype, const void* q, const void* k, const void* v, const void* o, const float* lse,
                    const void* dout, void* dq, void* dk, void* dv, void* workspace, int B, int H, int N, int d,
                    float scale, int causal, const uint8_t* mask, int32_t* trace, cudaStream_t stream,
-                   int phases = 7) {
-  fa_status s = check_common(dtype, B, H, N, d);
+                   int phases = 7, int Nk = 0) {
+  fa_status s = Nk > 0 ? check_qk(dtype, B, H, N, Nk, d) : check_common(dtype, B, H, N, d);
   if (s != FA_OK) return s;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) || !aligned16(dout) ||
       !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
@@ -116,6 +135,7 @@ fa_status bwd_impl(fa_dtype dtype, const void* q, const void* k, const void* v, 
   a.B = B;
   a.H = H;
   a.N = N;
+  a.Nk = Nk;
   a.d = d;
   a.scale = scale;
   a.causal = causal ? 1 : 0;
@@ -179,6 +199,29 @@ fa_status fa_blocksparse_bwd(fa_dtype dtype, const void* q, const void* k, const
   if (s != FA_OK) return s;
   return bwd_impl(dtype, q, k, v, o, lse, dout, dq, dk, dv, workspace, B, H, N, d, softmax_scale, causal,
                   block_mask, nullptr, stream);
+}
+
+fa_status fa_fwd_qk(fa_dtype dtype, const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                    int Nq, int Nk, int d, float softmax_scale, int causal, const uint8_t* block_mask,
+                    cudaStream_t stream) {
+  if (Nq < 1 || Nk < 1) return FA_ERR_INVALID_ARG;
+  if (block_mask != nullptr) {
+    fa_status s = check_mask_qk(Nq, Nk);
+    if (s != FA_OK) return s;
+  }
+  return fwd_impl(dtype, q, k, v, o, lse, B, H, Nq, d, softmax_scale, causal, block_mask, nullptr, stream, Nk);
+}
+
+fa_status fa_bwd_qk(fa_dtype dtype, const void* q, const void* k, const void* v, const void* o, const float* lse,
+                    const void* dout, void* dq, void* dk, void* dv, void* workspace, int B, int H, int Nq, int Nk,
+                    int d, float softmax_scale, int causal, const uint8_t* block_mask, cudaStream_t stream) {
+  if (Nq < 1 || Nk < 1) return FA_ERR_INVALID_ARG;
+  if (block_mask != nullptr) {
+    fa_status s = check_mask_qk(Nq, Nk);
+    if (s != FA_OK) return s;
+  }
+  return bwd_impl(dtype, q, k, v, o, lse, dout, dq, dk, dv, workspace, B, H, Nq, d, softmax_scale, causal,
+                  block_mask, nullptr, stream, 7, Nk);
 }
 
 size_t fa_fwd_trace_size(int B, int H, int N) {

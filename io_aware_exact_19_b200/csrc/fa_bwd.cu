@@ -42,15 +42,19 @@ int launch_bwd_t(const AttnArgs& a, cudaStream_t stream) {
   p.block_mask = a.block_mask;
   p.trace = a.trace;
   p.status = a.status;
+  const int Nk = a.Nk > 0 ? a.Nk : a.N;
   p.N = a.N;
+  p.Nk = Nk;
   p.Npad = (a.N + 127) / 128 * 128;
   p.BH = BH;
-  p.T = (a.N + 127) / 128;
+  p.Tq = (a.N + 127) / 128;
+  p.Tk = (Nk + 127) / 128;
   p.causal = a.causal;
   p.scale = a.scale;
-  // Heads per CTA-order group: their Q, dO, K, V (N*d*2 bytes each) fit ~48 MB of L2.
+  // Heads per CTA-order group: their Q, dO (N*d*2 bytes each) and K, V (Nk*d*2
+  // bytes each) fit ~48 MB of L2.
   {
-    const long long per_head = 8LL * a.N * D;
+    const long long per_head = 4LL * (a.N + Nk) * D;
     long long g = (48LL << 20) / (per_head > 0 ? per_head : 1);
     p.head_group = static_cast<int>(g < 1 ? 1 : (g > BH ? BH : g));
   }
@@ -74,17 +78,17 @@ int launch_bwd_t(const AttnArgs& a, cudaStream_t stream) {
     const bool dq64 = D / 2 >= 64;
     bool ok = host::make_map_3d(&tq, dt, 2, a.q, D, a.N, BH, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B) &&
               host::make_map_3d(&tdo, dt, 2, a.dout, D, a.N, BH, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B) &&
-              host::make_map_3d(&tk, dt, 2, a.k, D, a.N, BH, 64, bwd::kBlockN, CU_TENSOR_MAP_SWIZZLE_128B) &&
-              host::make_map_3d(&tv, dt, 2, a.v, D, a.N, BH, 64, bwd::kBlockN, CU_TENSOR_MAP_SWIZZLE_128B) &&
-              host::make_map_3d(&tdk, dt, 2, a.dk, D, a.N, BH, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B) &&
-              host::make_map_3d(&tdv, dt, 2, a.dv, D, a.N, BH, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B) &&
+              host::make_map_3d(&tk, dt, 2, a.k, D, Nk, BH, 64, bwd::kBlockN, CU_TENSOR_MAP_SWIZZLE_128B) &&
+              host::make_map_3d(&tv, dt, 2, a.v, D, Nk, BH, 64, bwd::kBlockN, CU_TENSOR_MAP_SWIZZLE_128B) &&
+              host::make_map_3d(&tdk, dt, 2, a.dk, D, Nk, BH, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B) &&
+              host::make_map_3d(&tdv, dt, 2, a.dv, D, Nk, BH, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B) &&
               host::make_map_3d(&tdq, dt, 2, a.dq, D, a.N, BH, dq64 ? 64 : 32, 32,
                                 dq64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE);
     if (!ok) return static_cast<int>(cudaErrorInvalidValue);
     auto kern = bwd::fa_bwd_main_kernel<D, BF16>;
     cudaError_t e = host::ensure_dynamic_smem(reinterpret_cast<const void*>(kern), C::kAlloc);
     if (e != cudaSuccess) return static_cast<int>(e);
-    dim3 grid(static_cast<unsigned>(BH) * 2u * static_cast<unsigned>(p.T));
+    dim3 grid(static_cast<unsigned>(BH) * static_cast<unsigned>(p.Tq + p.Tk));
     kern<<<grid, bwd::kThreads, C::kAlloc, stream>>>(tq, tk, tv, tdo, tdq, tdk, tdv, p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return static_cast<int>(e);

@@ -108,21 +108,36 @@ struct QueryBars {
 // are arithmetic; a block mask is read from global memory (a few cached bytes
 // per step): key-stationary CTAs scan mask column j, query-stationary CTAs scan
 // mask row i, both with the causal valid-tile rule applied by AND.
+// The causal valid-tile rule ("当算力不再是瓶颈" essay, section 三.1) with the
+// diagonal shifted by off = Nk - N (the N queries are the last N of Nk positions):
+// query tile x and key tile y share an allowed pair iff y*128 <= (x's last row,
+// at most N - 1) + off. `first`/`last` below solve it for x and for y.
 struct TileCursor {
-  const uint8_t* mask;
-  int kind;  // 0 key-stationary, 1 query-stationary
-  int tile, T, causal, pos;
-  __device__ __forceinline__ bool allowed(int x) const {
-    if (kind == 0) {
-      if (causal && x < tile) return false;
-      return mask[static_cast<size_t>(x) * T + tile] != 0;
-    }
-    if (causal && x > tile) return false;
-    return mask[static_cast<size_t>(tile) * T + x] != 0;
+  const uint8_t* mask;  // [Tq][Tk]
+  int kind;  // 0 key-stationary (walks query tiles), 1 query-stationary (walks key tiles)
+  int tile, Tq, Tk, N, off, causal, pos;
+  __device__ __forceinline__ bool causal_ok(int x) const {
+    if (!causal) return true;
+    const int qt = kind == 0 ? x : tile, kt = kind == 0 ? tile : x;
+    return kt * 128 <= min(qt * 128 + 127, N - 1) + off;
   }
+  __device__ __forceinline__ bool allowed(int x) const {
+    if (!causal_ok(x)) return false;
+    const size_t e = kind == 0 ? static_cast<size_t>(x) * Tk + tile : static_cast<size_t>(tile) * Tk + x;
+    return mask[e] != 0;
+  }
+  // Key-stationary: first query tile reaching this key tile (the last query tile
+  // always does: its last row N - 1 reaches key Nk - 1).
   __device__ __forceinline__ int first() const {
-    if (mask != nullptr) return 0;
-    return (kind == 0 && causal) ? tile : 0;
+    if (mask != nullptr || kind != 0 || !causal) return 0;
+    const int y = tile * 128 - off - 127;
+    return y <= 0 ? 0 : (y + 127) / 128;
+  }
+  // Query-stationary: one past the last key tile this query tile reaches.
+  __device__ __forceinline__ int end() const {
+    if (!causal) return Tk;
+    const int last_key = min(tile * 128 + 127, N - 1) + off;
+    return last_key < 0 ? 0 : min(Tk, last_key / 128 + 1);
   }
   // Next visited tile (call exactly `len` times).
   __device__ __forceinline__ int next() {
@@ -142,13 +157,15 @@ struct Params {
   void* dv;
   float* delta;  // [BH][Npad]
   float* lse2;   // [BH][Npad]
-  const uint8_t* block_mask;
+  const uint8_t* block_mask;  // [Tq][Tk] or null
   int32_t* trace;
   int* status;
-  int N;
-  int Npad;
+  int N;     // query rows
+  int Nk;    // key / value rows
+  int Npad;  // query rows rounded up to 128
   int BH;
-  int T;  // ceil(N / 128): key tiles, and query tiles
+  int Tq;    // ceil(N / 128) query tiles
+  int Tk;    // ceil(Nk / 128) key tiles
   int head_group;  // heads walked together (CTA order)
   int causal;
   float scale;
@@ -291,7 +308,7 @@ __device__ __forceinline__ void key_cta(const Ctx& c, const Params& p, const CUt
     if (c.warp == 0 && c.lane == 0) {
       // ---------------------------------------------------------- producer
       TileCursor cur = c.cursor;
-      int32_t* tr = p.trace ? p.trace + (static_cast<size_t>(c.bh) * p.T + j) * (p.T + 1) : nullptr;
+      int32_t* tr = p.trace ? p.trace + (static_cast<size_t>(c.bh) * p.Tk + j) * (p.Tq + 1) : nullptr;
       if (tr) tr[0] = len;
       if (len > 0) {
         mbar_arrive_expect_tx(c.bar(B::kv_full), 2 * C::kTile);
@@ -393,7 +410,7 @@ __device__ __forceinline__ void key_cta(const Ctx& c, const Params& p, const CUt
     const int wq = c.warp % 4;
     const int r = wq * 32 + c.lane;
     const int key = j * kBlockN + r;
-    const bool key_valid = key < p.N;
+    const bool key_valid = key < p.Nk;
     const uint32_t tl = c.tmem + (static_cast<uint32_t>(wq * 32) << 16);
     const float sl2 = p.scale_log2;
     const int qo = 64 * h;
@@ -410,12 +427,13 @@ __device__ __forceinline__ void key_cta(const Ctx& c, const Params& p, const CUt
       tc_fence_before();
       mbar_arrive(c.bar(B::s_free));
       if (!(ok = mbar_wait_warp(c.bar(B::qdo_full + s), (n / S) & 1, c.wait))) break;  // lse2, D of tile i
-      // Columns x < lim are masked (causal: key > query; or the key row lies past N).
+      // Columns x < lim are masked (causal: key > query + Nk - N; or the key row
+      // lies past Nk).
       int lim = 0;
       if (!key_valid) {
         lim = 64;
-      } else if (p.causal && j * kBlockN + kBlockN - 1 > i * kBR) {
-        lim = min(64, max(0, key - (i * kBR + qo)));
+      } else if (p.causal) {
+        lim = min(64, max(0, key - (p.Nk - p.N) - (i * kBR + qo)));
       }
       const uint32_t aL = smem_u32(sL + s * kBR + qo);
       float pv[64];
@@ -466,7 +484,7 @@ __device__ __forceinline__ void key_cta(const Ctx& c, const Params& p, const CUt
     if (ok) {
       const uint32_t stage = smem_u32(sQ) + static_cast<uint32_t>(c.warp - 4) * (32 * D * 2);
       store_rows_tma<BF16, D>(tl + 256 + h * D, h == 0 ? 1.0f : p.scale, have, stage, h == 0 ? tdv : tdk, 0,
-                              j * kBlockN + wq * 32, c.bh, p.N);
+                              j * kBlockN + wq * 32, c.bh, p.Nk);
     }
     if (c.lane == 0) bulk_wait_group_read<0>();  // shared memory read; the writes complete on their own
   }
@@ -495,8 +513,8 @@ __device__ __forceinline__ void query_cta(const Ctx& c, const Params& p, const C
     if (c.warp == 0 && c.lane == 0) {
       // ---------------------------------------------------------- producer
       TileCursor cur = c.cursor;
-      int32_t* tr = p.trace ? p.trace + static_cast<size_t>(p.BH) * p.T * (p.T + 1) +
-                                  (static_cast<size_t>(c.bh) * p.T + i) * (p.T + 1)
+      int32_t* tr = p.trace ? p.trace + static_cast<size_t>(p.BH) * p.Tk * (p.Tq + 1) +
+                                  (static_cast<size_t>(c.bh) * p.Tq + i) * (p.Tk + 1)
                             : nullptr;
       if (tr) tr[0] = len;
       if constexpr (kStageQdo) {
@@ -659,8 +677,8 @@ __device__ __forceinline__ void query_cta(const Ctx& c, const Params& p, const C
       mbar_arrive(c.bar(B::s_free));
       // Mask columns x > lim: causal (key > query) and keys past N.
       int lim = 63;
-      if (p.causal && jt * kBlockN + 64 * h + 63 > qrow) lim = qrow - jt * kBlockN - 64 * h;
-      const int kv_left = p.N - jt * kBlockN - 64 * h - 1;
+      if (p.causal) lim = min(lim, qrow + (p.Nk - p.N) - jt * kBlockN - 64 * h);
+      const int kv_left = p.Nk - jt * kBlockN - 64 * h - 1;
       if (kv_left < lim) lim = kv_left;
       float pv[64];
 #pragma unroll
@@ -727,14 +745,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   c.warp = threadIdx.x / 32;
   c.lane = threadIdx.x % 32;
   int rank = 0;
-  grouped_order(static_cast<int>(blockIdx.x), p.BH, 2 * p.T, p.head_group, c.bh, rank);
-  const bool keys = (rank & 1) == 0;
-  const int tile = keys ? (rank >> 1) : p.T - 1 - (rank >> 1);
+  grouped_order(static_cast<int>(blockIdx.x), p.BH, p.Tk + p.Tq, p.head_group, c.bh, rank);
+  // Ranks alternate key / query CTAs while both kinds remain, then the rest of
+  // the longer kind; small key tiles and large query tiles (the heaviest under a
+  // causal mask) come first.
+  const int both = 2 * min(p.Tk, p.Tq);
+  const bool keys = rank < both ? (rank & 1) == 0 : p.Tk > p.Tq;
+  const int t = rank < both ? (rank >> 1) : (both >> 1) + (rank - both);
+  const int tile = keys ? t : p.Tq - 1 - t;
 
   c.cursor.mask = p.block_mask;
   c.cursor.kind = keys ? 0 : 1;
   c.cursor.tile = tile;
-  c.cursor.T = p.T;
+  c.cursor.Tq = p.Tq;
+  c.cursor.Tk = p.Tk;
+  c.cursor.N = p.N;
+  c.cursor.off = p.Nk - p.N;
   c.cursor.causal = p.causal;
   c.cursor.pos = c.cursor.first();
 
@@ -777,16 +803,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (c.warp == 2) {
     // Number of tiles this CTA visits.
     int count = 0;
+    const int range = keys ? p.Tq : p.Tk;  // candidate tiles of the other kind
     if (p.block_mask != nullptr) {
-      for (int base = 0; base < p.T; base += 32) {
+      for (int base = 0; base < range; base += 32) {
         const int x = base + c.lane;
-        const bool use = x < p.T && c.cursor.allowed(x);
+        const bool use = x < range && c.cursor.allowed(x);
         count += __popc(__ballot_sync(0xffffffffu, use));
       }
     } else if (keys) {
-      count = p.T - c.cursor.first();
+      count = p.Tq - c.cursor.first();
     } else {
-      count = p.causal ? tile + 1 : p.T;
+      count = c.cursor.end();
     }
     if (c.lane == 0) *tile_count = count;
   }

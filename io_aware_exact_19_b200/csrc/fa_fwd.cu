@@ -12,11 +12,12 @@ int launch_fwd_t(const AttnArgs& a, cudaStream_t stream) {
   using L = fwd::Smem<D>;
   const int BH = a.B * a.H;
   const CUtensorMapDataType dt = BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  const int Nk = a.Nk > 0 ? a.Nk : a.N;
   CUtensorMap tq, tk, tv, to;
   // O is written by 64-column x 32-row boxes, one per warp and 64 columns.
   bool ok = host::make_map_3d(&tq, dt, 2, a.q, D, a.N, BH, 64, fwd::kBlockM, CU_TENSOR_MAP_SWIZZLE_128B) &&
-            host::make_map_3d(&tk, dt, 2, a.k, D, a.N, BH, 64, fwd::kBlockN, CU_TENSOR_MAP_SWIZZLE_128B) &&
-            host::make_map_3d(&tv, dt, 2, a.v, D, a.N, BH, 64, fwd::kBlockN, CU_TENSOR_MAP_SWIZZLE_128B) &&
+            host::make_map_3d(&tk, dt, 2, a.k, D, Nk, BH, 64, fwd::kBlockN, CU_TENSOR_MAP_SWIZZLE_128B) &&
+            host::make_map_3d(&tv, dt, 2, a.v, D, Nk, BH, 64, fwd::kBlockN, CU_TENSOR_MAP_SWIZZLE_128B) &&
             host::make_map_3d(&to, dt, 2, a.o, D, a.N, BH, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B);
   if (!ok) return static_cast<int>(cudaErrorInvalidValue);
   fwd::Params p;
@@ -26,14 +27,15 @@ int launch_fwd_t(const AttnArgs& a, cudaStream_t stream) {
   p.trace = a.trace;
   p.status = a.status;
   p.N = a.N;
+  p.Nk = Nk;
   p.BH = BH;
   const int Tq = (a.N + fwd::kBlockM - 1) / fwd::kBlockM;
   p.n_pairs = (Tq + 1) / 2;
-  p.Tc = (a.N + fwd::kBlockN - 1) / fwd::kBlockN;
+  p.Tc = (Nk + fwd::kBlockN - 1) / fwd::kBlockN;
   p.causal = a.causal;
   // Heads per CTA-order group: their K and V (2*N*d*2 bytes each) fit ~48 MB of L2.
   {
-    const long long per_head = 4LL * a.N * D;
+    const long long per_head = 4LL * Nk * D;
     long long g = (48LL << 20) / (per_head > 0 ? per_head : 1);
     p.head_group = static_cast<int>(g < 1 ? 1 : (g > BH ? BH : g));
   }

@@ -50,13 +50,14 @@ static_assert(128 * kRegsLow + 256 * kRegsHigh <= kThreads * kRegsLaunch, "regis
 struct Params {
   void* o;
   float* lse;
-  const uint8_t* block_mask;  // null unless block-sparse
+  const uint8_t* block_mask;  // null unless block-sparse: [ceil(N/128)][Tc]
   int32_t* trace;             // null unless tracing
   int* status;
-  int N;
+  int N;        // query rows
+  int Nk;       // key / value rows
   int BH;
   int n_pairs;  // ceil(T_q / 2)
-  int Tc;       // ceil(N / 128)
+  int Tc;       // ceil(Nk / 128)
   int head_group;  // heads walked together (CTA order)
   int causal;
   float scale_log2;  // softmax scale * log2(e)
@@ -81,22 +82,26 @@ struct Smem {
 // tile j(n) with flags f(n) (bit q set: query tile 2p+q uses it).
 struct TileList {
   int len;
-  int mode;  // 0 dense, 1 causal, 2 list in shared memory
-  int q0;    // first query tile index (2p)
-  int q1_active;
+  int mode;        // 0 dense, 1 causal, 2 list in shared memory
+  int lim0, lim1;  // last key tile query tile 0 / 1 uses (-1: none, e.g. no tile 1)
   const uint32_t* list;
 
   __device__ __forceinline__ uint32_t entry(int n) const {
     if (mode == 2) return list[n];
-    uint32_t f;
-    if (mode == 0) {
-      f = 1u | (q1_active ? 2u : 0u);
-    } else {
-      f = (n <= q0 ? 1u : 0u) | ((q1_active && n <= q0 + 1) ? 2u : 0u);
-    }
+    const uint32_t f = (n <= lim0 ? 1u : 0u) | (n <= lim1 ? 2u : 0u);
     return static_cast<uint32_t>(n) | (f << 16);
   }
 };
+
+// Causal valid-tile rule ("当算力不再是瓶颈" essay, section 三.1, with the diagonal
+// shifted by Nk - N when the N queries are the last N of Nk positions): query
+// tile qt reaches key tile j iff j*128 <= (its last row, at most N - 1) + Nk - N.
+// Returns the last such j, or -1 if the tile reaches no key.
+__device__ __forceinline__ int causal_last_key_tile(int qt, int N, int Nk) {
+  const int last_row = min(qt * kBlockM + kBlockM - 1, N - 1);
+  const int last_key = last_row + (Nk - N);
+  return last_key < 0 ? -1 : last_key / kBlockN;
+}
 
 template <int D, bool BF16>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -154,10 +159,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
   }
+  // Causal reach of the two query tiles (every key tile when not causal). Each
+  // role derives it where it needs it, so it is not live across the register split.
+  auto reach = [&](int qi) {
+    if (qi == 1 && !q1_active) return -1;
+    return p.causal ? causal_last_key_tile(q0 + qi, p.N, p.Nk) : p.Tc - 1;
+  };
   if (warp == 2) {
+    const int lim0 = reach(0), lim1 = reach(1);
     if (p.block_mask != nullptr) {
       // Union of the non-zero key tiles of mask rows q0 and q0+1, in order, with
-      // the causal valid-tile rule (j <= q for 128x128 tiles) applied by AND.
+      // the causal valid-tile rule applied by AND.
       const uint8_t* row0 = p.block_mask + static_cast<size_t>(q0) * p.Tc;
       const uint8_t* row1 = row0 + p.Tc;
       int count = 0;
@@ -165,8 +177,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int j = base + lane;
         uint32_t f = 0;
         if (j < p.Tc) {
-          if (row0[j] && (!p.causal || j <= q0)) f |= 1u;
-          if (q1_active && row1[j] && (!p.causal || j <= q0 + 1)) f |= 2u;
+          if (row0[j] && j <= lim0) f |= 1u;
+          if (q1_active && row1[j] && j <= lim1) f |= 2u;
         }
         const uint32_t ballot = __ballot_sync(0xffffffffu, f != 0);
         if (f != 0) {
@@ -185,20 +197,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
   WaitCtx ctx{abort_flag, p.status};
 
-  TileList tl;
-  tl.q0 = q0;
-  tl.q1_active = q1_active;
-  tl.list = list;
-  if (p.block_mask != nullptr) {
-    tl.mode = 2;
-    tl.len = *list_len;
-  } else if (p.causal) {
-    tl.mode = 1;
-    tl.len = min(p.Tc, q1_active ? q0 + 2 : q0 + 1);
-  } else {
-    tl.mode = 0;
-    tl.len = p.Tc;
-  }
+  auto make_tiles = [&]() {
+    TileList tl;
+    tl.lim0 = reach(0);
+    tl.lim1 = reach(1);
+    tl.list = list;
+    if (p.block_mask != nullptr) {
+      tl.mode = 2;
+      tl.len = *list_len;
+    } else if (p.causal) {
+      tl.mode = 1;
+      tl.len = min(p.Tc, max(tl.lim0, tl.lim1) + 1);
+    } else {
+      tl.mode = 0;
+      tl.len = p.Tc;
+    }
+    return tl;
+  };
 
   uint8_t* sQ = smem + L::kQOff;
   uint8_t* sK = smem + L::kKOff;
@@ -212,6 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // sees the budget of every code path.
   if (warp < 4) {
    reg_dealloc<kRegsLow>();
+   const TileList tl = make_tiles();
    if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0 && tl.len > 0) {
@@ -321,6 +337,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   } else {
     reg_alloc<kRegsHigh>();
+    const TileList tl = make_tiles();
     // ------------------------------------------------------------ softmax
     const int q = (warp - 4) / 4;  // query tile within the pair
     const int wq = warp % 4;       // TMEM lane quarter
@@ -353,10 +370,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld_wait();
         float* s = reinterpret_cast<float*>(sr);
 
-        // Element mask: causal diagonal tile (key > row) and keys past N.
+        // Element mask: causal (key > row + Nk - N) and keys past Nk.
         int limit = kBlockN - 1;
-        if (p.causal && j == qt) limit = row_local;
-        const int kv_left = p.N - j * kBlockN - 1;
+        if (p.causal) limit = min(limit, row + (p.Nk - p.N) - j * kBlockN);
+        const int kv_left = p.Nk - j * kBlockN - 1;
         if (kv_left < limit) limit = kv_left;
         if (limit < kBlockN - 1) {
 #pragma unroll

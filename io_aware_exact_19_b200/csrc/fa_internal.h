@@ -19,7 +19,8 @@ struct AttnArgs {
   void* dk;
   void* dv;
   void* workspace;
-  int B, H, N, d;
+  int B, H, N, d;  // N: query rows
+  int Nk = 0;      // key / value rows (0: equal to N)
   float scale;
   int causal;
   const uint8_t* block_mask;

@@ -74,6 +74,16 @@ def test_host_argument_errors_return_before_launch(lib):
     assert lib.fa_bwd(1, p, p, p, p, p, p, p, p, p, _fake(4096 + 16), 1, 1, 128, 64, 0.1, 0, None) \
         == fa.FA_ERR_INVALID_ARG
     assert lib.fa_debug_timeout_probe(0, None) == fa.FA_ERR_INVALID_ARG
+    # N_q != N_k entry points: sizes, head dimension, block-mask shape rules
+    assert lib.fa_fwd_qk(1, p, p, p, p, p, 1, 1, 0, 128, 64, 0.1, 1, None, None) == fa.FA_ERR_INVALID_ARG
+    assert lib.fa_fwd_qk(1, p, p, p, p, p, 1, 1, 128, 0, 64, 0.1, 1, None, None) == fa.FA_ERR_INVALID_ARG
+    assert lib.fa_fwd_qk(1, p, p, p, p, p, 1, 1, 128, 256, 96, 0.1, 1, None, None) == fa.FA_ERR_UNSUPPORTED
+    assert lib.fa_fwd_qk(1, p, p, p, p, p, 1, 1, 128, 200, 64, 0.1, 0, p, None) == fa.FA_ERR_UNSUPPORTED
+    assert lib.fa_fwd_qk(1, None, p, p, p, p, 1, 1, 128, 256, 64, 0.1, 0, None, None) == fa.FA_ERR_INVALID_ARG
+    assert lib.fa_bwd_qk(1, p, p, p, p, p, p, p, p, p, _fake(4096 + 16), 1, 1, 128, 256, 64, 0.1, 0, None, None) \
+        == fa.FA_ERR_INVALID_ARG
+    assert lib.fa_bwd_qk(1, p, p, p, p, p, p, p, p, p, p, 1, 1, 256, 100, 64, 0.1, 1, p, None) \
+        == fa.FA_ERR_UNSUPPORTED
 
 
 def test_trace_sizes(lib):
