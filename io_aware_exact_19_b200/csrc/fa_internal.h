@@ -26,7 +26,7 @@ struct AttnArgs {
   const uint8_t* block_mask;
   int32_t* trace;
   int* status;
-  int phases = 7;  // backward launches to run: bit 0 prep, bit 1 main, bit 2 finish
+  int phases = 7;  // backward launches to run: bit 0 prep, bit 1 main
 };
 
 // Return 0 on success, a cudaError_t value otherwise.
@@ -35,7 +35,6 @@ int launch_bwd(const AttnArgs& a, cudaStream_t stream);
 
 // Workspace layout of the backward, in bytes from the workspace base.
 struct BwdWorkspace {
-  size_t dq_acc;    // fp32 [BH][N][d]
   size_t delta;     // fp32 [BH][Npad]  D = rowsum(dO o O)
   size_t lse2;      // fp32 [BH][Npad]  lse * log2(e), +inf on padding rows
   size_t total;
