@@ -29,6 +29,8 @@ from .attention import (  # noqa: F401
     backward,
     backward_rows,
     online_forward,
+    merge_partials,
+    split_kv_forward,
     causal_tile_set,
     forward_tile_lists,
     backward_tile_lists,

@@ -234,6 +234,55 @@ def online_forward(q, k, v, scale: float, bounds, causal: bool = False, block_ma
     return O, lse
 
 
+# --------------------------------------------------------------------------- split-KV merge
+
+def merge_partials(Os, lses):
+    """Merge partial results of disjoint key splits of the same query rows.
+
+    Each split s contributes O_s (its softmax-weighted average of its values) and
+    lse_s (the log of its exp-sum). The whole is
+        lse = log Σ_s exp(lse_s),   O = Σ_s exp(lse_s − lse)·O_s,
+    the online-softmax update of [interview] 三.2 applied to whole splits at once.
+    A split with no allowed key has lse_s = −inf and weight 0; a row whose splits
+    all have none gets O = 0, lse = −inf.
+    """
+    lses = np.stack([np.asarray(x, dtype=np.float64) for x in lses])   # [S, ..., N]
+    Os = np.stack([np.asarray(x, dtype=np.float64) for x in Os])       # [S, ..., N, dv]
+    m = lses.max(axis=0)
+    m_safe = np.where(np.isfinite(m), m, 0.0)
+    w = np.exp(lses - m_safe)                                          # exp(−inf) = 0
+    z = w.sum(axis=0)
+    lse = np.full(z.shape, -np.inf)
+    pos = z > 0
+    lse[pos] = m_safe[pos] + np.log(z[pos])
+    O = np.divide((w[..., None] * Os).sum(axis=0), z[..., None],
+                  out=np.zeros(Os.shape[1:]), where=pos[..., None])
+    return O, lse
+
+
+def split_kv_forward(q, k, v, scale: float, bounds, causal: bool = False, block_mask=None,
+                     tile: int = TILE):
+    """Forward for one head (q [N_q, d], k, v [N_k, d]) with the keys cut into
+    consecutive splits at ``bounds`` (0 = b_0 < … < b_S = N_k): each split is
+    computed on its own by the definition restricted to its keys, then the
+    partials are merged (:func:`merge_partials`) — the split-KV form used for
+    decoding, where one query row meets a long key sequence. Masks are those of
+    :func:`allowed_mask` on the whole problem. Returns (O, lse, Os, lses).
+    """
+    q, k, v = (np.asarray(t, dtype=np.float64) for t in (q, k, v))
+    allowed = allowed_mask(q.shape[0], k.shape[0], causal, block_mask, tile)
+    Os, lses = [], []
+    bounds = list(bounds)
+    for lo, hi in zip(bounds[:-1], bounds[1:]):
+        S = scale * (q @ k[lo:hi].T)
+        S = np.where(allowed[:, lo:hi], S, -np.inf)
+        P, lse_s = _softmax_rows(S)
+        Os.append(P @ v[lo:hi])
+        lses.append(lse_s)
+    O, lse = merge_partials(Os, lses)
+    return O, lse, Os, lses
+
+
 # --------------------------------------------------------------------------- tile enumeration
 
 def causal_tile_set(n: int, br: int, bc: int, nk: int | None = None):

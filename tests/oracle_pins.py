@@ -289,6 +289,40 @@ def check_causal_suffix_alignment(forward):
             _close(lse[e:], lsef, 1e-13, f"short keys lse nq={nq} nk={nk}")
 
 
+def check_split_kv_merge(forward, split_kv_forward, merge_partials):
+    """Split-KV: merging per-split partials equals the one-pass forward for any
+    split (sizes down to one key), with causal and block masks and N_q != N_k; a
+    split without allowed keys carries lse = -inf and changes nothing."""
+    r = _rng(13)
+    for nq, nk, causal, mask in ((1, 9, False, None), (1, 9, True, None), (4, 11, True, None),
+                                 (7, 5, True, None), (6, 8, False, np.array([[1, 0], [1, 1]], np.uint8))):
+        d = 3
+        q = r.standard_normal((nq, d))
+        k = r.standard_normal((nk, d))
+        v = r.standard_normal((nk, d + 1))
+        O, lse = forward(q, k, v, 0.8, causal=causal, block_mask=mask, tile=4)
+        cuts = sorted(set(r.choice(np.arange(1, nk), size=min(3, nk - 1), replace=False).tolist())) if nk > 1 else []
+        for bounds in ([0, nk], [0] + cuts + [nk], list(range(nk + 1))):
+            Om, lsem, Os, lses = split_kv_forward(q, k, v, 0.8, bounds, causal=causal, block_mask=mask, tile=4)
+            _close(Om, O, 1e-13, f"split-KV O nq={nq} nk={nk} bounds={bounds}")
+            _close(lsem, lse, 1e-13, f"split-KV lse nq={nq} nk={nk} bounds={bounds}")
+    # An empty split (every key masked for every row) has lse = -inf and no effect;
+    # the merge is associative.
+    q = r.standard_normal((3, 2))
+    k = r.standard_normal((6, 2))
+    v = r.standard_normal((6, 2))
+    mask = np.array([[1, 0, 1], [1, 0, 1]], np.uint8)  # key block 1 (keys 2, 3) removed for all rows
+    O, lse, Os, lses = split_kv_forward(q, k, v, 1.1, [0, 2, 4, 6], block_mask=mask, tile=2)
+    assert np.all(lses[1] == -np.inf) and np.all(Os[1] == 0.0), "empty split"
+    _merge = merge_partials
+    O2, lse2 = _merge([Os[0], Os[2]], [lses[0], lses[2]])
+    _close(O2, O, 1e-15, "empty split dropped")
+    Oa, lsea = _merge([Os[0], Os[1]], [lses[0], lses[1]])
+    O3, lse3 = _merge([Oa, Os[2]], [lsea, lses[2]])
+    _close(O3, O, 1e-14, "merge associativity O")
+    _close(lse3, lse, 1e-14, "merge associativity lse")
+
+
 ALL_FORWARD_CHECKS = (
     check_rows_sum_to_one, check_equal_keys, check_single_key, check_causal_first_row,
     check_constant_value_column, check_key_shift, check_bruteforce, check_causal_suffix_alignment,

@@ -29,6 +29,8 @@ MUTANTS = {
     "online rescale of l dropped": ("l = a_old * l + a_new * l_t", "l = l + a_new * l_t"),
     "online rescale of O dropped": ("O = a_old[:, None] * O + a_new[:, None] * O_t", "O = O + a_new[:, None] * O_t"),
     "causal diagonal not shifted for N_q != N_k": ("<= np.arange(nq)[:, None] + (nk - nq)", "<= np.arange(nq)[:, None]"),
+    "split-KV merge without the lse weights": ("w = np.exp(lses - m_safe)", "w = np.ones_like(lses)"),
+    "split-KV merged lse without the max": ("lse[pos] = m_safe[pos] + np.log(z[pos])", "lse[pos] = np.log(z[pos])"),
 }
 
 
@@ -51,6 +53,7 @@ def _run_all(mod):
         lambda: pins.check_finite_differences(mod.forward, mod.backward),
         lambda: pins.check_gradient_identities(mod.forward, mod.backward),
         lambda: pins.check_blocksparse_reductions(mod.forward, mod.backward),
+        lambda: pins.check_split_kv_merge(mod.forward, mod.split_kv_forward, mod.merge_partials),
     ] + [lambda c=c: c(mod.forward) for c in pins.ALL_FORWARD_CHECKS]
     for c in checks:
         try:

@@ -28,6 +28,10 @@ def test_gradient_identities():
     pins.check_gradient_identities(oracle.forward, oracle.backward)
 
 
+def test_split_kv_merge():
+    pins.check_split_kv_merge(oracle.forward, oracle.split_kv_forward, oracle.merge_partials)
+
+
 def test_blocksparse_reductions():
     pins.check_blocksparse_reductions(oracle.forward, oracle.backward)
 
