@@ -327,3 +327,45 @@ ALL_FORWARD_CHECKS = (
     check_rows_sum_to_one, check_equal_keys, check_single_key, check_causal_first_row,
     check_constant_value_column, check_key_shift, check_bruteforce, check_causal_suffix_alignment,
 )
+
+
+def check_rows_unequal_lengths(forward, forward_rows, backward_rows):
+    """The row-restricted routines with N_q != N_k (bottom-right causal diagonal):
+    forward_rows equals the rows of the whole forward (itself pinned by brute force
+    and suffix alignment), and backward_rows' gradients of
+    L = sum over the chosen rows of <dO_i, O_i> match central finite differences
+    of that loss computed through the forward."""
+    r = _rng(14)
+    mask = np.array([[1, 0, 1], [0, 1, 1]], dtype=np.uint8)
+    for nq, nk, causal, bm in ((3, 9, True, None), (9, 4, True, None), (5, 7, False, None), (7, 12, True, mask),
+                               (8, 5, False, mask[:, :2])):
+        d = 3
+        q = r.standard_normal((nq, d))
+        k = r.standard_normal((nk, d))
+        v = r.standard_normal((nk, d))
+        do = r.standard_normal((nq, d))
+        rows = np.array(sorted(set([0, nq // 2, nq - 1])))
+        O, lse = forward(q, k, v, 0.6, causal=causal, block_mask=bm, tile=4)
+        Or, lser = forward_rows(q, k, v, 0.6, rows, causal=causal, block_mask=bm, tile=4)
+        _close(Or, O[rows], 1e-13, f"forward_rows O nq={nq} nk={nk} causal={causal}")
+        _close(lser, lse[rows], 1e-13, f"forward_rows lse nq={nq} nk={nk} causal={causal}")
+        o2, l2, dq_r, dk, dv = backward_rows(q, k, v, do, 0.6, rows, causal=causal, block_mask=bm, tile=4)
+        _close(o2, O[rows], 1e-13, f"backward_rows O nq={nq} nk={nk}")
+        _close(l2, lse[rows], 1e-13, f"backward_rows lse nq={nq} nk={nk}")
+        dq = np.zeros_like(q)
+        dq[rows] = dq_r
+
+        def L(q_, k_, v_):
+            Ox, _ = forward(q_, k_, v_, 0.6, causal=causal, block_mask=bm, tile=4)
+            return float(np.sum(do[rows] * Ox[rows]))
+
+        h = 1e-5
+        for which, grad in (("q", dq), ("k", dk), ("v", dv)):
+            base = {"q": q, "k": k, "v": v}
+            R = r.standard_normal(base[which].shape)
+            plus = {n: a + h * R if n == which else a for n, a in base.items()}
+            minus = {n: a - h * R if n == which else a for n, a in base.items()}
+            fd = (L(plus["q"], plus["k"], plus["v"]) - L(minus["q"], minus["k"], minus["v"])) / (2 * h)
+            an = float(np.sum(grad * R))
+            assert abs(fd - an) <= 1e-7 * max(1.0, abs(an)), \
+                f"backward_rows finite differences d{which} nq={nq} nk={nk} causal={causal}: {fd} vs {an}"

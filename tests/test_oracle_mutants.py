@@ -31,6 +31,8 @@ MUTANTS = {
     "causal diagonal not shifted for N_q != N_k": ("<= np.arange(nq)[:, None] + (nk - nq)", "<= np.arange(nq)[:, None]"),
     "split-KV merge without the lse weights": ("w = np.exp(lses - m_safe)", "w = np.ones_like(lses)"),
     "split-KV merged lse without the max": ("lse[pos] = m_safe[pos] + np.log(z[pos])", "lse[pos] = np.log(z[pos])"),
+    "row routines' causal diagonal not shifted for N_q != N_k": ("a &= cols[None, :] <= rows[:, None] + offset",
+                                                                 "a &= cols[None, :] <= rows[:, None]"),
 }
 
 
@@ -54,6 +56,7 @@ def _run_all(mod):
         lambda: pins.check_gradient_identities(mod.forward, mod.backward),
         lambda: pins.check_blocksparse_reductions(mod.forward, mod.backward),
         lambda: pins.check_split_kv_merge(mod.forward, mod.split_kv_forward, mod.merge_partials),
+        lambda: pins.check_rows_unequal_lengths(mod.forward, mod.forward_rows, mod.backward_rows),
     ] + [lambda c=c: c(mod.forward) for c in pins.ALL_FORWARD_CHECKS]
     for c in checks:
         try:

@@ -155,3 +155,7 @@ def test_backward_rows_finite_differences():
             fd = (L(plus["q"], plus["k"], plus["v"]) - L(minus["q"], minus["k"], minus["v"])) / (2 * h)
             an = float(np.sum(g * R))
             assert abs(fd - an) <= 1e-7 * max(1.0, abs(an)), (name, causal, fd, an)
+
+
+def test_row_routines_with_unequal_lengths():
+    pins.check_rows_unequal_lengths(oracle.forward, oracle.forward_rows, oracle.backward_rows)
