@@ -76,6 +76,11 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d);
  * incoming gradient dout = dL/dO, writes dq, dk, dv [B,H,N,d] (dtype):
  *   D = rowsum(dO o O), P = exp(scale*Q K^T - lse), dV = P^T dO,
  *   dP = dO V^T, dS = P o (dP - D), dQ = scale*dS K, dK = scale*dS^T Q.
+ * P is recomputed from Q, K and lse rather than stored ("FlashAttention"
+ * concept card, lukebest.github.io, "反向：重算而非存储"). dS is the softmax
+ * Jacobian applied to dP: the softmax gradient printed in the cloud.baidu.com
+ * explainer ("梯度计算优化") is dimensionally inconsistent, so the textbook
+ * form above is used; D_i = rowsum(P o dP)_i equals rowsum(dO o O)_i.
  * workspace: device buffer of at least fa_bwd_workspace_size() bytes, 256-byte
  * aligned; its contents on entry do not matter and are overwritten.
  */
@@ -94,10 +99,11 @@ fa_status fa_bwd(fa_dtype dtype, const void* q, const void* k, const void* v, co
  * until the process exits. If fa_bwd_workspace_size(B, H, N, d) exceeds it the
  * call returns FA_ERR_UNSUPPORTED and launches nothing. All calls on a device
  * share that array: calls whose kernels may overlap on the GPU race and must be
- * ordered by the caller. The dQ accumulator is re-zeroed by every call. The
- * first call on a device looks up the array's device address
- * (cudaGetSymbolAddress) and caches it; make that first call before any stream
- * capture. Allocates nothing.
+ * ordered by the caller. Nothing in it needs to start at zero: every call's
+ * first kernel rewrites all the entries (D and lse in log2 units) its second
+ * kernel reads. Every other limit is that of fa_bwd. The first call on a device
+ * looks up the array's device address (cudaGetSymbolAddress) and caches it;
+ * make that first call before any stream capture. Allocates nothing.
  */
 #define FA_BWD_NOALLOC_SCRATCH_BYTES (32u << 20)
 fa_status fa_bwd_noalloc(fa_dtype dtype, const void* q, const void* k, const void* v, const void* o,

@@ -220,7 +220,7 @@ def fa_debug_bwd_trace(q, k, v, o, lse, dout, dq, dk, dv, workspace, trace, caus
 
 def fa_debug_bwd_phase(phase: int, q, k, v, o, lse, dout, dq, dk, dv, workspace, causal: bool = False,
                        block_mask=None, scale=None, stream=None) -> None:
-    """One of the backward's three launches (0 prep, 1 main, 2 finish); see include/fa.h."""
+    """One of the backward's two launches (0 prep, 1 main); see include/fa.h."""
     B, H, N, d = _shape(q)
     st = load_library().fa_debug_bwd_phase(int(phase), _dtype_code(q), _ptr(q), _ptr(k), _ptr(v), _ptr(o),
                                            _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace),

@@ -46,16 +46,7 @@ int* status_word() {
 
 bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-fa_status check_common(fa_dtype dtype, int B, int H, int N, int d) {
-  if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_INVALID_ARG;
-  if (B < 1 || H < 1 || N < 1 || d < 1) return FA_ERR_INVALID_ARG;
-  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
-  const long long bh = static_cast<long long>(B) * H;
-  const long long tiles = (static_cast<long long>(N) + 127) / 128;
-  // Grids are 1-D over batch*heads*(2*tiles) CTAs (< 2^31); key-tile indices fit 16 bits.
-  if (bh > 65535 || tiles > 32767 || bh * 2 * tiles > 0x7FFFFFFFLL) return FA_ERR_UNSUPPORTED;
-  return FA_OK;
-}
+using fa::check_common;
 
 // The same limits for a problem with Nq query rows and Nk key rows (the
 // backward grid holds batch*heads*(Tq + Tk) CTAs).
@@ -150,6 +141,17 @@ fa_status bwd_impl(fa_dtype dtype, const void* q, const void* k, const void* v, 
 }  // namespace
 
 int* fa::device_status_word() { return status_word(); }
+
+fa_status fa::check_common(fa_dtype dtype, int B, int H, int N, int d) {
+  if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || N < 1 || d < 1) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  const long long bh = static_cast<long long>(B) * H;
+  const long long tiles = (static_cast<long long>(N) + 127) / 128;
+  // Grids are 1-D over batch*heads*(2*tiles) CTAs (< 2^31); key-tile indices fit 16 bits.
+  if (bh > 65535 || tiles > 32767 || bh * 2 * tiles > 0x7FFFFFFFLL) return FA_ERR_UNSUPPORTED;
+  return FA_OK;
+}
 
 extern "C" {
 

@@ -1,23 +1,23 @@
 // fa_bwd_noalloc: the backward for callers that cannot allocate device memory.
 //
-// fa_bwd needs a device workspace (an fp32 dQ accumulator and two fp32 row
-// vectors). Some callers have no way to provide one: a host application that
-// plans every byte of device memory up front and gives plugins no allocator,
-// or a latency-critical loop in which cudaMalloc (which may synchronise the
-// device and may fail) is not allowed. For them this entry point keeps its
-// scratch in a fixed array in the library's own static device memory, so no
-// call allocates anything.
+// fa_bwd needs a device workspace (two fp32 row vectors: D = rowsum(dO o O) and
+// lse in log2 units). Some callers have no way to provide one: a host
+// application that plans every byte of device memory up front and gives plugins
+// no allocator, or a latency-critical loop in which cudaMalloc (which may
+// synchronise the device and may fail) is not allowed. For them this entry point
+// keeps that workspace in a fixed array in the library's own static device
+// memory, so no call allocates anything.
 //
 // Limits and sharing:
 //   * The array holds FA_BWD_NOALLOC_SCRATCH_BYTES bytes on every GPU that loads
 //     the library, for the life of the process. Problems whose workspace
 //     (fa_bwd_workspace_size) is larger are rejected with FA_ERR_UNSUPPORTED
-//     before anything is launched.
+//     before anything is launched; every other limit is that of fa_bwd.
 //   * Every call on a device uses the same array. Calls whose kernels overlap
 //     on the GPU (different streams without ordering between them) race on it
-//     and give wrong gradients; callers must order such calls. Each call
-//     re-initialises what must start at zero (the dQ accumulator) in its first
-//     kernel, so leftovers from the previous call do not matter.
+//     and give wrong gradients; callers must order such calls. Nothing in the
+//     array has to start at zero: each call's first kernel rewrites every entry
+//     its second kernel reads, so what the previous call left does not matter.
 //   * The first call on a device looks up the array's device address with
 //     cudaGetSymbolAddress (a host-side stand-in name is not a device address)
 //     and caches it; that first call should come before any stream capture.
@@ -62,14 +62,12 @@ bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr
 extern "C" fa_status fa_bwd_noalloc(fa_dtype dtype, const void* q, const void* k, const void* v, const void* o,
                                     const float* lse, const void* dout, void* dq, void* dk, void* dv, int B, int H,
                                     int N, int d, float softmax_scale, int causal, cudaStream_t stream) {
-  if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_INVALID_ARG;
-  if (B < 1 || H < 1 || N < 1) return FA_ERR_INVALID_ARG;
-  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  // The same limits as fa_bwd, then the size of the static array.
+  const fa_status st = fa::check_common(dtype, B, H, N, d);
+  if (st != FA_OK) return st;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) || !aligned16(dout) ||
       !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
     return FA_ERR_INVALID_ARG;
-  const long long tiles = (static_cast<long long>(N) + 127) / 128;
-  if (static_cast<long long>(B) * H > 0x7FFFFFFFLL || tiles > 65535) return FA_ERR_UNSUPPORTED;
   const fa::BwdWorkspace ws = fa::bwd_workspace_layout(B, H, N, d);
   if (ws.total > static_cast<size_t>(FA_BWD_NOALLOC_SCRATCH_BYTES)) return FA_ERR_UNSUPPORTED;
 
@@ -98,5 +96,6 @@ extern "C" fa_status fa_bwd_noalloc(fa_dtype dtype, const void* q, const void* k
   a.block_mask = nullptr;
   a.trace = nullptr;
   a.status = fa::device_status_word();
+  if (a.status == nullptr) return FA_ERR_CUDA;
   return fa::launch_bwd(a, stream) == 0 ? FA_OK : FA_ERR_CUDA;
 }

@@ -5,6 +5,8 @@
 
 #include <cstdint>
 
+#include "fa.h"
+
 namespace fa {
 
 struct AttnArgs {
@@ -44,5 +46,9 @@ int bwd_row_tile(int d);
 
 // Device address of the per-device status word (nullptr on failure).
 int* device_status_word();
+
+// Limits every entry point applies to the element type and sizes of a square
+// (N queries, N keys) problem: FA_OK, FA_ERR_INVALID_ARG or FA_ERR_UNSUPPORTED.
+fa_status check_common(fa_dtype dtype, int B, int H, int N, int d);
 
 }  // namespace fa

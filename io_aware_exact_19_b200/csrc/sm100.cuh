@@ -158,16 +158,6 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
-// 3-D tiled element-wise add shared -> global (fp32 reduction in L2).
-__device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* map, uint32_t src,
-                                                  int c0, int c1, int c2) {
-  asm volatile(
-      "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group"
-      " [%0, {%2, %3, %4}], [%1];" ::"l"(reinterpret_cast<uint64_t>(map)),
-      "r"(src), "r"(c0), "r"(c1), "r"(c2)
-      : "memory");
-}
-
 // 3-D tiled store shared -> global.
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, uint32_t src,
                                              int c0, int c1, int c2) {
@@ -186,11 +176,6 @@ __device__ __forceinline__ void bulk_commit_group() {
 template <int N>
 __device__ __forceinline__ void bulk_wait_group_read() {
   asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
-}
-
-template <int N>
-__device__ __forceinline__ void bulk_wait_group() {
-  asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
 }
 
 // Contiguous bulk copy global -> shared (16-byte aligned, size a multiple of 16).

@@ -46,3 +46,51 @@ def max_abs(a, b):
 def rel_fro(a, b):
     a, b = np.asarray(a, np.float64), np.asarray(b, np.float64)
     return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-30))
+
+
+def grad_errors(g, G, tile=128, floor=1e-4):
+    """Errors of a gradient g against the oracle's G, both [heads, rows, d]:
+
+    * ``fro``: relative Frobenius error over the whole tensor (the stated metric);
+    * ``tile``: the worst relative Frobenius error of one block of ``tile``
+      consecutive rows of one head, its denominator floored at the norm such a
+      block would have at the tensor's RMS, so one wrong row or ragged tail tile
+      cannot hide inside a large tensor;
+    * ``elem``: the largest element error in units of the tensor's RMS.
+
+    The RMS has an absolute floor (``floor``) so a gradient that is exactly zero in
+    exact arithmetic (a single key: P = 1, dS = 0) is compared against that scale.
+    """
+    g = np.asarray(g, np.float64)
+    G = np.asarray(G, np.float64)
+    assert g.shape == G.shape, (g.shape, G.shape)
+    err = g - G
+    rms = max(float(np.sqrt(np.mean(G * G))) if G.size else 0.0, floor)
+    fro = float(np.linalg.norm(err) / max(np.linalg.norm(G), rms * np.sqrt(max(G.size, 1))))
+    worst = 0.0
+    rows = G.shape[-2]
+    E = err.reshape((-1,) + G.shape[-2:])
+    R = G.reshape((-1,) + G.shape[-2:])
+    for r0 in range(0, rows, tile):
+        e_blk = E[:, r0:r0 + tile]
+        g_blk = R[:, r0:r0 + tile]
+        num = np.sqrt((e_blk * e_blk).sum(axis=(1, 2)))
+        den = np.maximum(np.sqrt((g_blk * g_blk).sum(axis=(1, 2))), rms * np.sqrt(e_blk[0].size))
+        worst = max(worst, float(np.max(num / den)))
+    elem = float(np.max(np.abs(err)) / rms) if err.size else 0.0
+    return {"fro": fro, "tile": worst, "elem": elem}
+
+
+# Gradient bounds: relative Frobenius <= 2e-2 over the tensor and over every block
+# of rows; every element within 0.1 x RMS (five times the Frobenius bound: a
+# single wrong element of typical size fails it).
+G_TOL = 2e-2
+G_ELEM_TOL = 0.1
+
+
+def assert_grads(pairs, tile=128, what="dQ/dK/dV"):
+    """Assert the gradient bounds for a sequence of (g, G) pairs; returns their errors."""
+    errs = [grad_errors(g, G, tile) for g, G in pairs]
+    bad = [e for e in errs if e["fro"] > G_TOL or e["tile"] > G_TOL or e["elem"] > G_ELEM_TOL]
+    assert not bad, f"{what} errors {errs}"
+    return errs

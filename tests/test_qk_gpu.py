@@ -3,19 +3,19 @@ fp64 oracle. The causal mask is bottom-right aligned: query i sees key j iff
 j <= i + N_k - N_q, so a query block of N_q rows is the last N_q positions of
 the key sequence; rows with no key get O = 0, lse = -inf and no gradient.
 Tolerances as for the square case: O max-abs <= 1e-2, lse max-abs <= 1e-3,
-dQ/dK/dV relative Frobenius <= 2e-2."""
+dQ/dK/dV relative Frobenius <= 2e-2 over each tensor and each 128-row block, and
+every element within 0.1 x the gradient's RMS."""
 import numpy as np
 import pytest
 import torch
 
 import io_aware_exact_19_b200 as fa
 import oracle
-from tests.gpu_inputs import Case, max_abs
-from tests.test_bwd_gpu import _grad_err
+from tests.gpu_inputs import Case, assert_grads, max_abs
 
 pytestmark = pytest.mark.gpu
 
-O_TOL, LSE_TOL, G_TOL = 1e-2, 1e-3, 2e-2
+O_TOL, LSE_TOL = 1e-2, 1e-3
 
 
 def _run_qk(B, H, Nq, Nk, d, fmt, causal, mask=None):
@@ -39,8 +39,7 @@ def _run_qk(B, H, Nq, Nk, d, fmt, causal, mask=None):
     eo = max_abs(cq.flat(o), O)
     el = max_abs(lse.cpu().numpy().reshape(B * H, Nq), LSE)
     assert eo <= O_TOL and el <= LSE_TOL, f"O {eo:.3e} lse {el:.3e}"
-    errs = [_grad_err(cq.flat(dq), DQ), _grad_err(ck.flat(dk), DK), _grad_err(ck.flat(dv), DV)]
-    assert max(errs) <= G_TOL, f"rel Frobenius dQ/dK/dV = {errs}"
+    assert_grads([(cq.flat(dq), DQ), (ck.flat(dk), DK), (ck.flat(dv), DV)])
     for g in (o, dq, dk, dv):
         assert torch.isfinite(g).all()
     return o, lse, dq

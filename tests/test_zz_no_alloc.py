@@ -4,10 +4,10 @@ Those callers (a host application that plans all device memory itself and gives
 this library no allocator, or a latency-critical loop where cudaMalloc is not
 allowed) call fa_bwd_noalloc, whose scratch lives in a fixed static array inside
 the library. This test calls it through the C ABI twice in a row and checks each
-result against fa_bwd (which takes a caller-provided workspace) with the
-gradient tolerance the parity tests use, and that a problem whose workspace does
-not fit the static array is rejected before anything runs. The file is named so
-that pytest collects it after every other test file.
+result against fa_bwd (which takes a caller-provided workspace) and against the
+fp64 oracle, with the gradient bounds the parity tests use, and that a problem
+whose workspace does not fit the static array is rejected before anything runs.
+The file is named so that pytest collects it after every other test file.
 """
 import ctypes
 
@@ -15,7 +15,8 @@ import pytest
 import torch
 
 import io_aware_exact_19_b200 as fa
-from tests.gpu_inputs import Case
+import oracle
+from tests.gpu_inputs import Case, assert_grads
 
 pytestmark = pytest.mark.gpu
 
@@ -36,6 +37,8 @@ def test_noalloc_backward_matches_workspace_backward(B, H, N, d, causal):
     o, lse = fa.attention_forward(q, k, v, causal=causal)
     ref = fa.attention_backward(q, k, v, o, lse, do, causal=causal)
     torch.cuda.synchronize()
+    vals = [c.values(n) for n in ("q", "k", "v", "do")]
+    exact = oracle.backward(*vals, c.scale, causal=causal)
     for _ in range(2):  # two calls in a row share the static scratch
         dq, dk, dv = (torch.full_like(t, float("nan")) for t in (q, k, v))
         fa.fa_bwd_noalloc(q, k, v, o, lse, do, dq, dk, dv, causal=causal)
@@ -44,6 +47,7 @@ def test_noalloc_backward_matches_workspace_backward(B, H, N, d, causal):
         for got, exp in zip((dq, dk, dv), ref):
             assert torch.isfinite(got).all()
             assert _rel(got, exp) <= G_TOL
+        assert_grads([(c.flat(g), G) for g, G in zip((dq, dk, dv), exact)])
 
 
 def test_noalloc_rejects_problems_larger_than_its_scratch():
