@@ -171,6 +171,24 @@ def oracle_inputs(w, heads, seed=0):
     return {n: fa_synth.bits_to_values(b.reshape((-1,) + b.shape[2:])[heads], w["fmt"]) for n, b in bits.items()}
 
 
+def cpu_description():
+    """Model name and logical core count of the host running the oracle."""
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.lower().startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    try:
+        usable = len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):
+        usable = os.cpu_count() or 1
+    return {"cpu_model": model, "nproc": usable}
+
+
 def blas_threads():
     try:
         from threadpoolctl import threadpool_info
@@ -260,7 +278,8 @@ def run_reference(args, w, rank, world):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": config_block(w, args.workload),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle", "sample": sample,
+                         **cpu_description()},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -287,56 +306,138 @@ def config_block(w, name):
 
 # ----------------------------------------------------------------------------- GPU arm
 
+class Problem:
+    """Device buffers of one workload (seeded synthetic inputs) and its launches
+    through the binding of the C ABI."""
+
+    def __init__(self, w, dev, seed):
+        import numpy as np
+        import torch
+
+        import fa_synth
+        import io_aware_exact_19_b200 as fa
+
+        self.fa = fa
+        self.w = w
+        B, H, N, d = w["B"], w["H"], w["N"], w["d"]
+        tdt = torch.bfloat16 if w["fmt"] == "bf16" else torch.float16
+        bits = fa_synth.attention_input_bits(B, H, N, d, w["fmt"], seed=seed)
+        self.host = {n: torch.from_numpy(b.view(np.int16)).view(tdt) for n, b in bits.items()}
+        self.q, self.k, self.v, self.do = (self.host[n].to(dev) for n in ("q", "k", "v", "do"))
+        self.mask = None
+        if w["mask"]:
+            self.mask = torch.from_numpy(fa_synth.block_mask_recipe(N // 128)).to(dev)
+        self.o = torch.empty_like(self.q)
+        self.lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+        self.dq, self.dk, self.dv = (torch.empty_like(t) for t in (self.q, self.k, self.v))
+        self.ws = torch.empty(fa.fa_bwd_workspace_size(B, H, N, d), dtype=torch.uint8, device=dev)
+        self.stream = torch.cuda.current_stream()
+
+    def fwd(self):
+        fa, w = self.fa, self.w
+        if self.mask is None:
+            fa.fa_fwd(self.q, self.k, self.v, self.o, self.lse, w["causal"])
+        else:
+            fa.fa_blocksparse_fwd(self.q, self.k, self.v, self.o, self.lse, self.mask, w["causal"])
+
+    def bwd_phase(self, ph):
+        self.fa.fa_debug_bwd_phase(ph, self.q, self.k, self.v, self.o, self.lse, self.do, self.dq, self.dk, self.dv,
+                                   self.ws, causal=self.w["causal"], block_mask=self.mask)
+
+    def bwd(self):
+        fa, w = self.fa, self.w
+        if self.mask is None:
+            fa.fa_bwd(self.q, self.k, self.v, self.o, self.lse, self.do, self.dq, self.dk, self.dv, self.ws,
+                      w["causal"])
+        else:
+            fa.fa_blocksparse_bwd(self.q, self.k, self.v, self.o, self.lse, self.do, self.dq, self.dk, self.dv,
+                                  self.ws, self.mask, w["causal"])
+
+    def step(self, ev=None):
+        """Forward, then the backward's two launches (prep, main); `ev` = four CUDA
+        events recorded on the launching stream around them."""
+        if ev is not None:
+            ev[0].record(self.stream)
+        self.fwd()
+        if ev is not None:
+            ev[1].record(self.stream)
+        self.bwd_phase(0)
+        if ev is not None:
+            ev[2].record(self.stream)
+        self.bwd_phase(1)
+        if ev is not None:
+            ev[3].record(self.stream)
+
+
+def timed_steps(prob, steps, warmup, dev, flush_l2, between=None):
+    """Run `warmup` untimed steps, then `steps` steps each bracketed by CUDA events
+    on the launching stream. With `flush_l2`, a buffer twice the L2 size is written
+    between steps, outside the events. Returns per-step (total, fwd, prep, main) ms."""
+    import torch
+    for _ in range(max(warmup, 3)):
+        prob.step()
+    torch.cuda.synchronize()
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev) if flush_l2 else None
+    if between is not None:
+        between()
+    for s in range(steps):
+        if flush is not None:
+            flush.fill_(s & 0xFF)
+        prob.step(events[s])
+    torch.cuda.synchronize()
+    return [(e[0].elapsed_time(e[3]), e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3]))
+            for e in events]
+
+
+def prep_bytes(w):
+    """Algorithmic bytes of the backward's prep launch: read O, dO (16-bit) and lse;
+    write D and lse in log2 units (fp32)."""
+    return w["B"] * w["H"] * w["N"] * (w["d"] * 2 * 2 + 4 * 3)
+
+
+def summarize(w, times, peaks):
+    """Per-launch averages and rates of one workload's timed steps."""
+    f_fwd, f_bwd = step_flops(w)
+    n = len(times)
+    fwd = sum(t[1] for t in times) / n
+    prep = sum(t[2] for t in times) / n
+    main = sum(t[3] for t in times) / n
+    tot = sum(t[0] for t in times) / n
+    bwd = prep + main
+    return {
+        "ms_per_step": tot, "step_tflops": (f_fwd + f_bwd) / (tot * 1e-3) / 1e12,
+        "fwd_ms": fwd, "fwd_tflops": f_fwd / (fwd * 1e-3) / 1e12,
+        "fwd_frac_of_measured_peak": f_fwd / (fwd * 1e-3) / 1e12 / peaks["bf16"],
+        "bwd_ms": bwd, "bwd_tflops": f_bwd / (bwd * 1e-3) / 1e12,
+        "bwd_frac_of_measured_peak": f_bwd / (bwd * 1e-3) / 1e12 / peaks["bf16"],
+        "bwd_main_ms": main, "bwd_main_tflops": f_bwd / (main * 1e-3) / 1e12,
+        "bwd_prep_ms": prep, "bwd_prep_gbs": prep_bytes(w) / (prep * 1e-3) / 1e9,
+        "bwd_prep_frac_of_measured_hbm": prep_bytes(w) / (prep * 1e-3) / 1e9 / peaks["hbm"],
+        # Algorithmic HBM bytes of the whole step (Q, K, V, dO read once; O, dQ, dK,
+        # dV and lse written once) over its time: the figure that matters for the
+        # small cases, which are latency rather than tensor bound.
+        "step_min_hbm_gbs": (w["B"] * w["H"] * w["N"] * (w["d"] * 2 * 8 + 4)) / (tot * 1e-3) / 1e9,
+        "vendor_peak_tflops": 2250.0,
+        "fwd_frac_of_vendor_peak": f_fwd / (fwd * 1e-3) / 1e12 / 2250.0,
+        "bwd_frac_of_vendor_peak": f_bwd / (bwd * 1e-3) / 1e12 / 2250.0,
+        "steps": n,
+    }
+
+
 def run_gpu(args, w, rank, world, local_rank):
-    import numpy as np
     import torch
     import torch.distributed as dist
 
-    import fa_synth
     import io_aware_exact_19_b200 as fa
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     B, H, N, d = w["B"], w["H"], w["N"], w["d"]
-    causal = w["causal"]
-    tdt = torch.bfloat16 if w["fmt"] == "bf16" else torch.float16
-
-    bits = fa_synth.attention_input_bits(B, H, N, d, w["fmt"], seed=rank_seed(rank))
-    host = {n: torch.from_numpy(b.view(np.int16)).view(tdt) for n, b in bits.items()}
-    q, k, v, do = (host[n].to(dev) for n in ("q", "k", "v", "do"))
-    mask = None
-    if w["mask"]:
-        mask = torch.from_numpy(fa_synth.block_mask_recipe(N // 128)).to(dev)
-    o = torch.empty_like(q)
-    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    ws = torch.empty(fa.fa_bwd_workspace_size(B, H, N, d), dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream()
-
-    def fwd():
-        if mask is None:
-            fa.fa_fwd(q, k, v, o, lse, causal)
-        else:
-            fa.fa_blocksparse_fwd(q, k, v, o, lse, mask, causal)
-
-    def bwd_phase(ph):
-        fa.fa_debug_bwd_phase(ph, q, k, v, o, lse, do, dq, dk, dv, ws, causal=causal, block_mask=mask)
-
-    def step(ev=None):
-        if ev is not None:
-            ev[0].record(stream)
-        fwd()
-        if ev is not None:
-            ev[1].record(stream)
-        bwd_phase(0)
-        if ev is not None:
-            ev[2].record(stream)
-        bwd_phase(1)
-        if ev is not None:
-            ev[3].record(stream)
+    prob = Problem(w, dev, rank_seed(rank))
 
     for _ in range(max(args.warmup, 3)):
-        step()
+        prob.step()
     torch.cuda.synchronize()
     if fa.fa_device_status() != fa.FA_OK:
         raise RuntimeError("device status reported a time-out during warm-up")
@@ -345,66 +446,56 @@ def run_gpu(args, w, rank, world, local_rank):
     gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
     sampler = ClockSampler(gpu_id, os.path.join(tempfile.gettempdir(), f"fa_bench_clocks_rank{rank}_{os.getpid()}.csv"))
     time.sleep(0.3)
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    t_wall0 = time.time()
-    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev) if needs_l2_flush(w) else None
-    for s in range(args.steps):
-        if flush is not None:
-            flush.fill_(s & 0xFF)
-        step(events[s])
-    torch.cuda.synchronize()
+    marks = {}
+
+    def start():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        marks["t0"] = time.time()
+
+    times = timed_steps(prob, args.steps, 0, dev, needs_l2_flush(w), between=start)
     t_wall1 = time.time()
     if world > 1:
         dist.barrier()
     time.sleep(0.2)
     sampler.stop()
-    clocks = sampler.summary(t_wall0, t_wall1)
+    clocks = sampler.summary(marks["t0"], t_wall1)
     status = fa.fa_device_status()
 
     # Sum of the per-step spans (first to last launch of each step): the L2 flush
     # between steps, where there is one, stays outside.
-    ms_total = sum(e[0].elapsed_time(e[3]) for e in events)
-    fwd_ms = [e[0].elapsed_time(e[1]) for e in events]
-    prep_ms = [e[1].elapsed_time(e[2]) for e in events]
-    main_ms = [e[2].elapsed_time(e[3]) for e in events]
-    ms_total, main_sum, fwd_sum = max_over_ranks([ms_total, sum(main_ms), sum(fwd_ms)], dev, world)
+    ms_total = sum(t[0] for t in times)
+    main_sum = sum(t[3] for t in times)
+    fwd_sum = sum(t[1] for t in times)
+    ms_total, main_sum, fwd_sum = max_over_ranks([ms_total, main_sum, fwd_sum], dev, world)
 
     f_fwd, f_bwd = step_flops(w)
     value = whole_job_tflops(f_fwd + f_bwd, args.steps, world, ms_total)
     peaks = load_peaks()
     main_avg = main_sum / args.steps
-    fwd_avg = fwd_sum / args.steps
     achieved = f_bwd / (main_avg * 1e-3) / 1e12
-    bwd_all = statistics.mean(p + m for p, m in zip(prep_ms, main_ms))
-    prep_avg = statistics.mean(prep_ms)
-    prep_bytes = B * H * N * d * (2 + 2) + B * H * N * 4 * 3  # read O, dO and lse; write D and lse2
+    breakdown = summarize(w, times, peaks)
 
     # ---- end to end through the C ABI: pinned host inputs in, results back to pinned host memory
-    pin = {n: t.pin_memory() for n, t in host.items()}
-    out_host = {n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for n, t in
-                (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv))}
+    pin = {n: t.pin_memory() for n, t in prob.host.items()}
+    outs = (("o", prob.o), ("lse", prob.lse), ("dq", prob.dq), ("dk", prob.dk), ("dv", prob.dv))
+    out_host = {n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for n, t in outs}
     e2e_steps = max(1, min(args.steps, 20))
 
     def e2e_step():
-        q.copy_(pin["q"], non_blocking=True)
-        k.copy_(pin["k"], non_blocking=True)
-        v.copy_(pin["v"], non_blocking=True)
-        do.copy_(pin["do"], non_blocking=True)
-        fwd()
-        if mask is None:
-            fa.fa_bwd(q, k, v, o, lse, do, dq, dk, dv, ws, causal)
-        else:
-            fa.fa_blocksparse_bwd(q, k, v, o, lse, do, dq, dk, dv, ws, mask, causal)
-        for n, t in (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv)):
+        for n in ("q", "k", "v", "do"):
+            getattr(prob, n).copy_(pin[n], non_blocking=True)
+        prob.fwd()
+        prob.bwd()
+        for n, t in outs:
             out_host[n].copy_(t, non_blocking=True)
 
     e2e_step()
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
+    stream = torch.cuda.current_stream()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(e2e_steps):
@@ -415,6 +506,26 @@ def run_gpu(args, w, rank, world, local_rank):
     h2d = sum(t.numel() * t.element_size() for t in pin.values())
     d2h = sum(t.numel() * t.element_size() for t in out_host.values())
     e2e_value = whole_job_tflops(f_fwd + f_bwd, e2e_steps, world, e2e_ms)
+    del prob
+
+    # ---- the other workloads, each timed the same way (after the headline, outside its timed region)
+    per_workload = {}
+    if not args.no_per_workload:
+        for name, ow in WORKLOADS.items():
+            if name == args.workload:
+                continue
+            p2 = Problem(ow, dev, rank_seed(rank))
+            steps = 10 if ow["N"] >= 32768 else 50
+            t2 = timed_steps(p2, steps, 3, dev, needs_l2_flush(ow))
+            st2 = fa.fa_device_status()
+            tot = max_over_ranks([sum(t[0] for t in t2)], dev, world)[0]
+            ff, fb = step_flops(ow)
+            rec = {"workload": ow["desc"], "value": whole_job_tflops(ff + fb, steps, world, tot),
+                   "unit": UNIT, "l2": config_block(ow, name)["l2"], "device_status": int(st2)}
+            rec.update(summarize(ow, t2, peaks))
+            per_workload[name] = rec
+            del p2
+            torch.cuda.empty_cache()
 
     if rank != 0:
         return 0
@@ -425,7 +536,7 @@ def run_gpu(args, w, rank, world, local_rank):
         rate, n_steps, secs = cpu_rate(w, vals, 512 if N >= 4096 else min(N, 256), budget_s=12.0)
         cpu = {"value": rate, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
                "sample": f"{n_steps} samples x 512 of {N} query rows of one (batch, head), forward + backward "
-                         f"of the loss on those rows, fp64, {secs:.1f} s"}
+                         f"of the loss on those rows, fp64, {secs:.1f} s", **cpu_description()}
 
     kernel_key = f"fa_bwd_main_kernel<{d},{'bf16' if w['fmt'] == 'bf16' else 'fp16'}>"
     line = {
@@ -439,28 +550,31 @@ def run_gpu(args, w, rank, world, local_rank):
                          "; fp16 MMAs run at the bf16 rate (nominal ratio 1)" if w["fmt"] == "fp16" else ""),
                      "traffic": load_traffic(kernel_key),
                      "flops_per_launch": f_bwd},
-        "breakdown": {
-            "fwd_ms": fwd_avg, "fwd_tflops": f_fwd / (fwd_avg * 1e-3) / 1e12,
-            "fwd_frac_of_measured_peak": f_fwd / (fwd_avg * 1e-3) / 1e12 / peaks["bf16"],
-            "bwd_ms": bwd_all, "bwd_tflops": f_bwd / (bwd_all * 1e-3) / 1e12,
-            "bwd_frac_of_measured_peak": f_bwd / (bwd_all * 1e-3) / 1e12 / peaks["bf16"],
-            "bwd_main_ms": main_avg, "bwd_prep_ms": prep_avg,
-            "bwd_prep_gbs": prep_bytes / (prep_avg * 1e-3) / 1e9,
-            "vendor_peak_tflops": 2250.0,
-            "fwd_frac_of_vendor_peak": f_fwd / (fwd_avg * 1e-3) / 1e12 / 2250.0,
-            "bwd_frac_of_vendor_peak": f_bwd / (bwd_all * 1e-3) / 1e12 / 2250.0,
-        },
+        "breakdown": breakdown,
+        "per_workload": per_workload,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": e2e_steps},
         "gpu_launches": 3 * args.steps,
         "clocks": clocks,
         "device_status": int(status),
-        "wall_s_timed_region": t_wall1 - t_wall0,
+        "wall_s_timed_region": t_wall1 - marks["t0"],
     }
     if cpu is not None:
         line["cpu_baseline"] = cpu
     print(json.dumps(line), flush=True)
     return 0
+
+
+def spawn_ranks(n, argv):
+    """Run this script as n ranks, one process per GPU, under torch.distributed.run
+    (rendezvous on 127.0.0.1); returns its exit status."""
+    import socket
+    with socket.socket() as sock:
+        sock.bind(("127.0.0.1", 0))
+        port = sock.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", str(n),
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__), *argv]
+    return subprocess.call(cmd)
 
 
 def main(argv=None):
@@ -471,15 +585,20 @@ def main(argv=None):
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-workload", action="store_true",
+                    help="time only the selected workload (the default also times every other one)")
     ap.add_argument("--reference-seconds", type=float, default=120.0,
                     help="approximate CPU time budget of the reference arm (warm-up plus timed steps)")
     args = ap.parse_args(argv)
     w = WORKLOADS[args.workload]
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        return spawn_ranks(args.gpus, sys.argv[1:] if argv is None else list(argv))
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
-    if world != args.gpus and "RANK" in os.environ:
-        print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
+    if world != args.gpus:
+        print(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={world}; launch one process per GPU", file=sys.stderr)
+        return 2
     if args.impl == "reference":
         return run_reference(args, w, rank, world)
     if world > 1:
