@@ -425,6 +425,61 @@ def summarize(w, times, peaks):
     }
 
 
+DECODE = dict(B=1, H=16, Nq=1, Nk=65536, d=64, fmt="bf16", causal=True,
+              desc="decoding: one query row against a 64K key cache, B=1 H=16 d=64 bf16, split-KV forward")
+
+
+def time_decode(dev, peaks, steps=50):
+    """Split-KV forward (fa_fwd_splitkv) on the decoding shape, against the same
+    forward without splitting (fa_fwd_qk). HBM bound: the bytes are K and V
+    (read once) plus Q, O and lse; the L2 is flushed between steps."""
+    import numpy as np
+    import torch
+
+    import fa_synth
+    import io_aware_exact_19_b200 as fa
+
+    w = DECODE
+    B, H, Nq, Nk, d = w["B"], w["H"], w["Nq"], w["Nk"], w["d"]
+    bq = fa_synth.attention_input_bits(B, H, Nq, d, w["fmt"], seed=11)
+    bk = fa_synth.attention_input_bits(B, H, Nk, d, w["fmt"], seed=12)
+    to = lambda b: torch.from_numpy(b.view(np.int16)).view(torch.bfloat16).to(dev)
+    q, k, v = to(bq["q"]), to(bk["k"]), to(bk["v"])
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, Nq), dtype=torch.float32, device=dev)
+    ns = fa.fa_fwd_splitkv_splits(B, H, Nq, Nk)
+    ws = torch.empty(fa.fa_fwd_splitkv_workspace_size(B, H, Nq, d, ns), dtype=torch.uint8, device=dev)
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        tot = 0.0
+        for i in range(steps):
+            flush.fill_(i & 0xFF)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            tot += e0.elapsed_time(e1)
+        return tot / steps
+
+    ms_split = timed(lambda: fa.fa_fwd_splitkv(q, k, v, o, lse, ns, ws, causal=w["causal"]))
+    ms_plain = timed(lambda: fa.fa_fwd_qk(q, k, v, o, lse, causal=w["causal"]))
+    status = fa.fa_device_status()
+    nbytes = 2 * B * H * Nk * d * 2 + 2 * B * H * Nq * d * 2 + B * H * Nq * 4
+    flops = 4.0 * B * H * Nq * Nk * d
+    gbs = nbytes / (ms_split * 1e-3) / 1e9
+    return {"workload": w["desc"], "n_splits": ns, "ms": ms_split, "hbm_gbs": gbs,
+            "hbm_frac_of_measured_peak": gbs / peaks["hbm"], "tflops": flops / (ms_split * 1e-3) / 1e12,
+            "unsplit_ms": ms_plain, "speedup_vs_unsplit": ms_plain / ms_split,
+            "bytes_per_step": nbytes, "l2": "L2 flushed between steps", "device_status": int(status),
+            "launches_per_step": 2, "steps": steps}
+
+
 def run_gpu(args, w, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -526,6 +581,8 @@ def run_gpu(args, w, rank, world, local_rank):
             per_workload[name] = rec
             del p2
             torch.cuda.empty_cache()
+        per_workload["decode_splitkv_64k"] = time_decode(dev, peaks)
+        torch.cuda.empty_cache()
 
     if rank != 0:
         return 0

@@ -18,8 +18,10 @@
  *     [B, H, N]. All are DEVICE pointers, 16-byte aligned.
  *   - lse_i = ln sum_j exp(scale * q_i . k_j) over the keys row i may see
  *     (natural log, in the units of the scaled scores).
- *   - d must be 64 or 128; N >= 1 (any value; ragged last tiles are handled);
- *     B, H >= 1 and B*H <= 65535.
+ *   - d must be 32, 64, 96 or 128 (32 and 96 run in the 64 and 128 kernels
+ *     with the missing columns zero-filled, at the cost of the padded width);
+ *     N >= 1 (any value; ragged last tiles are handled); B, H >= 1 and
+ *     B*H <= 65535.
  *   - causal != 0 masks key j > query i (top-left aligned; the essay's
  *     section 3.1 causal mask P_ij = 0 for j > i).
  *   - The caller owns all memory. The library allocates no device memory; the
@@ -47,7 +49,7 @@ extern "C" {
 typedef enum {
   FA_OK = 0,
   FA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, non-positive size, bad dtype */
-  FA_ERR_UNSUPPORTED = 2, /* valid but unsupported shape (d not 64/128, size limits) */
+  FA_ERR_UNSUPPORTED = 2, /* valid but unsupported shape (d not 32/64/96/128, size limits) */
   FA_ERR_CUDA = 3,        /* a CUDA runtime call or kernel launch failed */
   FA_ERR_TIMEOUT = 4      /* a device-side wait gave up (see fa_device_status) */
 } fa_status;
@@ -154,6 +156,36 @@ fa_status fa_bwd_qk(fa_dtype dtype, const void* q, const void* k, const void* v,
                     int d, float softmax_scale, int causal, const uint8_t* block_mask, cudaStream_t stream);
 
 /*
+ * Split-KV forward (FlashDecoding, the "FlashAttention" concept card's lineage
+ * table: partial softmax per key range, then a synchronising merge). Computes
+ * exactly what fa_fwd_qk computes, with more parallelism when B*H*ceil(Nq/128)
+ * is small next to the GPU (decoding: a few query rows against a long key
+ * sequence). The Nk keys are cut into n_splits consecutive ranges of whole
+ * 128-key tiles: range s holds key tiles [s*T/n_splits, (s+1)*T/n_splits),
+ * T = ceil(Nk/128). Step 1 computes, for every query row and range, the
+ * softmax-weighted mean of that range's values, O_s (fp32), and the log of its
+ * exp-sum, lse_s (fp32, -inf if the row has no allowed key in the range); step 2
+ * merges them: lse = log sum_s exp(lse_s), O = sum_s exp(lse_s - lse) O_s (the
+ * online-softmax update of the interview explainer, section 3.2, applied to
+ * whole ranges).
+ * Arguments as fa_fwd_qk (q, o [B,H,Nq,d]; k, v [B,H,Nk,d]; lse [B,H,Nq];
+ * bottom-right causal; optional block_mask [Nq/128][Nk/128]), plus:
+ *   n_splits  1 <= n_splits <= ceil(Nk/128) (else FA_ERR_INVALID_ARG);
+ *             fa_fwd_splitkv_splits() suggests one.
+ *   workspace DEVICE buffer of fa_fwd_splitkv_workspace_size() bytes, 256-byte
+ *             aligned, owned by the caller; on return (after the stream
+ *             completes) it holds the partials: O_s as fp32
+ *             [n_splits][B*H][Nq][d] at offset 0, then lse_s as fp32
+ *             [n_splits][B*H][Nq] at the next 256-byte boundary after O_s.
+ * Two launches on `stream`; asynchronous, allocates nothing.
+ */
+size_t fa_fwd_splitkv_workspace_size(int B, int H, int Nq, int d, int n_splits);
+int fa_fwd_splitkv_splits(int B, int H, int Nq, int Nk);
+fa_status fa_fwd_splitkv(fa_dtype dtype, const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                         int H, int Nq, int Nk, int d, float softmax_scale, int causal, const uint8_t* block_mask,
+                         int n_splits, void* workspace, cudaStream_t stream);
+
+/*
  * Debug: the forward / backward with a record of the tiles each CTA loaded.
  * trace: DEVICE int32 buffer of fa_*_trace_size() entries; each record is a
  * count followed by entries (tile index) | (flags << 16).
@@ -203,6 +235,19 @@ fa_status fa_device_status(cudaStream_t stream);
  * the status word and the CTA exits normally. Used to test the time-out path.
  */
 fa_status fa_debug_timeout_probe(int timeout_ms, cudaStream_t stream);
+
+/*
+ * Debug: the real forward kernel with its TMA producer issuing no load at all
+ * and every device-side wait limited to `timeout_ms` (1..5000). The MMA
+ * issuer's first wait (for Q) runs out, records FA_ERR_TIMEOUT in the status
+ * word and raises the CTA's abort flag; every role then leaves its loop, and,
+ * as nothing was issued, nothing is in flight when the CTAs exit. o and lse
+ * are not written. Used to test the abort path of the production kernel
+ * without a fault. Arguments otherwise as fa_fwd.
+ */
+fa_status fa_debug_fwd_withhold(fa_dtype dtype, const void* q, const void* k, const void* v, void* o, float* lse,
+                                int B, int H, int N, int d, float softmax_scale, int causal, int timeout_ms,
+                                cudaStream_t stream);
 
 #ifdef __cplusplus
 }

@@ -25,7 +25,8 @@ EXPORTED = (
     "fa_status_string", "fa_fwd", "fa_bwd", "fa_blocksparse_fwd", "fa_blocksparse_bwd",
     "fa_bwd_workspace_size", "fa_fwd_trace_size", "fa_bwd_trace_size", "fa_bwd_row_tile",
     "fa_debug_fwd_trace", "fa_debug_bwd_trace", "fa_debug_bwd_phase", "fa_device_status",
-    "fa_debug_timeout_probe", "fa_bwd_noalloc", "fa_fwd_qk", "fa_bwd_qk",
+    "fa_debug_timeout_probe", "fa_bwd_noalloc", "fa_fwd_qk", "fa_bwd_qk", "fa_debug_fwd_withhold",
+    "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_size", "fa_fwd_splitkv_splits",
 )
 
 
@@ -64,10 +65,14 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "fa_bwd_row_tile": ([i], i),
         "fa_device_status": ([vp], i),
         "fa_debug_timeout_probe": ([i, vp], i),
+        "fa_debug_fwd_withhold": (fwd_args + [i, vp], i),
         "fa_bwd_noalloc": (bwd_args[:10] + bwd_args[11:] + [vp], i),
         # N_q, N_k in place of N
         "fa_fwd_qk": (fwd_args[:8] + [i] + fwd_args[8:] + [vp, vp], i),
         "fa_bwd_qk": (bwd_args[:13] + [i] + bwd_args[13:] + [vp, vp], i),
+        "fa_fwd_splitkv": (fwd_args[:8] + [i] + fwd_args[8:] + [vp, i, vp, vp], i),
+        "fa_fwd_splitkv_workspace_size": ([i, i, i, i, i], sz),
+        "fa_fwd_splitkv_splits": ([i, i, i, i], i),
     }
     for name, (argtypes, restype) in sigs.items():
         fn = getattr(lib, name)
@@ -234,6 +239,16 @@ def fa_device_status(stream=None) -> int:
     return int(load_library().fa_device_status(_stream(stream)))
 
 
+def fa_debug_fwd_withhold(q, k, v, o, lse, timeout_ms: int, causal: bool = False, scale=None, stream=None) -> None:
+    """The forward kernel with a producer that issues no load: its waits run out after
+    ``timeout_ms`` and record FA_ERR_TIMEOUT (see include/fa.h)."""
+    B, H, N, d = _shape(q)
+    st = load_library().fa_debug_fwd_withhold(_dtype_code(q), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H,
+                                              N, d, _scale(scale, d), int(bool(causal)), int(timeout_ms),
+                                              _stream(stream))
+    _check(st, "fa_debug_fwd_withhold")
+
+
 def fa_debug_timeout_probe(timeout_ms: int, stream=None) -> None:
     _check(load_library().fa_debug_timeout_probe(int(timeout_ms), _stream(stream)), "fa_debug_timeout_probe")
 
@@ -265,6 +280,28 @@ def fa_bwd_qk(q, k, v, o, lse, dout, dq, dk, dv, workspace, causal: bool = False
                                   _scale(scale, d), int(bool(causal)),
                                   _ptr(block_mask) if block_mask is not None else None, _stream(stream))
     _check(st, "fa_bwd_qk")
+
+
+def fa_fwd_splitkv_workspace_size(B: int, H: int, Nq: int, d: int, n_splits: int) -> int:
+    return int(load_library().fa_fwd_splitkv_workspace_size(B, H, Nq, d, n_splits))
+
+
+def fa_fwd_splitkv_splits(B: int, H: int, Nq: int, Nk: int) -> int:
+    return int(load_library().fa_fwd_splitkv_splits(B, H, Nq, Nk))
+
+
+def fa_fwd_splitkv(q, k, v, o, lse, n_splits: int, workspace, causal: bool = False, block_mask=None,
+                   scale: float | None = None, stream=None) -> None:
+    """Split-KV forward: ``n_splits`` key ranges computed apart, then merged; the
+    partials stay in ``workspace`` (see include/fa.h for its layout)."""
+    B, H, Nq, d = _shape(q)
+    Nk = _shape(k)[2]
+    _check_tensors(q, k, v, o, lse, workspace, block_mask)
+    st = load_library().fa_fwd_splitkv(_dtype_code(q), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Nq, Nk,
+                                       d, _scale(scale, d), int(bool(causal)),
+                                       _ptr(block_mask) if block_mask is not None else None, int(n_splits),
+                                       _ptr(workspace), _stream(stream))
+    _check(st, "fa_fwd_splitkv")
 
 
 def attention_forward(q, k, v, causal: bool = False, block_mask=None, scale=None, stream=None):

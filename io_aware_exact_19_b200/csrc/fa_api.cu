@@ -9,6 +9,7 @@
 
 #include "fa_internal.h"
 #include "sm100.cuh"
+#include "tma_host.h"
 
 namespace {
 
@@ -75,7 +76,7 @@ fa_status check_mask(int N, int d, const uint8_t* block_mask) {
 
 fa_status fwd_impl(fa_dtype dtype, const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
                    int N, int d, float scale, int causal, const uint8_t* mask, int32_t* trace,
-                   cudaStream_t stream, int Nk = 0) {
+                   cudaStream_t stream, int Nk = 0, uint64_t withhold_timeout_ns = 0) {
   fa_status s = Nk > 0 ? check_qk(dtype, B, H, N, Nk, d) : check_common(dtype, B, H, N, d);
   if (s != FA_OK) return s;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
@@ -96,6 +97,10 @@ fa_status fwd_impl(fa_dtype dtype, const void* q, const void* k, const void* v, 
   a.causal = causal ? 1 : 0;
   a.block_mask = mask;
   a.trace = trace;
+  if (withhold_timeout_ns != 0) {
+    a.withhold = 1;
+    a.timeout_ns = withhold_timeout_ns;
+  }
   a.status = status_word();
   if (!a.status) return FA_ERR_CUDA;
   return fa::launch_fwd(a, stream) == 0 ? FA_OK : FA_ERR_CUDA;
@@ -142,10 +147,12 @@ fa_status bwd_impl(fa_dtype dtype, const void* q, const void* k, const void* v, 
 
 int* fa::device_status_word() { return status_word(); }
 
+bool fa::head_dim_supported(int d) { return d == 32 || d == 64 || d == 96 || d == 128; }
+
 fa_status fa::check_common(fa_dtype dtype, int B, int H, int N, int d) {
   if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_INVALID_ARG;
   if (B < 1 || H < 1 || N < 1 || d < 1) return FA_ERR_INVALID_ARG;
-  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (!fa::head_dim_supported(d)) return FA_ERR_UNSUPPORTED;
   const long long bh = static_cast<long long>(B) * H;
   const long long tiles = (static_cast<long long>(N) + 127) / 128;
   // Grids are 1-D over batch*heads*(2*tiles) CTAs (< 2^31); key-tile indices fit 16 bits.
@@ -180,7 +187,7 @@ fa_status fa_blocksparse_fwd(fa_dtype dtype, const void* q, const void* k, const
 }
 
 size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
-  if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 128)) return 0;
+  if (B < 1 || H < 1 || N < 1 || !fa::head_dim_supported(d)) return 0;
   return fa::bwd_workspace_layout(B, H, N, d).total;
 }
 
@@ -234,7 +241,7 @@ size_t fa_fwd_trace_size(int B, int H, int N) {
 }
 
 size_t fa_bwd_trace_size(int B, int H, int N, int d) {
-  if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 128)) return 0;
+  if (B < 1 || H < 1 || N < 1 || !fa::head_dim_supported(d)) return 0;
   const size_t t = (static_cast<size_t>(N) + 127) / 128;
   const size_t br = static_cast<size_t>(fa::bwd_row_tile(d));
   const size_t tq = (static_cast<size_t>(N) + br - 1) / br;
@@ -287,6 +294,74 @@ fa_status fa_device_status(cudaStream_t stream) {
   if (cudaMemsetAsync(w, 0, sizeof(int), stream) != cudaSuccess) return FA_ERR_CUDA;
   if (cudaStreamSynchronize(stream) != cudaSuccess) return FA_ERR_CUDA;
   return static_cast<fa_status>(h);
+}
+
+size_t fa_fwd_splitkv_workspace_size(int B, int H, int Nq, int d, int n_splits) {
+  if (B < 1 || H < 1 || Nq < 1 || n_splits < 1 || !fa::head_dim_supported(d)) return 0;
+  return fa::splitkv_workspace_layout(B, H, Nq, d, n_splits).total;
+}
+
+int fa_fwd_splitkv_splits(int B, int H, int Nq, int Nk) {
+  if (B < 1 || H < 1 || Nq < 1 || Nk < 1) return 0;
+  const int sms = fa::host::sm_count();
+  if (sms < 1) return 1;
+  const long long tq = (static_cast<long long>(Nq) + 127) / 128;
+  const long long base = static_cast<long long>(B) * H * ((tq + 1) / 2);  // CTAs without splitting
+  const long long tk = (static_cast<long long>(Nk) + 127) / 128;
+  long long ns = base >= sms ? 1 : sms / base;  // one wave of CTAs
+  if (ns > tk) ns = tk;
+  return static_cast<int>(ns < 1 ? 1 : ns);
+}
+
+fa_status fa_fwd_splitkv(fa_dtype dtype, const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                         int H, int Nq, int Nk, int d, float softmax_scale, int causal, const uint8_t* block_mask,
+                         int n_splits, void* workspace, cudaStream_t stream) {
+  if (Nq < 1 || Nk < 1) return FA_ERR_INVALID_ARG;
+  fa_status s = check_qk(dtype, B, H, Nq, Nk, d);
+  if (s != FA_OK) return s;
+  if (block_mask != nullptr) {
+    s = check_mask_qk(Nq, Nk);
+    if (s != FA_OK) return s;
+  }
+  const long long tk = (static_cast<long long>(Nk) + 127) / 128;
+  if (n_splits < 1 || n_splits > tk) return FA_ERR_INVALID_ARG;
+  const long long pairs = ((static_cast<long long>(Nq) + 127) / 128 + 1) / 2;
+  if (static_cast<long long>(B) * H * pairs * n_splits > 0x7FFFFFFFLL) return FA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_INVALID_ARG;
+  if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FA_ERR_INVALID_ARG;
+  const fa::SplitWorkspace ws = fa::splitkv_workspace_layout(B, H, Nq, d, n_splits);
+  uint8_t* base = static_cast<uint8_t*>(workspace);
+  fa::AttnArgs a{};
+  a.dtype = dtype;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.o = o;
+  a.lse = lse;
+  a.B = B;
+  a.H = H;
+  a.N = Nq;
+  a.Nk = Nk;
+  a.d = d;
+  a.scale = softmax_scale;
+  a.causal = causal ? 1 : 0;
+  a.block_mask = block_mask;
+  a.trace = nullptr;
+  a.n_splits = n_splits;
+  a.o_part = reinterpret_cast<float*>(base + ws.o_part);
+  a.lse_part = reinterpret_cast<float*>(base + ws.lse_part);
+  a.status = status_word();
+  if (!a.status) return FA_ERR_CUDA;
+  if (fa::launch_fwd(a, stream) != 0) return FA_ERR_CUDA;
+  return fa::launch_splitkv_merge(a, stream) == 0 ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status fa_debug_fwd_withhold(fa_dtype dtype, const void* q, const void* k, const void* v, void* o, float* lse,
+                                int B, int H, int N, int d, float softmax_scale, int causal, int timeout_ms,
+                                cudaStream_t stream) {
+  if (timeout_ms < 1 || timeout_ms > 5000) return FA_ERR_INVALID_ARG;
+  return fwd_impl(dtype, q, k, v, o, lse, B, H, N, d, softmax_scale, causal, nullptr, nullptr, stream, 0,
+                  static_cast<uint64_t>(timeout_ms) * 1000000ull);
 }
 
 fa_status fa_debug_timeout_probe(int timeout_ms, cudaStream_t stream) {

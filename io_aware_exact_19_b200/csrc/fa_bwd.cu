@@ -45,6 +45,7 @@ int launch_bwd_t(const AttnArgs& a, cudaStream_t stream) {
   const int Nk = a.Nk > 0 ? a.Nk : a.N;
   p.N = a.N;
   p.Nk = Nk;
+  p.d = a.d;
   p.Npad = (a.N + 127) / 128 * 128;
   p.BH = BH;
   p.Tq = (a.N + 127) / 128;
@@ -60,11 +61,11 @@ int launch_bwd_t(const AttnArgs& a, cudaStream_t stream) {
   }
   p.scale_log2 = a.scale * 1.4426950408889634f;
 
-  // prep: D/8 threads per padded row.
+  // prep: blocks of kPrepRows<D> padded rows (a divisor of 128, so of Npad).
   if (a.phases & 1) {
-    const long long threads = static_cast<long long>(BH) * p.Npad * (D / 8);
-    const long long blocks = threads / 256;  // Npad*(D/8) is a multiple of 1024
-    bwd::fa_bwd_prep_kernel<D, BF16><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p);
+    static_assert(128 % bwd::kPrepRows<D> == 0, "prep rows per block must divide the row padding");
+    const long long blocks = static_cast<long long>(BH) * p.Npad / bwd::kPrepRows<D>;
+    bwd::fa_bwd_prep_kernel<D, BF16><<<static_cast<unsigned>(blocks), bwd::kPrepThreads, 0, stream>>>(p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return static_cast<int>(e);
   }
@@ -76,13 +77,13 @@ int launch_bwd_t(const AttnArgs& a, cudaStream_t stream) {
     // 32-row boxes: 64 columns with the 128-byte swizzle, or (dQ at d = 64, where
     // a warpgroup owns 32 columns) 32 columns unswizzled.
     const bool dq64 = D / 2 >= 64;
-    bool ok = host::make_map_3d(&tq, dt, 2, a.q, D, a.N, BH, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B) &&
-              host::make_map_3d(&tdo, dt, 2, a.dout, D, a.N, BH, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B) &&
-              host::make_map_3d(&tk, dt, 2, a.k, D, Nk, BH, 64, bwd::kBlockN, CU_TENSOR_MAP_SWIZZLE_128B) &&
-              host::make_map_3d(&tv, dt, 2, a.v, D, Nk, BH, 64, bwd::kBlockN, CU_TENSOR_MAP_SWIZZLE_128B) &&
-              host::make_map_3d(&tdk, dt, 2, a.dk, D, Nk, BH, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B) &&
-              host::make_map_3d(&tdv, dt, 2, a.dv, D, Nk, BH, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B) &&
-              host::make_map_3d(&tdq, dt, 2, a.dq, D, a.N, BH, dq64 ? 64 : 32, 32,
+    bool ok = host::make_map_3d(&tq, dt, 2, a.q, a.d, a.N, BH, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B) &&
+              host::make_map_3d(&tdo, dt, 2, a.dout, a.d, a.N, BH, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B) &&
+              host::make_map_3d(&tk, dt, 2, a.k, a.d, Nk, BH, 64, bwd::kBlockN, CU_TENSOR_MAP_SWIZZLE_128B) &&
+              host::make_map_3d(&tv, dt, 2, a.v, a.d, Nk, BH, 64, bwd::kBlockN, CU_TENSOR_MAP_SWIZZLE_128B) &&
+              host::make_map_3d(&tdk, dt, 2, a.dk, a.d, Nk, BH, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B) &&
+              host::make_map_3d(&tdv, dt, 2, a.dv, a.d, Nk, BH, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B) &&
+              host::make_map_3d(&tdq, dt, 2, a.dq, a.d, a.N, BH, dq64 ? 64 : 32, 32,
                                 dq64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE);
     if (!ok) return static_cast<int>(cudaErrorInvalidValue);
     auto kern = bwd::fa_bwd_main_kernel<D, BF16>;
@@ -98,8 +99,11 @@ int launch_bwd_t(const AttnArgs& a, cudaStream_t stream) {
 
 }  // namespace
 
+// Head dimensions 32 and 96 run in the 64 and 128 kernels: the tensor maps have
+// the tensors' d columns, so TMA loads fill columns d..D-1 with zeros (which add
+// nothing to any product) and stores clip them.
 int launch_bwd(const AttnArgs& a, cudaStream_t stream) {
-  if (a.d == 64) return a.dtype == 1 ? launch_bwd_t<64, true>(a, stream) : launch_bwd_t<64, false>(a, stream);
+  if (a.d <= 64) return a.dtype == 1 ? launch_bwd_t<64, true>(a, stream) : launch_bwd_t<64, false>(a, stream);
   return a.dtype == 1 ? launch_bwd_t<128, true>(a, stream) : launch_bwd_t<128, false>(a, stream);
 }
 

@@ -162,6 +162,7 @@ struct Params {
   int* status;
   int N;     // query rows
   int Nk;    // key / value rows
+  int d;     // head dimension of the tensors (<= D; columns d..D-1 are zero in the kernel)
   int Npad;  // query rows rounded up to 128
   int BH;
   int Tq;    // ceil(N / 128) query tiles
@@ -174,25 +175,43 @@ struct Params {
 
 // --------------------------------------------------------------------------- prep
 
-// One group of D/8 threads per row: 16-byte loads of O and dO, fp32 dot product.
+// HBM bound. A group of D/8 threads per row, each with one 16-byte piece of O
+// and of dO; every thread covers kPrepRounds rows and issues all its loads
+// before the first product, so each warp keeps 2 x kPrepRounds x 512 bytes in
+// flight. A block covers kPrepRows(D) consecutive padded rows (a divisor of 128).
+constexpr int kPrepThreads = 256;
+constexpr int kPrepRounds = 2;
+template <int D>
+constexpr int kPrepRows = kPrepThreads / (D / 8) * kPrepRounds;
+
 template <int D, bool BF16>
-__global__ void __launch_bounds__(256) fa_bwd_prep_kernel(Params p) {
+__global__ void __launch_bounds__(kPrepThreads) fa_bwd_prep_kernel(Params p) {
   constexpr int kTPR = D / 8;
-  const long long gt = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const long long row = gt / kTPR;  // over BH * Npad (Npad * kTPR is a multiple of 256)
-  const int part = static_cast<int>(gt % kTPR);
-  const long long total = static_cast<long long>(p.BH) * p.Npad;
-  if (row >= total) return;
-  const int bh = static_cast<int>(row / p.Npad);
-  const int r = static_cast<int>(row % p.Npad);
-  float acc = 0.0f;
-  const bool valid = r < p.N;
-  if (valid) {
-    const size_t off = (static_cast<size_t>(bh) * p.N + r) * D + part * 8;
-    const uint4 a = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(p.o) + off);
-    const uint4 b = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(p.dout) + off);
-    const uint32_t aw[4] = {a.x, a.y, a.z, a.w};
-    const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
+  constexpr int kRowsPerRound = kPrepThreads / kTPR;
+  const int part = static_cast<int>(threadIdx.x % kTPR);
+  // The block's rows lie in one head (kPrepRows divides Npad).
+  const long long block_row = static_cast<long long>(blockIdx.x) * kPrepRows<D>;
+  const int bh = static_cast<int>(block_row / p.Npad);
+  const int r_first = static_cast<int>(block_row - static_cast<long long>(bh) * p.Npad) +
+                      static_cast<int>(threadIdx.x / kTPR);
+  uint4 a[kPrepRounds], b[kPrepRounds];
+#pragma unroll
+  for (int k = 0; k < kPrepRounds; ++k) {
+    const int r = r_first + k * kRowsPerRound;
+    a[k] = make_uint4(0, 0, 0, 0);
+    b[k] = make_uint4(0, 0, 0, 0);
+    if (r < p.N && part * 8 < p.d) {
+      const size_t off = (static_cast<size_t>(bh) * p.N + r) * p.d + part * 8;
+      a[k] = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(p.o) + off);
+      b[k] = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(p.dout) + off);
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < kPrepRounds; ++k) {
+    const int r = r_first + k * kRowsPerRound;
+    const uint32_t aw[4] = {a[k].x, a[k].y, a[k].z, a[k].w};
+    const uint32_t bw[4] = {b[k].x, b[k].y, b[k].z, b[k].w};
+    float acc = 0.0f;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       float a0, a1, b0, b1;
@@ -212,18 +231,19 @@ __global__ void __launch_bounds__(256) fa_bwd_prep_kernel(Params p) {
       acc = fmaf(a0, b0, acc);
       acc = fmaf(a1, b1, acc);
     }
-  }
 #pragma unroll
-  for (int m = kTPR / 2; m > 0; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
-  if (part == 0) {
-    const size_t vo = static_cast<size_t>(bh) * p.Npad + r;
-    float l2 = INFINITY;
-    if (valid) {
-      const float l = p.lse[static_cast<size_t>(bh) * p.N + r];
-      if (l != -INFINITY) l2 = l * kLog2e;
+    for (int m = kTPR / 2; m > 0; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
+    if (part == 0) {
+      const bool valid = r < p.N;
+      const size_t vo = static_cast<size_t>(bh) * p.Npad + r;
+      float l2 = INFINITY;
+      if (valid) {
+        const float l = p.lse[static_cast<size_t>(bh) * p.N + r];
+        if (l != -INFINITY) l2 = l * kLog2e;
+      }
+      p.delta[vo] = valid ? acc : 0.0f;
+      p.lse2[vo] = l2;
     }
-    p.delta[vo] = valid ? acc : 0.0f;
-    p.lse2[vo] = l2;
   }
 }
 
@@ -250,7 +270,8 @@ struct Ctx {
 // caller waits for before the CTA exits.
 template <bool BF16, int NCOLS>
 __device__ __forceinline__ void store_rows_tma(uint32_t taddr, float mul, bool have, uint32_t stage,
-                                               const CUtensorMap* map, int col0, int row0, int bh, int N) {
+                                               const CUtensorMap* map, int col0, int row0, int bh, int N,
+                                               int ncols_tensor) {
   const uint32_t lane = threadIdx.x & 31u;
   constexpr int kBoxCols = NCOLS >= 64 ? 64 : NCOLS;
   constexpr uint32_t kRowBytes = kBoxCols * 2;
@@ -278,9 +299,12 @@ __device__ __forceinline__ void store_rows_tma(uint32_t taddr, float mul, bool h
   fence_proxy_async_smem();
   __syncwarp();
   if (lane == 0 && row0 < N) {
+    // Boxes that start past the tensor's last column (a padded head dimension)
+    // are not stored; a box that straddles it is clipped by the store.
 #pragma unroll
     for (int b = 0; b < NCOLS / kBoxCols; ++b)
-      tma_store_3d(map, stage + static_cast<uint32_t>(b) * kBoxBytes, col0 + b * kBoxCols, row0, bh);
+      if (col0 + b * kBoxCols < ncols_tensor)
+        tma_store_3d(map, stage + static_cast<uint32_t>(b) * kBoxBytes, col0 + b * kBoxCols, row0, bh);
     bulk_commit_group();
   }
 }
@@ -484,7 +508,7 @@ __device__ __forceinline__ void key_cta(const Ctx& c, const Params& p, const CUt
     if (ok) {
       const uint32_t stage = smem_u32(sQ) + static_cast<uint32_t>(c.warp - 4) * (32 * D * 2);
       store_rows_tma<BF16, D>(tl + 256 + h * D, h == 0 ? 1.0f : p.scale, have, stage, h == 0 ? tdv : tdk, 0,
-                              j * kBlockN + wq * 32, c.bh, p.Nk);
+                              j * kBlockN + wq * 32, c.bh, p.Nk, p.d);
     }
     if (c.lane == 0) bulk_wait_group_read<0>();  // shared memory read; the writes complete on their own
   }
@@ -643,14 +667,16 @@ __device__ __forceinline__ void query_cta(const Ctx& c, const Params& p, const C
           b[4 * v + 2] = __float_as_uint(y.z); b[4 * v + 3] = __float_as_uint(y.w);
         }
       } else {
-        // Straight from global memory; all loads first, then the TMEM stores.
-        const size_t roff = (static_cast<size_t>(c.bh) * p.N + (row_valid ? qrow : 0)) * D;
+        // Straight from global memory (row stride d; columns past d are zero); all
+        // loads first, then the TMEM stores.
+        const size_t roff = (static_cast<size_t>(c.bh) * p.N + (row_valid ? qrow : 0)) * p.d;
         const uint4* gq = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(p.q) + roff);
         const uint4* gdo = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(p.dout) + roff);
 #pragma unroll
         for (int v = 0; v < kWords / 4; ++v) {
-          const uint4 x = row_valid ? gq[h * kWords / 4 + v] : make_uint4(0, 0, 0, 0);
-          const uint4 y = row_valid ? gdo[h * kWords / 4 + v] : make_uint4(0, 0, 0, 0);
+          const bool in = row_valid && (h * (D / 2) + 8 * v) < p.d;
+          const uint4 x = in ? gq[h * kWords / 4 + v] : make_uint4(0, 0, 0, 0);
+          const uint4 y = in ? gdo[h * kWords / 4 + v] : make_uint4(0, 0, 0, 0);
           a[4 * v] = x.x; a[4 * v + 1] = x.y; a[4 * v + 2] = x.z; a[4 * v + 3] = x.w;
           b[4 * v] = y.x; b[4 * v + 1] = y.y; b[4 * v + 2] = y.z; b[4 * v + 3] = y.w;
         }
@@ -715,7 +741,7 @@ __device__ __forceinline__ void query_cta(const Ctx& c, const Params& p, const C
     if (ok) {
       const uint32_t stage = smem_u32(sK) + static_cast<uint32_t>(c.warp - 4) * (32 * (D / 2) * 2);
       store_rows_tma<BF16, D / 2>(tl + C::kColDQ + h * (D / 2), p.scale, have, stage, tdq, h * (D / 2),
-                                  i * kBlockQ + wq * 32, c.bh, p.N);
+                                  i * kBlockQ + wq * 32, c.bh, p.N, p.d);
     }
     if (c.lane == 0) bulk_wait_group_read<0>();  // shared memory read; the writes complete on their own
   }

@@ -15,10 +15,10 @@ int launch_fwd_t(const AttnArgs& a, cudaStream_t stream) {
   const int Nk = a.Nk > 0 ? a.Nk : a.N;
   CUtensorMap tq, tk, tv, to;
   // O is written by 64-column x 32-row boxes, one per warp and 64 columns.
-  bool ok = host::make_map_3d(&tq, dt, 2, a.q, D, a.N, BH, 64, fwd::kBlockM, CU_TENSOR_MAP_SWIZZLE_128B) &&
-            host::make_map_3d(&tk, dt, 2, a.k, D, Nk, BH, 64, fwd::kBlockN, CU_TENSOR_MAP_SWIZZLE_128B) &&
-            host::make_map_3d(&tv, dt, 2, a.v, D, Nk, BH, 64, fwd::kBlockN, CU_TENSOR_MAP_SWIZZLE_128B) &&
-            host::make_map_3d(&to, dt, 2, a.o, D, a.N, BH, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B);
+  bool ok = host::make_map_3d(&tq, dt, 2, a.q, a.d, a.N, BH, 64, fwd::kBlockM, CU_TENSOR_MAP_SWIZZLE_128B) &&
+            host::make_map_3d(&tk, dt, 2, a.k, a.d, Nk, BH, 64, fwd::kBlockN, CU_TENSOR_MAP_SWIZZLE_128B) &&
+            host::make_map_3d(&tv, dt, 2, a.v, a.d, Nk, BH, 64, fwd::kBlockN, CU_TENSOR_MAP_SWIZZLE_128B) &&
+            host::make_map_3d(&to, dt, 2, a.o, a.d, a.N, BH, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B);
   if (!ok) return static_cast<int>(cudaErrorInvalidValue);
   fwd::Params p;
   p.o = const_cast<void*>(a.o);
@@ -28,6 +28,12 @@ int launch_fwd_t(const AttnArgs& a, cudaStream_t stream) {
   p.status = a.status;
   p.N = a.N;
   p.Nk = Nk;
+  p.d = a.d;
+  p.timeout_ns = a.timeout_ns;
+  p.withhold = a.withhold;
+  p.n_splits = a.n_splits > 1 || a.o_part != nullptr ? a.n_splits : 1;
+  p.o_part = a.o_part;
+  p.lse_part = a.lse_part;
   p.BH = BH;
   const int Tq = (a.N + fwd::kBlockM - 1) / fwd::kBlockM;
   p.n_pairs = (Tq + 1) / 2;
@@ -40,18 +46,21 @@ int launch_fwd_t(const AttnArgs& a, cudaStream_t stream) {
     p.head_group = static_cast<int>(g < 1 ? 1 : (g > BH ? BH : g));
   }
   p.scale_log2 = a.scale * 1.4426950408889634f;
-  auto kern = fwd::fa_fwd_kernel<D, BF16>;
+  auto kern = p.o_part != nullptr ? fwd::fa_fwd_kernel<D, BF16, true> : fwd::fa_fwd_kernel<D, BF16, false>;
   cudaError_t e = host::ensure_dynamic_smem(reinterpret_cast<const void*>(kern), L::kAlloc);
   if (e != cudaSuccess) return static_cast<int>(e);
-  dim3 grid(BH * p.n_pairs);
+  dim3 grid(static_cast<unsigned>(static_cast<long long>(BH) * p.n_pairs * p.n_splits));
   kern<<<grid, fwd::kThreads, L::kAlloc, stream>>>(tq, tk, tv, to, p);
   return static_cast<int>(cudaGetLastError());
 }
 
 }  // namespace
 
+// Head dimensions 32 and 96 run in the 64 and 128 kernels: the tensor maps have
+// the tensors' d columns, so TMA loads fill columns d..D-1 with zeros (which add
+// nothing to S or to P V) and the O stores skip or clip them.
 int launch_fwd(const AttnArgs& a, cudaStream_t stream) {
-  if (a.d == 64) return a.dtype == 1 ? launch_fwd_t<64, true>(a, stream) : launch_fwd_t<64, false>(a, stream);
+  if (a.d <= 64) return a.dtype == 1 ? launch_fwd_t<64, true>(a, stream) : launch_fwd_t<64, false>(a, stream);
   return a.dtype == 1 ? launch_fwd_t<128, true>(a, stream) : launch_fwd_t<128, false>(a, stream);
 }
 

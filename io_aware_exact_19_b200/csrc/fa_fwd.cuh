@@ -53,8 +53,18 @@ struct Params {
   const uint8_t* block_mask;  // null unless block-sparse: [ceil(N/128)][Tc]
   int32_t* trace;             // null unless tracing
   int* status;
+  uint64_t timeout_ns;        // limit of every wait
   int N;        // query rows
   int Nk;       // key / value rows
+  int d;        // head dimension of the tensors (<= D; columns d..D-1 are zero in the kernel)
+  int withhold;  // debug: the producer issues no load, so the first wait runs out
+  // Split-KV: the key tiles are cut into n_splits consecutive ranges, one CTA per
+  // (query-tile pair, range); each writes its partial O (fp32, normalised by its
+  // own exp-sum) to o_part [n_splits][BH][N][d] and its lse to lse_part
+  // [n_splits][BH][N] instead of o / lse. n_splits = 1 and o_part = null otherwise.
+  int n_splits;
+  float* o_part;
+  float* lse_part;
   int BH;
   int n_pairs;  // ceil(T_q / 2)
   int Tc;       // ceil(Nk / 128)
@@ -71,25 +81,28 @@ struct Smem {
   static constexpr int kKOff = kQOff + 2 * kTileBytes;
   static constexpr int kVOff = kKOff + kStages * kTileBytes;
   static constexpr int kBarOff = kVOff + kStages * kTileBytes;
-  // barriers: q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_full[2], o_full[2]
-  static constexpr int kNumBars = 1 + 4 * kStages + 6;
+  // barriers: q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_full[2], o_full[2], drain
+  static constexpr int kNumBars = 1 + 4 * kStages + 7;
   static constexpr int kListOff = kBarOff + 8 * kNumBars + 16;  // + tmem slot, abort flag, list length
   static constexpr int kBytes = kListOff + 4 * kMaxSparseTiles;
   static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1024
 };
 
 // Key-tile iteration shared by every role: entry n of the CTA's list is key
-// tile j(n) with flags f(n) (bit q set: query tile 2p+q uses it).
+// tile j(n) with flags f(n) (bit q set: query tile 2p+q uses it). The tiles are
+// those of the CTA's key range [lo, hi) (all of them unless split-KV).
 struct TileList {
   int len;
   int mode;        // 0 dense, 1 causal, 2 list in shared memory
+  int lo;          // first key tile of the range
   int lim0, lim1;  // last key tile query tile 0 / 1 uses (-1: none, e.g. no tile 1)
   const uint32_t* list;
 
   __device__ __forceinline__ uint32_t entry(int n) const {
     if (mode == 2) return list[n];
-    const uint32_t f = (n <= lim0 ? 1u : 0u) | (n <= lim1 ? 2u : 0u);
-    return static_cast<uint32_t>(n) | (f << 16);
+    const int j = lo + n;
+    const uint32_t f = (j <= lim0 ? 1u : 0u) | (j <= lim1 ? 2u : 0u);
+    return static_cast<uint32_t>(j) | (f << 16);
   }
 };
 
@@ -103,7 +116,9 @@ __device__ __forceinline__ int causal_last_key_tile(int qt, int N, int Nk) {
   return last_key < 0 ? -1 : last_key / kBlockN;
 }
 
-template <int D, bool BF16>
+// kSplit: split-KV launch (key ranges, fp32 partials); a separate instance so the
+// plain forward compiles without its bookkeeping.
+template <int D, bool BF16, bool kSplit>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                   const __grid_constant__ CUtensorMap tmap_v, const __grid_constant__ CUtensorMap tmap_o,
@@ -126,18 +141,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto bar_s_full = [&](int q) { return smem_u32(&bars[1 + 4 * S + q]); };
   auto bar_p_full = [&](int q) { return smem_u32(&bars[1 + 4 * S + 2 + q]); };
   auto bar_o_full = [&](int q) { return smem_u32(&bars[1 + 4 * S + 4 + q]); };
+  const uint32_t bar_drain = smem_u32(&bars[1 + 4 * S + 6]);
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
   // Heads in groups of p.head_group (their K/V stay in L2); inside a group the
   // heaviest query-tile pairs (the last ones, under a causal mask) start first.
+  const int n_splits = kSplit ? p.n_splits : 1;
   int bh, rank;
-  grouped_order(static_cast<int>(blockIdx.x), p.BH, p.n_pairs, p.head_group, bh, rank);
-  const int pair = p.n_pairs - 1 - rank;
+  grouped_order(static_cast<int>(blockIdx.x), p.BH, p.n_pairs * n_splits, p.head_group, bh, rank);
+  const int pair = p.n_pairs - 1 - rank / n_splits;
+  const int split = kSplit ? rank % n_splits : 0;
+  const int key_lo = kSplit ? static_cast<int>(static_cast<long long>(split) * p.Tc / n_splits) : 0;
+  const int key_hi = kSplit ? static_cast<int>(static_cast<long long>(split + 1) * p.Tc / n_splits) : p.Tc;
   const int q0 = 2 * pair;
   const int Tq = (p.N + kBlockM - 1) / kBlockM;
   const int q1_active = (q0 + 1) < Tq;
-  const int cta = bh * p.n_pairs + pair;
+  const int cta = bh * p.n_pairs + pair;  // trace record (never split)
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
@@ -153,6 +173,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar_p_full(q), 128);
       mbar_init(bar_o_full(q), 1);
     }
+    mbar_init(bar_drain, 1);
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -173,10 +194,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint8_t* row0 = p.block_mask + static_cast<size_t>(q0) * p.Tc;
       const uint8_t* row1 = row0 + p.Tc;
       int count = 0;
-      for (int base = 0; base < p.Tc; base += 32) {
+      for (int base = key_lo; base < key_hi; base += 32) {
         const int j = base + lane;
         uint32_t f = 0;
-        if (j < p.Tc) {
+        if (j < key_hi) {
           if (row0[j] && j <= lim0) f |= 1u;
           if (q1_active && row1[j] && j <= lim1) f |= 2u;
         }
@@ -195,22 +216,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
 
   const uint32_t tmem = *tmem_slot;
-  WaitCtx ctx{abort_flag, p.status};
+  WaitCtx ctx{abort_flag, p.status, p.timeout_ns};
 
   auto make_tiles = [&]() {
     TileList tl;
     tl.lim0 = reach(0);
     tl.lim1 = reach(1);
     tl.list = list;
+    tl.lo = key_lo;
     if (p.block_mask != nullptr) {
       tl.mode = 2;
       tl.len = *list_len;
     } else if (p.causal) {
       tl.mode = 1;
-      tl.len = min(p.Tc, max(tl.lim0, tl.lim1) + 1);
+      tl.len = max(0, min(key_hi, max(tl.lim0, tl.lim1) + 1) - key_lo);
     } else {
       tl.mode = 0;
-      tl.len = p.Tc;
+      tl.len = key_hi - key_lo;
     }
     return tl;
   };
@@ -230,10 +252,11 @@ __global__ void __launch_bounds__(kThreads, 1)
    const TileList tl = make_tiles();
    if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0 && tl.len > 0) {
+    if (lane == 0 && tl.len > 0 && !p.withhold) {
       prefetch_tmap(&tmap_q);
       prefetch_tmap(&tmap_k);
       prefetch_tmap(&tmap_v);
+      int k_issued = 0, v_issued = 0;  // K and V loads issued (for the abort drain)
       const int nq = 1 + q1_active;
       mbar_arrive_expect_tx(bar_q_full, nq * L::kTileBytes);
       for (int q = 0; q < nq; ++q)
@@ -252,11 +275,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < D / 64; ++c)
           tma_load_3d(smem_u32(sK + s * L::kTileBytes + c * kChunkBytes), &tmap_k, bar_k_full(s), c * 64,
                       j * kBlockN, bh);
+        ++k_issued;
         if (!mbar_wait(bar_v_empty(s), ph, ctx)) break;
         mbar_arrive_expect_tx(bar_v_full(s), L::kTileBytes);
         for (int c = 0; c < D / 64; ++c)
           tma_load_3d(smem_u32(sV + s * L::kTileBytes + c * kChunkBytes), &tmap_v, bar_v_full(s), c * 64,
                       j * kBlockN, bh);
+        ++v_issued;
+      }
+      if (*abort_flag) {
+        // Aborting: wait (bounded, whatever the flag says) for every load this
+        // thread issued, so no copy still writes shared memory when the CTA exits.
+        // The last load into stage s completes that stage's barrier phase.
+        for (int s = 0; s < S; ++s) {
+          if (k_issued > s) {
+            const int last = k_issued - 1 - ((k_issued - 1 - s) % S);
+            mbar_wait_bounded(bar_k_full(s), (last / S) & 1, p.timeout_ns);
+          }
+          if (v_issued > s) {
+            const int last = v_issued - 1 - ((v_issued - 1 - s) % S);
+            mbar_wait_bounded(bar_v_full(s), (last / S) & 1, p.timeout_ns);
+          }
+        }
+        mbar_wait_bounded(bar_q_full, 0, p.timeout_ns);
       }
     }
   } else if (warp == 1) {
@@ -300,6 +341,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       // Prologue: S of the first key tile for each query tile that uses it.
       if (ok) ok = mbar_wait(bar_k_full(0), 0, ctx);
+      bool issued = ok;  // an MMA has been issued (from here on)
       if (ok) {
         tc_fence_after();
         const uint32_t f0 = tl.entry(0) >> 16;
@@ -332,6 +374,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok) {
         for (int q = 0; q < 2; ++q)
           if (started[q]) umma_commit(bar_o_full(q));
+      } else if (issued) {
+        // Aborting: let every MMA this thread issued complete before TMEM and the
+        // shared-memory operands are released.
+        umma_commit(bar_drain);
+        mbar_wait_bounded(bar_drain, 0, p.timeout_ns);
       }
     }
   }
@@ -355,7 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int count = 0;
     bool ok = true;
 
-    if (tile_active) {
+    if (tile_active && !p.withhold) {
       for (int n = 0; n < tl.len; ++n) {
         const uint32_t e = tl.entry(n);
         if (!((e >> 16) & (1u << q))) continue;
@@ -458,7 +505,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       const size_t row_base = static_cast<size_t>(bh) * p.N;
       const bool row_valid = row < p.N;
       const float inv_l = (l_sum > 0.0f) ? 1.0f / l_sum : 0.0f;
-      if (ok) {
+      if (kSplit && ok) {
+        // Split-KV partial: fp32 O / l of this key range (0 if it has no key for
+        // the row) and its lse (-inf then), stored straight from the row's thread.
+        const size_t prow = (static_cast<size_t>(split) * p.BH + bh) * p.N + row;
+#pragma unroll
+        for (int c = 0; c < D; c += 32) {
+          uint32_t o[32];
+          if (have_o) {
+            tmem_ld32(t_o + c, o);
+            tmem_ld_wait();
+          }
+          if (row_valid && c < p.d) {
+            float4* dst = reinterpret_cast<float4*>(p.o_part + prow * p.d + c);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              float4 v;
+              v.x = have_o ? __uint_as_float(o[4 * k]) * inv_l : 0.0f;
+              v.y = have_o ? __uint_as_float(o[4 * k + 1]) * inv_l : 0.0f;
+              v.z = have_o ? __uint_as_float(o[4 * k + 2]) * inv_l : 0.0f;
+              v.w = have_o ? __uint_as_float(o[4 * k + 3]) * inv_l : 0.0f;
+              dst[k] = v;
+            }
+          }
+        }
+        if (row_valid)
+          p.lse_part[prow] = (l_sum > 0.0f) ? (m_ref + lg2(l_sum)) * 0.6931471805599453f : -INFINITY;
+      } else if (ok) {
         constexpr uint32_t kBoxBytes = 32 * 128;  // 32 rows x 64 columns x 2 bytes
         const uint32_t stage = smem_u32(sK) + static_cast<uint32_t>(warp - 4) * (D / 64) * kBoxBytes;
 #pragma unroll
@@ -487,9 +560,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         const int row0 = qt * kBlockM + wq * 32;
         if (lane == 0 && row0 < p.N) {
+          // Boxes past the tensor's last column (a padded head dimension) are not
+          // stored; a box that straddles it is clipped by the store.
 #pragma unroll
           for (int b = 0; b < D / 64; ++b)
-            tma_store_3d(&tmap_o, stage + b * kBoxBytes, b * 64, row0, bh);
+            if (b * 64 < p.d) tma_store_3d(&tmap_o, stage + b * kBoxBytes, b * 64, row0, bh);
           bulk_commit_group();
         }
         if (row_valid) {

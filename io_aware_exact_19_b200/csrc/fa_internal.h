@@ -29,10 +29,26 @@ struct AttnArgs {
   int32_t* trace;
   int* status;
   int phases = 7;  // backward launches to run: bit 0 prep, bit 1 main
+  uint64_t timeout_ns = 2000000000ull;  // limit of every device-side wait
+  int withhold = 0;  // debug (forward): the producer issues no load, so the first wait runs out
+  // split-KV forward: partial results per key range (see launch_splitkv_merge)
+  int n_splits = 1;
+  float* o_part = nullptr;    // fp32 [n_splits][B*H][N][d]
+  float* lse_part = nullptr;  // fp32 [n_splits][B*H][N]
 };
 
 // Return 0 on success, a cudaError_t value otherwise.
 int launch_fwd(const AttnArgs& a, cudaStream_t stream);
+// Merge of the split-KV partials (a.o_part, a.lse_part, a.n_splits) into a.o, a.lse.
+int launch_splitkv_merge(const AttnArgs& a, cudaStream_t stream);
+
+// Workspace of the split-KV forward: partial O then partial lse, in bytes.
+struct SplitWorkspace {
+  size_t o_part;
+  size_t lse_part;
+  size_t total;
+};
+SplitWorkspace splitkv_workspace_layout(int B, int H, int Nq, int d, int n_splits);
 int launch_bwd(const AttnArgs& a, cudaStream_t stream);
 
 // Workspace layout of the backward, in bytes from the workspace base.
@@ -46,6 +62,10 @@ int bwd_row_tile(int d);
 
 // Device address of the per-device status word (nullptr on failure).
 int* device_status_word();
+
+// Head dimensions the kernels take: 64 and 128 natively, 32 and 96 inside the
+// 64 and 128 kernels with the missing columns zero-filled by TMA.
+bool head_dim_supported(int d);
 
 // Limits every entry point applies to the element type and sizes of a square
 // (N queries, N keys) problem: FA_OK, FA_ERR_INVALID_ARG or FA_ERR_UNSUPPORTED.

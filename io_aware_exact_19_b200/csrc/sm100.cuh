@@ -135,6 +135,17 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const W
   return false;
 }
 
+// A wait that ignores the abort flag and gives up after `timeout_ns`: used on the
+// abort path to let copies and MMAs already issued complete before the CTA exits.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, uint64_t timeout_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 >= timeout_ns) return false;
+  }
+  return true;
+}
+
 // The same wait taken by every lane of a warp; the result is the same in all
 // lanes, so warp-collective tcgen05 instructions that follow stay converged.
 __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, const WaitCtx& ctx) {
@@ -370,7 +381,7 @@ __device__ __forceinline__ void reg_dealloc() {
 // then group 1, and so on. Blocks are dispatched roughly in index order, so the
 // CTAs in flight touch only about G heads' tensors, which stay in L2, while the
 // heaviest items of each group still start first.
-__device__ __forceinline__ void grouped_order(int L, int BH, int R, int G, int& head, int& rank) {
+__host__ __device__ __forceinline__ void grouped_order(int L, int BH, int R, int G, int& head, int& rank) {
   const int nfull = BH / G;
   const long long span = static_cast<long long>(G) * R;
   if (static_cast<long long>(L) < nfull * span) {

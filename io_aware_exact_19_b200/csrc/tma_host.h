@@ -49,6 +49,21 @@ inline bool make_map_3d(CUtensorMap* map, CUtensorMapDataType dtype, int elem_by
   return r == CUDA_SUCCESS;
 }
 
+// Number of SMs of the current device (cached per device; 0 on failure).
+inline int sm_count() {
+  static std::mutex mu;
+  static int counts[128] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return 0;
+  std::lock_guard<std::mutex> lock(mu);
+  if (counts[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    counts[dev] = n;
+  }
+  return counts[dev];
+}
+
 // Raise a kernel's dynamic shared-memory limit once per (kernel, device).
 inline cudaError_t ensure_dynamic_smem(const void* kernel, int bytes) {
   static std::mutex mu;

@@ -49,7 +49,8 @@ def test_workspace_is_linear_in_n(lib):
     for a, b in zip(diffs, diffs[1:]):
         assert b == 2 * a
     assert lib.fa_bwd_workspace_size(1, 16, 65536, 64) == 1 * 16 * 65536 * 8
-    assert lib.fa_bwd_workspace_size(1, 1, 100, 96) == 0
+    assert lib.fa_bwd_workspace_size(1, 1, 100, 80) == 0
+    assert lib.fa_bwd_workspace_size(1, 1, 100, 96) == lib.fa_bwd_workspace_size(1, 1, 100, 64)
 
 
 def _fake(addr=4096):
@@ -58,8 +59,9 @@ def _fake(addr=4096):
 
 def test_host_argument_errors_return_before_launch(lib):
     p = _fake()
-    # unsupported head dimension
-    assert lib.fa_fwd(1, p, p, p, p, p, 1, 1, 128, 96, 0.1, 0, None) == fa.FA_ERR_UNSUPPORTED
+    # unsupported head dimension (32, 64, 96 and 128 are supported)
+    for d in (16, 48, 80, 160, 512):
+        assert lib.fa_fwd(1, p, p, p, p, p, 1, 1, 128, d, 0.1, 0, None) == fa.FA_ERR_UNSUPPORTED
     # non-positive sizes, bad dtype
     assert lib.fa_fwd(1, p, p, p, p, p, 0, 1, 128, 64, 0.1, 0, None) == fa.FA_ERR_INVALID_ARG
     assert lib.fa_fwd(1, p, p, p, p, p, 1, 1, 0, 64, 0.1, 0, None) == fa.FA_ERR_INVALID_ARG
@@ -74,10 +76,18 @@ def test_host_argument_errors_return_before_launch(lib):
     assert lib.fa_bwd(1, p, p, p, p, p, p, p, p, p, _fake(4096 + 16), 1, 1, 128, 64, 0.1, 0, None) \
         == fa.FA_ERR_INVALID_ARG
     assert lib.fa_debug_timeout_probe(0, None) == fa.FA_ERR_INVALID_ARG
+    assert lib.fa_debug_fwd_withhold(1, p, p, p, p, p, 1, 1, 128, 64, 0.1, 0, 0, None) == fa.FA_ERR_INVALID_ARG
+    # split-KV: range count within 1..ceil(Nk/128), aligned workspace, sizes
+    assert lib.fa_fwd_splitkv(1, p, p, p, p, p, 1, 1, 1, 1000, 64, 0.1, 1, None, 0, p, None) == fa.FA_ERR_INVALID_ARG
+    assert lib.fa_fwd_splitkv(1, p, p, p, p, p, 1, 1, 1, 1000, 64, 0.1, 1, None, 9, p, None) == fa.FA_ERR_INVALID_ARG
+    assert lib.fa_fwd_splitkv(1, p, p, p, p, p, 1, 1, 1, 1000, 64, 0.1, 1, None, 4, _fake(4096 + 16), None) \
+        == fa.FA_ERR_INVALID_ARG
+    assert lib.fa_fwd_splitkv(1, p, p, p, p, p, 1, 1, 1, 1000, 80, 0.1, 1, None, 4, p, None) == fa.FA_ERR_UNSUPPORTED
+    assert lib.fa_fwd_splitkv(1, p, p, p, p, p, 1, 1, 1, 1000, 64, 0.1, 1, p, 4, p, None) == fa.FA_ERR_UNSUPPORTED
     # N_q != N_k entry points: sizes, head dimension, block-mask shape rules
     assert lib.fa_fwd_qk(1, p, p, p, p, p, 1, 1, 0, 128, 64, 0.1, 1, None, None) == fa.FA_ERR_INVALID_ARG
     assert lib.fa_fwd_qk(1, p, p, p, p, p, 1, 1, 128, 0, 64, 0.1, 1, None, None) == fa.FA_ERR_INVALID_ARG
-    assert lib.fa_fwd_qk(1, p, p, p, p, p, 1, 1, 128, 256, 96, 0.1, 1, None, None) == fa.FA_ERR_UNSUPPORTED
+    assert lib.fa_fwd_qk(1, p, p, p, p, p, 1, 1, 128, 256, 80, 0.1, 1, None, None) == fa.FA_ERR_UNSUPPORTED
     assert lib.fa_fwd_qk(1, p, p, p, p, p, 1, 1, 128, 200, 64, 0.1, 0, p, None) == fa.FA_ERR_UNSUPPORTED
     assert lib.fa_fwd_qk(1, None, p, p, p, p, 1, 1, 128, 256, 64, 0.1, 0, None, None) == fa.FA_ERR_INVALID_ARG
     assert lib.fa_bwd_qk(1, p, p, p, p, p, p, p, p, p, _fake(4096 + 16), 1, 1, 128, 256, 64, 0.1, 0, None, None) \
@@ -90,3 +100,13 @@ def test_trace_sizes(lib):
     assert lib.fa_fwd_trace_size(2, 3, 1000) == 2 * 3 * 4 * (8 + 1)
     assert lib.fa_bwd_row_tile(64) == 128 and lib.fa_bwd_row_tile(128) == 128
     assert lib.fa_bwd_trace_size(2, 3, 1000, 128) == 2 * 3 * 8 * ((8 + 1) + (8 + 1))
+
+
+def test_splitkv_workspace_layout(lib):
+    # partial O fp32 [n][B*H][Nq][d], then partial lse fp32 [n][B*H][Nq] at a 256-byte boundary
+    n, B, H, Nq, d = 5, 2, 3, 7, 64
+    o_bytes = n * B * H * Nq * d * 4
+    lse_off = -(-o_bytes // 256) * 256
+    assert lib.fa_fwd_splitkv_workspace_size(B, H, Nq, d, n) == lse_off + -(-(n * B * H * Nq * 4) // 256) * 256
+    assert lib.fa_fwd_splitkv_workspace_size(B, H, Nq, 80, n) == 0
+    assert lib.fa_fwd_splitkv_workspace_size(B, H, Nq, d, 0) == 0

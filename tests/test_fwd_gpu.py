@@ -45,6 +45,9 @@ def test_tiny_fp16_exact_check():
     (1, 1, 1, 64, "bf16", False), (1, 1, 1, 128, "fp16", True),
     (1, 2, 129, 64, "bf16", True), (2, 1, 256, 128, "bf16", False),
     (1, 1, 384, 64, "fp16", True), (1, 3, 640, 128, "bf16", True),
+    # head dimensions 32 and 96 (inside the 64 and 128 kernels, zero-filled columns)
+    (2, 3, 1000, 32, "bf16", False), (1, 2, 777, 32, "fp16", True), (1, 1, 1, 32, "bf16", True),
+    (2, 2, 1000, 96, "bf16", True), (1, 2, 129, 96, "fp16", False), (1, 1, 1, 96, "bf16", False),
 ])
 def test_ragged_and_small(B, H, N, d, fmt, causal):
     _check_full(Case(B, H, N, d, fmt, seed=N + d), causal)
@@ -82,7 +85,7 @@ def test_block_sparse_workload_sampled_rows():
 
 
 @pytest.mark.parametrize("causal", [False, True])
-@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("d", [32, 64, 96, 128])
 def test_block_sparse_full(causal, d):
     mask = S.block_mask_recipe(8, seed=4)
     _check_full(Case(2, 2, 1024, d, "bf16", seed=9), causal, mask=mask)
@@ -142,10 +145,13 @@ def _expected_fwd_trace(N, causal, mask, BH):
     return exp
 
 
-@pytest.mark.parametrize("N,causal,use_mask", [(1000, False, False), (1000, True, False), (1024, False, True),
-                                               (1024, True, True), (128, True, False), (1408, True, True)])
-def test_tile_trace_matches_oracle_enumeration(N, causal, use_mask):
-    B, H, d = 1, 2, 64
+@pytest.mark.parametrize("N,causal,use_mask,B,H", [
+    (1000, False, False, 1, 2), (1000, True, False, 1, 2), (1024, False, True, 1, 2), (1024, True, True, 1, 2),
+    (128, True, False, 1, 2), (1408, True, True, 1, 2),
+    # more work items than SMs: the persistent CTAs follow a host-computed schedule
+    (1000, True, False, 3, 40), (1024, False, True, 2, 50)])
+def test_tile_trace_matches_oracle_enumeration(N, causal, use_mask, B, H):
+    d = 64
     c = Case(B, H, N, d, "bf16", seed=1)
     mask = S.block_mask_recipe(N // 128, seed=6) if use_mask else None
     mdev = torch.from_numpy(mask).cuda() if use_mask else None
@@ -168,3 +174,19 @@ def test_device_timeout_is_reported_and_cleared():
     fa.fa_debug_timeout_probe(20)
     assert fa.fa_device_status() == fa.FA_ERR_TIMEOUT
     assert fa.fa_device_status() == fa.FA_OK
+
+
+def test_forward_kernel_abort_path_reports_timeout_and_context_survives():
+    # The production forward kernel with a producer that issues no load: the MMA
+    # issuer's wait for Q runs out (20 ms), every role leaves its loop and the CTAs
+    # exit with nothing in flight. The status word reports the time-out and the
+    # next, normal launch is still correct.
+    c = Case(2, 3, 1000, 128, "bf16", seed=17)
+    assert fa.fa_device_status() == fa.FA_OK
+    o = torch.zeros_like(c.dev["q"])
+    lse = torch.zeros((2, 3, 1000), dtype=torch.float32, device="cuda")
+    fa.fa_debug_fwd_withhold(c.dev["q"], c.dev["k"], c.dev["v"], o, lse, 20, causal=True)
+    assert fa.fa_device_status() == fa.FA_ERR_TIMEOUT
+    assert fa.fa_device_status() == fa.FA_OK
+    assert torch.count_nonzero(o) == 0 and torch.count_nonzero(lse) == 0
+    _check_full(c, True)

@@ -4,7 +4,7 @@ j <= i + N_k - N_q, so a query block of N_q rows is the last N_q positions of
 the key sequence; rows with no key get O = 0, lse = -inf and no gradient.
 Tolerances as for the square case: O max-abs <= 1e-2, lse max-abs <= 1e-3,
 dQ/dK/dV relative Frobenius <= 2e-2 over each tensor and each 128-row block, and
-every element within 0.1 x the gradient's RMS."""
+every element within 10% of (the gradient's RMS + its row's RMS)."""
 import numpy as np
 import pytest
 import torch
@@ -53,6 +53,8 @@ def _run_qk(B, H, Nq, Nk, d, fmt, causal, mask=None):
     (1, 2, 300, 129, 128, "bf16", True),
     (1, 2, 129, 300, 64, "bf16", False),
     (1, 1, 640, 1, 64, "bf16", True),        # one key: only the last query row sees it
+    (1, 2, 300, 777, 96, "bf16", True),
+    (2, 1, 500, 200, 32, "fp16", True),
 ])
 def test_unequal_lengths(B, H, Nq, Nk, d, fmt, causal):
     _run_qk(B, H, Nq, Nk, d, fmt, causal)
