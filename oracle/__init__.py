@@ -21,6 +21,8 @@ Dao et al., NeurIPS 2022):
               with the row maximum subtracted), "梯度计算优化" (softmax gradient).
 
 Readings where the pages are silent or garbled are listed per function.
+``oracle.dropout`` adds attention with dropout on P (keep decisions from a
+Philox4x32-10 counter-based generator, regenerated in the backward).
 """
 from .attention import (  # noqa: F401
     allowed_mask,
@@ -36,3 +38,4 @@ from .attention import (  # noqa: F401
     backward_tile_lists,
     sampled_forward_backward,
 )
+from . import dropout  # noqa: F401

@@ -369,3 +369,99 @@ def check_rows_unequal_lengths(forward, forward_rows, backward_rows):
             an = float(np.sum(grad * R))
             assert abs(fd - an) <= 1e-7 * max(1.0, abs(an)), \
                 f"backward_rows finite differences d{which} nq={nq} nk={nk} causal={causal}: {fd} vs {an}"
+
+
+# ----------------------------------------------------------------------------- dropout
+
+def check_philox_against_numpy(philox4):
+    """The Philox round function and key schedule, through the 4x64 instance,
+    against numpy's Philox bit generator (numpy increments its 256-bit counter
+    before each block, so its block for counter c is Philox(c + 1))."""
+    r = _rng(20)
+    for _ in range(20):
+        c = [int(x) for x in r.integers(0, 2 ** 63, size=4, dtype=np.uint64)]
+        key = [int(x) for x in r.integers(0, 2 ** 63, size=2, dtype=np.uint64)]
+        bg = np.random.Philox(key=np.array(key, dtype=np.uint64), counter=np.array(c, dtype=np.uint64))
+        got = [int(x) for x in bg.random_raw(4)]
+        exp = philox4([c[0] + 1] + c[1:], key, 64)
+        assert got == list(exp), "Philox4x64-10 differs from numpy's Philox"
+
+
+def check_philox_vectorised(philox4, philox4x32_arrays):
+    """The numpy-vectorised 4x32 rounds equal the integer rounds, word for word."""
+    r = _rng(21)
+    c = r.integers(0, 2 ** 32, size=(4, 64), dtype=np.uint64)
+    k0, k1 = (int(x) for x in r.integers(0, 2 ** 32, size=2))
+    words = philox4x32_arrays(c[0], c[1], c[2], c[3], k0, k1)
+    for n in range(64):
+        exp = philox4([int(c[w, n]) for w in range(4)], [k0, k1], 32)
+        assert [int(words[w][n]) for w in range(4)] == list(exp), "vectorised Philox4x32 differs"
+
+
+def check_dropout_layout(draws, philox4):
+    """Element (i, j) of head bh draws byte (j & 3) of output word (i & 3) of the
+    Philox4x32-10 block with counter (j >> 2, i >> 2, bh, 0) and key (seed low, high)."""
+    seed = 0x1234_5678_9ABC_DEF0
+    for bh in (0, 5):
+        u = draws(11, 13, bh, seed)
+        for i in range(11):
+            for j in range(13):
+                w = philox4([j >> 2, i >> 2, bh, 0], [seed & 0xFFFFFFFF, seed >> 32], 32)[i & 3]
+                assert u[i, j] == (w >> (8 * (j & 3))) & 0xFF, f"draw layout at ({i}, {j}, {bh})"
+
+
+def check_dropout_statistics(draws, keep_scale):
+    """Draws are uniform bytes; kept entries are scaled so that E[Z] = 1."""
+    u = np.concatenate([draws(256, 256, bh, 77 + bh).ravel() for bh in range(4)]).astype(np.float64)
+    n = u.size
+    counts = np.bincount(u.astype(np.int64), minlength=256)
+    mean, sd = n / 256, np.sqrt(n / 256 * (1 - 1 / 256))
+    assert np.all(np.abs(counts - mean) <= 6 * sd), "byte draws are not uniform"
+    for p in (0.1, 0.5, 0.9):
+        Z = np.concatenate([keep_scale(256, 256, bh, 99, p).ravel() for bh in range(4)])
+        t = int(round(256 * p))
+        q = 1 - t / 256
+        kept = np.mean(Z > 0)
+        assert abs(kept - q) <= 5 * np.sqrt(q * (1 - q) / Z.size), f"keep rate at p={p}"
+        assert abs(Z.mean() - 1.0) <= 5 * np.sqrt((1 - q) / q / Z.size), f"E[Z] != 1 at p={p}"
+
+
+def check_dropout_reductions(forward, backward, forward_dropout, backward_dropout):
+    """p = 0 keeps every element with Z = 1: the plain attention."""
+    r = _rng(22)
+    q, k, v, do = (r.standard_normal((2, 9, 4)) for _ in range(4))
+    for causal in (False, True):
+        O, lse = forward(q, k, v, 0.5, causal=causal)
+        Od, lsed = forward_dropout(q, k, v, 0.5, 0.0, 123, causal=causal)
+        _close(Od, O, 1e-13, "dropout p=0 O")
+        _close(lsed, lse, 1e-13, "dropout p=0 lse")
+        for a, b in zip(backward(q, k, v, do, 0.5, causal=causal), backward_dropout(q, k, v, do, 0.5, 0.0, 123,
+                                                                                      causal=causal)):
+            _close(b, a, 1e-12, "dropout p=0 gradients")
+
+
+def check_dropout_finite_differences(forward_dropout, backward_dropout):
+    """For a fixed seed the mask is fixed: central differences of L = <dO, O>."""
+    r = _rng(23)
+    n, nk, d, h = 6, 9, 3, 1e-5
+    mask = np.array([[1, 0, 1], [1, 1, 0]], dtype=np.uint8)
+    for causal, bm, p in ((False, None, 0.3), (True, None, 0.5), (False, mask, 0.2)):
+        q, do = r.standard_normal((n, d)), r.standard_normal((n, d))
+        k, v = r.standard_normal((nk, d)), r.standard_normal((nk, d))
+        dq, dk, dv, D = backward_dropout(q, k, v, do, 0.45, p, 2024, causal=causal, block_mask=bm, tile=3,
+                                         return_d=True)
+        O, _ = forward_dropout(q, k, v, 0.45, p, 2024, causal=causal, block_mask=bm, tile=3)
+        _close(D, (do * O).sum(axis=1), 1e-12, "dropout: rowsum(P∘dP) = rowsum(dO∘O)")
+
+        def L(q_, k_, v_):
+            Ox, _ = forward_dropout(q_, k_, v_, 0.45, p, 2024, causal=causal, block_mask=bm, tile=3)
+            return float(np.sum(do * Ox))
+
+        for which, grad in (("q", dq), ("k", dk), ("v", dv)):
+            base = {"q": q, "k": k, "v": v}
+            R = r.standard_normal(base[which].shape)
+            plus = {x: a + h * R if x == which else a for x, a in base.items()}
+            minus = {x: a - h * R if x == which else a for x, a in base.items()}
+            fd = (L(plus["q"], plus["k"], plus["v"]) - L(minus["q"], minus["k"], minus["v"])) / (2 * h)
+            an = float(np.sum(grad * R))
+            assert abs(fd - an) <= 1e-7 * max(1.0, abs(an)), f"dropout finite differences d{which}: {fd} vs {an}"

@@ -68,6 +68,66 @@ def _run_all(mod):
     return failures
 
 
+DROPOUT_SRC = os.path.join(os.path.dirname(SRC), "dropout.py")
+
+DROPOUT_MUTANTS = {
+    "dropout scale 1/q dropped": ("256.0 / (256 - t), 0.0)", "1.0, 0.0)"),
+    "dropout mask missing from dP": ("dP = (do[idx] @ v[idx].T) * Z", "dP = (do[idx] @ v[idx].T)"),
+    "dropout counter rows and columns swapped": ("philox4x32_arrays(j >> np.uint64(2), i >> np.uint64(2),",
+                                                 "philox4x32_arrays(i >> np.uint64(2), j >> np.uint64(2),"),
+    "dropout word picked by column": ("sel = (i & np.uint64(3))", "sel = (j & np.uint64(3))"),
+    "Philox key bump missing": ("kk0, kk1 = (kk0 + w0) & 0xFFFFFFFF, (kk1 + w1) & 0xFFFFFFFF",
+                                "kk0, kk1 = kk0, kk1"),
+    "Philox high and low halves swapped": ("x0, x1, x2, x3 = (p1 >> width) ^ x1 ^ k0, p1 & mask,",
+                                           "x0, x1, x2, x3 = (p1 & mask) ^ x1 ^ k0, p1 >> width,"),
+    "dropout keeps draws below the threshold": ("np.where(draws(nq, nk, bh, seed) >= t,",
+                                                "np.where(draws(nq, nk, bh, seed) < t,"),
+}
+
+
+def _dropout_mutant(old, new):
+    import oracle
+    with open(DROPOUT_SRC) as f:
+        text = f.read()
+    assert text.count(old) >= 1, f"mutation site not found: {old!r}"
+    text = text.replace(old, new).replace("from .attention import", "from oracle.attention import")
+    mod = types.ModuleType("oracle_dropout_mutant")
+    mod.__file__ = DROPOUT_SRC
+    exec(compile(text, DROPOUT_SRC + " (mutant)", "exec"), mod.__dict__)
+    return oracle, mod
+
+
+def _run_dropout(oracle, mod):
+    failures = []
+    checks = [
+        lambda: pins.check_philox_against_numpy(mod.philox4),
+        lambda: pins.check_philox_vectorised(mod.philox4, mod.philox4x32_arrays),
+        lambda: pins.check_dropout_layout(mod.draws, mod.philox4),
+        lambda: pins.check_dropout_statistics(mod.draws, mod.keep_scale),
+        lambda: pins.check_dropout_reductions(oracle.forward, oracle.backward, mod.forward_dropout,
+                                              mod.backward_dropout),
+        lambda: pins.check_dropout_finite_differences(mod.forward_dropout, mod.backward_dropout),
+    ]
+    for c in checks:
+        try:
+            c()
+        except AssertionError as e:
+            failures.append(str(e))
+        except Exception as e:  # a crash also counts as caught
+            failures.append(repr(e))
+    return failures
+
+
+def test_unmutated_dropout_copy_passes():
+    assert _run_dropout(*_dropout_mutant("import numpy as np", "import numpy as np")) == []
+
+
+@pytest.mark.parametrize("name", sorted(DROPOUT_MUTANTS))
+def test_dropout_mutant_is_caught(name):
+    old, new = DROPOUT_MUTANTS[name]
+    assert _run_dropout(*_dropout_mutant(old, new)), f"no pin caught the planted mistake: {name}"
+
+
 def test_unmutated_copy_passes():
     with open(SRC) as f:
         text = f.read()

@@ -159,3 +159,13 @@ def test_backward_rows_finite_differences():
 
 def test_row_routines_with_unequal_lengths():
     pins.check_rows_unequal_lengths(oracle.forward, oracle.forward_rows, oracle.backward_rows)
+
+
+def test_dropout():
+    from oracle import dropout as Dr
+    pins.check_philox_against_numpy(Dr.philox4)
+    pins.check_philox_vectorised(Dr.philox4, Dr.philox4x32_arrays)
+    pins.check_dropout_layout(Dr.draws, Dr.philox4)
+    pins.check_dropout_statistics(Dr.draws, Dr.keep_scale)
+    pins.check_dropout_reductions(oracle.forward, oracle.backward, Dr.forward_dropout, Dr.backward_dropout)
+    pins.check_dropout_finite_differences(Dr.forward_dropout, Dr.backward_dropout)
