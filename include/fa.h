@@ -186,6 +186,43 @@ fa_status fa_fwd_splitkv(fa_dtype dtype, const void* q, const void* k, const voi
                          int n_splits, void* workspace, cudaStream_t stream);
 
 /*
+ * Attention with dropout on the probabilities, fused in the same kernels
+ * ("FlashAttention" concept card, 算法要点 "Kernel fusion": QK^T -> softmax
+ * (+ mask / dropout) -> PV). O = (P o Z) V, with P the softmax of the scaled,
+ * masked scores (lse is that of P) and Z the dropout keep decisions: element
+ * (i, j) of head bh = b*H + h is kept iff its draw u >= t, t = floor(256 p + 1/2),
+ * and a kept entry is 256 / (256 - t) (so p is used rounded to t/256). The
+ * draws come from Philox4x32-10 (Salmon et al., SC'11): one block per 4 x 4
+ * block of (query row, key), counter (j >> 2, i >> 2, bh, 0), key (seed low
+ * 32 bits, seed high 32 bits); output word (i & 3) holds row i's draws, byte
+ * (j & 3) of it, least significant first, is u. The backward draws them again
+ * from the same seed (nothing is stored) and computes, through O = (P o Z) V:
+ * dV = (P o Z)^T dO, dP = (dO V^T) o Z, dS = P o (dP - D) with
+ * D = rowsum(dO o O), dQ = scale dS K, dK = scale dS^T Q.
+ * Arguments as fa_fwd_qk / fa_bwd_qk, plus p_drop in [0, 1) (else
+ * FA_ERR_INVALID_ARG; p_drop = 0 is exactly fa_fwd_qk / fa_bwd_qk) and the
+ * 64-bit seed; fa_bwd_dropout must get the forward's p_drop and seed.
+ */
+fa_status fa_fwd_dropout(fa_dtype dtype, const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                         int H, int Nq, int Nk, int d, float softmax_scale, int causal, const uint8_t* block_mask,
+                         float p_drop, unsigned long long seed, cudaStream_t stream);
+fa_status fa_bwd_dropout(fa_dtype dtype, const void* q, const void* k, const void* v, const void* o, const float* lse,
+                         const void* dout, void* dq, void* dk, void* dv, void* workspace, int B, int H, int Nq, int Nk,
+                         int d, float softmax_scale, int causal, const uint8_t* block_mask, float p_drop,
+                         unsigned long long seed, cudaStream_t stream);
+
+/*
+ * Debug: the dropout draws u (uint8) of every (head, query row, key) for
+ * B*H heads, Nq query rows, Nk keys, written to two DEVICE buffers of
+ * B*H*Nq*Nk bytes, [bh][i][j]: row_major through the generator path of the
+ * forward and query-stationary backward (a thread per query row), col_major
+ * through that of the key-stationary backward (a thread per key). Both equal
+ * the layout described at fa_fwd_dropout.
+ */
+fa_status fa_debug_dropout_draws(int B, int H, int Nq, int Nk, unsigned long long seed, uint8_t* row_major,
+                                 uint8_t* col_major, cudaStream_t stream);
+
+/*
  * Debug: the forward / backward with a record of the tiles each CTA loaded.
  * trace: DEVICE int32 buffer of fa_*_trace_size() entries; each record is a
  * count followed by entries (tile index) | (flags << 16).
@@ -246,6 +283,20 @@ fa_status fa_debug_timeout_probe(int timeout_ms, cudaStream_t stream);
  * without a fault. Arguments otherwise as fa_fwd.
  */
 fa_status fa_debug_fwd_withhold(fa_dtype dtype, const void* q, const void* k, const void* v, void* o, float* lse,
+                                int B, int H, int N, int d, float softmax_scale, int causal, int timeout_ms,
+                                cudaStream_t stream);
+
+/*
+ * Debug: fa_bwd with the main kernel's TMA producers issuing no load and every
+ * device-side wait limited to `timeout_ms` (1..5000): the MMA issuers' first
+ * waits run out (key-stationary CTAs: K/V; query-stationary CTAs: their first
+ * K), record FA_ERR_TIMEOUT and raise the CTA's abort flag; every role leaves
+ * its loop, the issuers wait for what they issued, and the CTAs exit. The prep
+ * launch runs normally. dq, dk, dv are not written. Arguments otherwise as
+ * fa_bwd.
+ */
+fa_status fa_debug_bwd_withhold(fa_dtype dtype, const void* q, const void* k, const void* v, const void* o,
+                                const float* lse, const void* dout, void* dq, void* dk, void* dv, void* workspace,
                                 int B, int H, int N, int d, float softmax_scale, int causal, int timeout_ms,
                                 cudaStream_t stream);
 

@@ -26,7 +26,8 @@ EXPORTED = (
     "fa_bwd_workspace_size", "fa_fwd_trace_size", "fa_bwd_trace_size", "fa_bwd_row_tile",
     "fa_debug_fwd_trace", "fa_debug_bwd_trace", "fa_debug_bwd_phase", "fa_device_status",
     "fa_debug_timeout_probe", "fa_bwd_noalloc", "fa_fwd_qk", "fa_bwd_qk", "fa_debug_fwd_withhold",
-    "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_size", "fa_fwd_splitkv_splits",
+    "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_size", "fa_fwd_splitkv_splits", "fa_debug_bwd_withhold",
+    "fa_fwd_dropout", "fa_bwd_dropout", "fa_debug_dropout_draws",
 )
 
 
@@ -66,6 +67,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "fa_device_status": ([vp], i),
         "fa_debug_timeout_probe": ([i, vp], i),
         "fa_debug_fwd_withhold": (fwd_args + [i, vp], i),
+        "fa_debug_bwd_withhold": (bwd_args + [i, vp], i),
         "fa_bwd_noalloc": (bwd_args[:10] + bwd_args[11:] + [vp], i),
         # N_q, N_k in place of N
         "fa_fwd_qk": (fwd_args[:8] + [i] + fwd_args[8:] + [vp, vp], i),
@@ -73,6 +75,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "fa_fwd_splitkv": (fwd_args[:8] + [i] + fwd_args[8:] + [vp, i, vp, vp], i),
         "fa_fwd_splitkv_workspace_size": ([i, i, i, i, i], sz),
         "fa_fwd_splitkv_splits": ([i, i, i, i], i),
+        "fa_fwd_dropout": (fwd_args[:8] + [i] + fwd_args[8:] + [vp, f, ctypes.c_ulonglong, vp], i),
+        "fa_bwd_dropout": (bwd_args[:13] + [i] + bwd_args[13:] + [vp, f, ctypes.c_ulonglong, vp], i),
+        "fa_debug_dropout_draws": ([i, i, i, i, ctypes.c_ulonglong, vp, vp, vp], i),
     }
     for name, (argtypes, restype) in sigs.items():
         fn = getattr(lib, name)
@@ -249,6 +254,17 @@ def fa_debug_fwd_withhold(q, k, v, o, lse, timeout_ms: int, causal: bool = False
     _check(st, "fa_debug_fwd_withhold")
 
 
+def fa_debug_bwd_withhold(q, k, v, o, lse, dout, dq, dk, dv, workspace, timeout_ms: int, causal: bool = False,
+                          scale=None, stream=None) -> None:
+    """The backward with main-kernel producers that issue no load: the waits run out
+    after ``timeout_ms`` and record FA_ERR_TIMEOUT (see include/fa.h)."""
+    B, H, N, d = _shape(q)
+    st = load_library().fa_debug_bwd_withhold(_dtype_code(q), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                                              _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace), B, H, N, d,
+                                              _scale(scale, d), int(bool(causal)), int(timeout_ms), _stream(stream))
+    _check(st, "fa_debug_bwd_withhold")
+
+
 def fa_debug_timeout_probe(timeout_ms: int, stream=None) -> None:
     _check(load_library().fa_debug_timeout_probe(int(timeout_ms), _stream(stream)), "fa_debug_timeout_probe")
 
@@ -302,6 +318,40 @@ def fa_fwd_splitkv(q, k, v, o, lse, n_splits: int, workspace, causal: bool = Fal
                                        _ptr(block_mask) if block_mask is not None else None, int(n_splits),
                                        _ptr(workspace), _stream(stream))
     _check(st, "fa_fwd_splitkv")
+
+
+def fa_fwd_dropout(q, k, v, o, lse, p_drop: float, seed: int, causal: bool = False, block_mask=None,
+                   scale: float | None = None, stream=None) -> None:
+    """Forward with dropout on P (keep decisions from Philox4x32-10; see include/fa.h)."""
+    B, H, Nq, d = _shape(q)
+    Nk = _shape(k)[2]
+    _check_tensors(q, k, v, o, lse, block_mask)
+    st = load_library().fa_fwd_dropout(_dtype_code(q), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Nq, Nk,
+                                       d, _scale(scale, d), int(bool(causal)),
+                                       _ptr(block_mask) if block_mask is not None else None, float(p_drop),
+                                       ctypes.c_ulonglong(int(seed)), _stream(stream))
+    _check(st, "fa_fwd_dropout")
+
+
+def fa_bwd_dropout(q, k, v, o, lse, dout, dq, dk, dv, workspace, p_drop: float, seed: int, causal: bool = False,
+                   block_mask=None, scale: float | None = None, stream=None) -> None:
+    """Backward of :func:`fa_fwd_dropout` (same p_drop and seed)."""
+    B, H, Nq, d = _shape(q)
+    Nk = _shape(k)[2]
+    _check_tensors(q, k, v, o, lse, dout, dq, dk, dv, workspace, block_mask)
+    st = load_library().fa_bwd_dropout(_dtype_code(q), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout),
+                                       _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace), B, H, Nq, Nk, d,
+                                       _scale(scale, d), int(bool(causal)),
+                                       _ptr(block_mask) if block_mask is not None else None, float(p_drop),
+                                       ctypes.c_ulonglong(int(seed)), _stream(stream))
+    _check(st, "fa_bwd_dropout")
+
+
+def fa_debug_dropout_draws(B: int, H: int, Nq: int, Nk: int, seed: int, row_major, col_major, stream=None) -> None:
+    """The dropout draws through both device generator paths (uint8 [B*H, Nq, Nk] each)."""
+    st = load_library().fa_debug_dropout_draws(B, H, Nq, Nk, ctypes.c_ulonglong(int(seed)), _ptr(row_major),
+                                               _ptr(col_major), _stream(stream))
+    _check(st, "fa_debug_dropout_draws")
 
 
 def attention_forward(q, k, v, causal: bool = False, block_mask=None, scale=None, stream=None):

@@ -49,6 +49,14 @@ bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr
 
 using fa::check_common;
 
+// Dropout threshold t of probability p (drop iff draw < t): t = floor(256 p + 1/2),
+// p in [0, 1); -1 if p is outside it.
+int drop_threshold(float p_drop) {
+  if (!(p_drop >= 0.0f && p_drop < 1.0f)) return -1;
+  const int t = static_cast<int>(p_drop * 256.0f + 0.5f);
+  return t > 255 ? 255 : t;
+}
+
 // The same limits for a problem with Nq query rows and Nk key rows (the
 // backward grid holds batch*heads*(Tq + Tk) CTAs).
 fa_status check_qk(fa_dtype dtype, int B, int H, int Nq, int Nk, int d) {
@@ -76,7 +84,8 @@ fa_status check_mask(int N, int d, const uint8_t* block_mask) {
 
 fa_status fwd_impl(fa_dtype dtype, const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
                    int N, int d, float scale, int causal, const uint8_t* mask, int32_t* trace,
-                   cudaStream_t stream, int Nk = 0, uint64_t withhold_timeout_ns = 0) {
+                   cudaStream_t stream, int Nk = 0, uint64_t withhold_timeout_ns = 0, int drop_t = 0,
+                   uint64_t drop_seed = 0) {
   fa_status s = Nk > 0 ? check_qk(dtype, B, H, N, Nk, d) : check_common(dtype, B, H, N, d);
   if (s != FA_OK) return s;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
@@ -101,6 +110,8 @@ fa_status fwd_impl(fa_dtype dtype, const void* q, const void* k, const void* v, 
     a.withhold = 1;
     a.timeout_ns = withhold_timeout_ns;
   }
+  a.drop_t = drop_t;
+  a.drop_seed = drop_seed;
   a.status = status_word();
   if (!a.status) return FA_ERR_CUDA;
   return fa::launch_fwd(a, stream) == 0 ? FA_OK : FA_ERR_CUDA;
@@ -109,7 +120,8 @@ fa_status fwd_impl(fa_dtype dtype, const void* q, const void* k, const void* v, 
 fa_status bwd_impl(fa_dtype dtype, const void* q, const void* k, const void* v, const void* o, const float* lse,
                    const void* dout, void* dq, void* dk, void* dv, void* workspace, int B, int H, int N, int d,
                    float scale, int causal, const uint8_t* mask, int32_t* trace, cudaStream_t stream,
-                   int phases = 7, int Nk = 0) {
+                   int phases = 7, int Nk = 0, uint64_t withhold_timeout_ns = 0, int drop_t = 0,
+                   uint64_t drop_seed = 0) {
   fa_status s = Nk > 0 ? check_qk(dtype, B, H, N, Nk, d) : check_common(dtype, B, H, N, d);
   if (s != FA_OK) return s;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) || !aligned16(dout) ||
@@ -138,6 +150,12 @@ fa_status bwd_impl(fa_dtype dtype, const void* q, const void* k, const void* v, 
   a.block_mask = mask;
   a.trace = trace;
   a.phases = phases;
+  if (withhold_timeout_ns != 0) {
+    a.withhold = 1;
+    a.timeout_ns = withhold_timeout_ns;
+  }
+  a.drop_t = drop_t;
+  a.drop_seed = drop_seed;
   a.status = status_word();
   if (!a.status) return FA_ERR_CUDA;
   return fa::launch_bwd(a, stream) == 0 ? FA_OK : FA_ERR_CUDA;
@@ -356,12 +374,57 @@ fa_status fa_fwd_splitkv(fa_dtype dtype, const void* q, const void* k, const voi
   return fa::launch_splitkv_merge(a, stream) == 0 ? FA_OK : FA_ERR_CUDA;
 }
 
+fa_status fa_fwd_dropout(fa_dtype dtype, const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                         int H, int Nq, int Nk, int d, float softmax_scale, int causal, const uint8_t* block_mask,
+                         float p_drop, unsigned long long seed, cudaStream_t stream) {
+  if (Nq < 1 || Nk < 1) return FA_ERR_INVALID_ARG;
+  const int t = drop_threshold(p_drop);
+  if (t < 0) return FA_ERR_INVALID_ARG;
+  if (block_mask != nullptr) {
+    fa_status s = check_mask_qk(Nq, Nk);
+    if (s != FA_OK) return s;
+  }
+  return fwd_impl(dtype, q, k, v, o, lse, B, H, Nq, d, softmax_scale, causal, block_mask, nullptr, stream, Nk, 0, t,
+                  seed);
+}
+
+fa_status fa_bwd_dropout(fa_dtype dtype, const void* q, const void* k, const void* v, const void* o, const float* lse,
+                         const void* dout, void* dq, void* dk, void* dv, void* workspace, int B, int H, int Nq, int Nk,
+                         int d, float softmax_scale, int causal, const uint8_t* block_mask, float p_drop,
+                         unsigned long long seed, cudaStream_t stream) {
+  if (Nq < 1 || Nk < 1) return FA_ERR_INVALID_ARG;
+  const int t = drop_threshold(p_drop);
+  if (t < 0) return FA_ERR_INVALID_ARG;
+  if (block_mask != nullptr) {
+    fa_status s = check_mask_qk(Nq, Nk);
+    if (s != FA_OK) return s;
+  }
+  return bwd_impl(dtype, q, k, v, o, lse, dout, dq, dk, dv, workspace, B, H, Nq, d, softmax_scale, causal, block_mask,
+                  nullptr, stream, 7, Nk, 0, t, seed);
+}
+
+fa_status fa_debug_dropout_draws(int B, int H, int Nq, int Nk, unsigned long long seed, uint8_t* row_major,
+                                 uint8_t* col_major, cudaStream_t stream) {
+  if (B < 1 || H < 1 || Nq < 1 || Nk < 1 || row_major == nullptr || col_major == nullptr) return FA_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * H > 65535) return FA_ERR_UNSUPPORTED;
+  return fa::launch_dropout_draws(B * H, Nq, Nk, seed, row_major, col_major, stream) == 0 ? FA_OK : FA_ERR_CUDA;
+}
+
 fa_status fa_debug_fwd_withhold(fa_dtype dtype, const void* q, const void* k, const void* v, void* o, float* lse,
                                 int B, int H, int N, int d, float softmax_scale, int causal, int timeout_ms,
                                 cudaStream_t stream) {
   if (timeout_ms < 1 || timeout_ms > 5000) return FA_ERR_INVALID_ARG;
   return fwd_impl(dtype, q, k, v, o, lse, B, H, N, d, softmax_scale, causal, nullptr, nullptr, stream, 0,
                   static_cast<uint64_t>(timeout_ms) * 1000000ull);
+}
+
+fa_status fa_debug_bwd_withhold(fa_dtype dtype, const void* q, const void* k, const void* v, const void* o,
+                                const float* lse, const void* dout, void* dq, void* dk, void* dv, void* workspace,
+                                int B, int H, int N, int d, float softmax_scale, int causal, int timeout_ms,
+                                cudaStream_t stream) {
+  if (timeout_ms < 1 || timeout_ms > 5000) return FA_ERR_INVALID_ARG;
+  return bwd_impl(dtype, q, k, v, o, lse, dout, dq, dk, dv, workspace, B, H, N, d, softmax_scale, causal, nullptr,
+                  nullptr, stream, 7, 0, static_cast<uint64_t>(timeout_ms) * 1000000ull);
 }
 
 fa_status fa_debug_timeout_probe(int timeout_ms, cudaStream_t stream) {

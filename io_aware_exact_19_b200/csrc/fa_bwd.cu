@@ -42,6 +42,12 @@ int launch_bwd_t(const AttnArgs& a, cudaStream_t stream) {
   p.block_mask = a.block_mask;
   p.trace = a.trace;
   p.status = a.status;
+  p.timeout_ns = a.timeout_ns;
+  p.withhold = a.withhold;
+  p.drop_t = static_cast<uint32_t>(a.drop_t);
+  p.drop_scale = 256.0f / static_cast<float>(256 - a.drop_t);
+  p.seed_lo = static_cast<uint32_t>(a.drop_seed);
+  p.seed_hi = static_cast<uint32_t>(a.drop_seed >> 32);
   const int Nk = a.Nk > 0 ? a.Nk : a.N;
   p.N = a.N;
   p.Nk = Nk;
@@ -86,7 +92,7 @@ int launch_bwd_t(const AttnArgs& a, cudaStream_t stream) {
               host::make_map_3d(&tdq, dt, 2, a.dq, a.d, a.N, BH, dq64 ? 64 : 32, 32,
                                 dq64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE);
     if (!ok) return static_cast<int>(cudaErrorInvalidValue);
-    auto kern = bwd::fa_bwd_main_kernel<D, BF16>;
+    auto kern = a.drop_t > 0 ? bwd::fa_bwd_main_kernel<D, BF16, true> : bwd::fa_bwd_main_kernel<D, BF16, false>;
     cudaError_t e = host::ensure_dynamic_smem(reinterpret_cast<const void*>(kern), C::kAlloc);
     if (e != cudaSuccess) return static_cast<int>(e);
     dim3 grid(static_cast<unsigned>(BH) * static_cast<unsigned>(p.Tq + p.Tk));

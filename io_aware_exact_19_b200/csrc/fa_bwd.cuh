@@ -47,6 +47,7 @@
 
 #include <cuda_fp16.h>
 
+#include "philox.cuh"
 #include "sm100.cuh"
 
 namespace fa {
@@ -95,14 +96,28 @@ struct Cfg {
 };
 
 // Barrier slots of the two CTA kinds (they share the same shared-memory words).
+// `drain` (both kinds) lets the MMA issuer wait for its own MMAs on the abort path.
 struct KeyBars {
   static constexpr int kv_full = 0, qdo_full = 1, qdo_empty = 4, s_full = 7, s_free = 8, dp_full = 9,
-                       p_full = 10, all_done = 11;
+                       p_full = 10, all_done = 11, drain = 19;
 };
 struct QueryBars {
   static constexpr int q_ready = 0, k_full = 1, k_empty = 4, v_full = 7, v_empty = 10, s_full = 13,
-                       s_free = 14, dp_full = 15, ds_full = 16, all_done = 17, qdo_in = 18;
+                       s_free = 14, dp_full = 15, ds_full = 16, all_done = 17, qdo_in = 18, drain = 19;
 };
+
+// Abort path of a producer: wait (bounded, whatever the abort flag says) for the
+// last load issued into each of the S stages of a ring whose full barriers start
+// at `bar0`, `issued` loads in all, so no copy still writes shared memory when
+// the CTA exits.
+__device__ __forceinline__ void drain_ring(const uint64_t* bars, int bar0, int S, int issued, uint64_t timeout_ns) {
+  for (int s = 0; s < S; ++s) {
+    if (issued > s) {
+      const int last = issued - 1 - ((issued - 1 - s) % S);
+      mbar_wait_bounded(smem_u32(&bars[bar0 + s]), (last / S) & 1, timeout_ns);
+    }
+  }
+}
 
 // Walks the tiles one CTA visits, in ascending order. Dense and causal ranges
 // are arithmetic; a block mask is read from global memory (a few cached bytes
@@ -160,6 +175,13 @@ struct Params {
   const uint8_t* block_mask;  // [Tq][Tk] or null
   int32_t* trace;
   int* status;
+  uint64_t timeout_ns;  // limit of every wait
+  int withhold;         // debug: the producers issue no load, so the first waits run out
+  // Dropout (kDropout instances, see philox.cuh): an element is dropped iff its
+  // draw is below drop_t; kept ones are scaled by drop_scale = 256 / (256 - drop_t).
+  uint32_t drop_t;
+  float drop_scale;
+  uint32_t seed_lo, seed_hi;
   int N;     // query rows
   int Nk;    // key / value rows
   int d;     // head dimension of the tensors (<= D; columns d..D-1 are zero in the kernel)
@@ -311,7 +333,7 @@ __device__ __forceinline__ void store_rows_tma(uint32_t taddr, float mul, bool h
 
 // --------------------------------------------------------------------------- key-stationary CTA
 
-template <int D, bool BF16>
+template <int D, bool BF16, bool kDropout>
 __device__ __forceinline__ void key_cta(const Ctx& c, const Params& p, const CUtensorMap* tq, const CUtensorMap* tk,
                                         const CUtensorMap* tv, const CUtensorMap* tdo, const CUtensorMap* tdk,
                                         const CUtensorMap* tdv, int j) {
@@ -334,18 +356,20 @@ __device__ __forceinline__ void key_cta(const Ctx& c, const Params& p, const CUt
       TileCursor cur = c.cursor;
       int32_t* tr = p.trace ? p.trace + (static_cast<size_t>(c.bh) * p.Tk + j) * (p.Tq + 1) : nullptr;
       if (tr) tr[0] = len;
-      if (len > 0) {
+      if (len > 0 && !p.withhold) {
         mbar_arrive_expect_tx(c.bar(B::kv_full), 2 * C::kTile);
         for (int ch = 0; ch < D / 64; ++ch) {
           tma_load_3d(smem_u32(sK + ch * kChunk), tk, c.bar(B::kv_full), ch * 64, j * kBlockN, c.bh);
           tma_load_3d(smem_u32(sV + ch * kChunk), tv, c.bar(B::kv_full), ch * 64, j * kBlockN, c.bh);
         }
       }
-      for (int n = 0; n < len; ++n) {
+      int issued = 0;
+      for (int n = 0; n < len && !p.withhold; ++n) {
         const int i = cur.next();
         if (tr) tr[1 + n] = i | (1 << 16);
         const int s = n % S;
         if (!mbar_wait(c.bar(B::qdo_empty + s), ((n / S) & 1) ^ 1, c.wait)) break;
+        ++issued;
         const uint32_t bar = c.bar(B::qdo_full + s);
         mbar_arrive_expect_tx(bar, 2 * C::kTile + 2 * kBR * 4);
         // The Q and dO maps have 64-row boxes: two boxes fill one 128-row chunk.
@@ -359,6 +383,10 @@ __device__ __forceinline__ void key_cta(const Ctx& c, const Params& p, const CUt
         const size_t vo = static_cast<size_t>(c.bh) * p.Npad + static_cast<size_t>(i) * kBR;
         bulk_load(smem_u32(sL + s * kBR), p.lse2 + vo, kBR * 4, bar);
         bulk_load(smem_u32(sDv + s * kBR), p.delta + vo, kBR * 4, bar);
+      }
+      if (*c.wait.abort_flag) {
+        if (len > 0 && !p.withhold) mbar_wait_bounded(c.bar(B::kv_full), 0, c.wait.timeout_ns);
+        drain_ring(c.bars, B::qdo_full, S, issued, c.wait.timeout_ns);
       }
     } else if (c.warp == 1 && c.lane == 0 && len > 0) {
       // ---------------------------------------------------------- MMA issuer
@@ -391,6 +419,7 @@ __device__ __forceinline__ void key_cta(const Ctx& c, const Params& p, const CUt
         umma_commit(c.bar(B::dp_full));
       };
       bool ok = mbar_wait(c.bar(B::kv_full), 0, c.wait) && mbar_wait(c.bar(B::qdo_full), 0, c.wait);
+      const bool issued = ok;  // MMAs are issued from here on
       if (ok) {
         tc_fence_after();
         issue_s(0);
@@ -424,7 +453,14 @@ __device__ __forceinline__ void key_cta(const Ctx& c, const Params& p, const CUt
         umma_commit(c.bar(B::qdo_empty + s));
         if (n + 1 < len) issue_dp(n + 1);  // dP^T columns: ordered after dV, dK read P^T, dS^T
       }
-      if (ok) umma_commit(c.bar(B::all_done));
+      if (ok) {
+        umma_commit(c.bar(B::all_done));
+      } else if (issued) {
+        // Aborting: let every MMA this thread issued complete before TMEM and the
+        // shared-memory operands are released.
+        umma_commit(c.bar(B::drain));
+        mbar_wait_bounded(c.bar(B::drain), 0, c.wait.timeout_ns);
+      }
     }
   } else {
     reg_alloc<kRegsHigh>();
@@ -474,6 +510,23 @@ __device__ __forceinline__ void key_cta(const Ctx& c, const Params& p, const CUt
         for (int x = 0; x < 64; ++x)
           if (x < lim) pv[x] = 0.0f;
       }
+      // Dropout: keep decisions of this key against query rows i*128 + qo .. +63
+      // (bit x), drawn while the dP^T MMA runs.
+      uint64_t keep = ~0ull;
+      if constexpr (kDropout) {
+        keep = 0;
+        const uint32_t rg_first = static_cast<uint32_t>(i * kBR + qo) / 4;
+#pragma unroll
+        for (int g = 0; g < 16; g += 4) {
+          const uint4 w = philox::draws_col(rg_first + g, static_cast<uint32_t>(key), static_cast<uint32_t>(c.bh),
+                                            p.seed_lo, p.seed_hi);
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+#pragma unroll
+            for (int b = 0; b < 4; ++b)
+              if (philox::draw_byte(w, k, b) >= p.drop_t) keep |= 1ull << (4 * (g + k) + b);
+        }
+      }
       if (!(ok = mbar_wait_warp(c.bar(B::dp_full), n & 1, c.wait))) break;
       tc_fence_after();
       uint32_t dr[64];
@@ -482,14 +535,32 @@ __device__ __forceinline__ void key_cta(const Ctx& c, const Params& p, const CUt
       tmem_ld_wait();
       const uint32_t aD = smem_u32(sDv + s * kBR + qo);
       uint32_t pk[32], dk[32];
+      if constexpr (kDropout) {
+        // dV takes (P o Z)^T, dS^T = P^T o (dP^T o Z - D), Z = keep * drop_scale.
+        const float zs = p.drop_scale;
 #pragma unroll
-      for (int x = 0; x < 64; x += 4) {
-        const float4 d4 = lds128(aD + x * 4);
-        pk[x / 2] = pack2<BF16>(pv[x], pv[x + 1]);
-        pk[x / 2 + 1] = pack2<BF16>(pv[x + 2], pv[x + 3]);
-        dk[x / 2] = pack2<BF16>(pv[x] * (__uint_as_float(dr[x]) - d4.x), pv[x + 1] * (__uint_as_float(dr[x + 1]) - d4.y));
-        dk[x / 2 + 1] =
-            pack2<BF16>(pv[x + 2] * (__uint_as_float(dr[x + 2]) - d4.z), pv[x + 3] * (__uint_as_float(dr[x + 3]) - d4.w));
+        for (int x = 0; x < 64; x += 4) {
+          const float4 d4 = lds128(aD + x * 4);
+          const float z0 = (keep >> x) & 1 ? zs : 0.0f, z1 = (keep >> (x + 1)) & 1 ? zs : 0.0f;
+          const float z2 = (keep >> (x + 2)) & 1 ? zs : 0.0f, z3 = (keep >> (x + 3)) & 1 ? zs : 0.0f;
+          pk[x / 2] = pack2<BF16>(pv[x] * z0, pv[x + 1] * z1);
+          pk[x / 2 + 1] = pack2<BF16>(pv[x + 2] * z2, pv[x + 3] * z3);
+          dk[x / 2] = pack2<BF16>(pv[x] * fmaf(__uint_as_float(dr[x]), z0, -d4.x),
+                                  pv[x + 1] * fmaf(__uint_as_float(dr[x + 1]), z1, -d4.y));
+          dk[x / 2 + 1] = pack2<BF16>(pv[x + 2] * fmaf(__uint_as_float(dr[x + 2]), z2, -d4.z),
+                                      pv[x + 3] * fmaf(__uint_as_float(dr[x + 3]), z3, -d4.w));
+        }
+      } else {
+#pragma unroll
+        for (int x = 0; x < 64; x += 4) {
+          const float4 d4 = lds128(aD + x * 4);
+          pk[x / 2] = pack2<BF16>(pv[x], pv[x + 1]);
+          pk[x / 2 + 1] = pack2<BF16>(pv[x + 2], pv[x + 3]);
+          dk[x / 2] =
+              pack2<BF16>(pv[x] * (__uint_as_float(dr[x]) - d4.x), pv[x + 1] * (__uint_as_float(dr[x + 1]) - d4.y));
+          dk[x / 2 + 1] = pack2<BF16>(pv[x + 2] * (__uint_as_float(dr[x + 2]) - d4.z),
+                                      pv[x + 3] * (__uint_as_float(dr[x + 3]) - d4.w));
+        }
       }
       tmem_st32(tl + 128 + qo, pk);
       tmem_st32(tl + 128 + qo + 32, dk);
@@ -516,7 +587,7 @@ __device__ __forceinline__ void key_cta(const Ctx& c, const Params& p, const CUt
 
 // --------------------------------------------------------------------------- query-stationary CTA
 
-template <int D, bool BF16>
+template <int D, bool BF16, bool kDropout>
 __device__ __forceinline__ void query_cta(const Ctx& c, const Params& p, const CUtensorMap* tq,
                                           const CUtensorMap* tk, const CUtensorMap* tv, const CUtensorMap* tdo,
                                           const CUtensorMap* tdq, int i) {
@@ -541,7 +612,7 @@ __device__ __forceinline__ void query_cta(const Ctx& c, const Params& p, const C
                                   (static_cast<size_t>(c.bh) * p.Tq + i) * (p.Tk + 1)
                             : nullptr;
       if (tr) tr[0] = len;
-      if constexpr (kStageQdo) {
+      if (kStageQdo && !p.withhold) {
         // Q_i and dO_i land in the last K and V stages, which the elementwise warps
         // copy into TMEM before those stages first take K and V.
         mbar_arrive_expect_tx(c.bar(B::qdo_in), 2 * C::kTile);
@@ -552,7 +623,8 @@ __device__ __forceinline__ void query_cta(const Ctx& c, const Params& p, const C
             tma_load_3d(smem_u32(sV + off), tdo, c.bar(B::qdo_in), ch * 64, i * kBlockQ + hr * 64, c.bh);
           }
       }
-      for (int n = 0; n < len; ++n) {
+      int k_issued = 0, v_issued = 0;
+      for (int n = 0; n < len && !p.withhold; ++n) {
         const int jt = cur.next();
         if (tr) tr[1 + n] = jt | (1 << 16);
         const int s = n % S;
@@ -562,11 +634,18 @@ __device__ __forceinline__ void query_cta(const Ctx& c, const Params& p, const C
         for (int ch = 0; ch < D / 64; ++ch)
           tma_load_3d(smem_u32(sK + s * C::kTile + ch * kChunk), tk, c.bar(B::k_full + s), ch * 64,
                       jt * kBlockN, c.bh);
+        ++k_issued;
         if (!mbar_wait(c.bar(B::v_empty + s), ((n / S) & 1) ^ 1, c.wait)) break;
         mbar_arrive_expect_tx(c.bar(B::v_full + s), C::kTile);
         for (int ch = 0; ch < D / 64; ++ch)
           tma_load_3d(smem_u32(sV + s * C::kTile + ch * kChunk), tv, c.bar(B::v_full + s), ch * 64,
                       jt * kBlockN, c.bh);
+        ++v_issued;
+      }
+      if (*c.wait.abort_flag) {
+        if (kStageQdo && !p.withhold) mbar_wait_bounded(c.bar(B::qdo_in), 0, c.wait.timeout_ns);
+        drain_ring(c.bars, B::k_full, S, k_issued, c.wait.timeout_ns);
+        drain_ring(c.bars, B::v_full, S, v_issued, c.wait.timeout_ns);
       }
     } else if (c.warp == 1 && c.lane == 0 && len > 0) {
       // ---------------------------------------------------------- MMA issuer
@@ -604,6 +683,7 @@ __device__ __forceinline__ void query_cta(const Ctx& c, const Params& p, const C
         return true;
       };
       bool ok = mbar_wait(c.bar(B::q_ready), 0, c.wait);
+      const bool issued = ok;  // MMAs may be issued from here on
       if (ok) {
         tc_fence_after();
         ok = issue_s(0) && issue_dp(0);
@@ -627,7 +707,14 @@ __device__ __forceinline__ void query_cta(const Ctx& c, const Params& p, const C
         umma_commit(c.bar(B::k_empty + s));               // K_n free once dQ_n is done
         if (n + 1 < len && !(ok = issue_dp(n + 1))) break;  // dP columns: ordered after dQ_n read dS_n
       }
-      if (ok) umma_commit(c.bar(B::all_done));
+      if (ok) {
+        umma_commit(c.bar(B::all_done));
+      } else if (issued) {
+        // Aborting: let every MMA this thread issued complete before TMEM and the
+        // shared-memory operands are released.
+        umma_commit(c.bar(B::drain));
+        mbar_wait_bounded(c.bar(B::drain), 0, c.wait.timeout_ns);
+      }
     }
   } else {
     reg_alloc<kRegsHigh>();
@@ -714,6 +801,23 @@ __device__ __forceinline__ void query_cta(const Ctx& c, const Params& p, const C
         for (int x = 0; x < 64; ++x)
           if (x > lim) pv[x] = 0.0f;
       }
+      // Dropout: keep decisions of this query row against keys jt*128 + 64h .. +63
+      // (bit x), drawn while the dP MMA runs.
+      uint64_t keep = ~0ull;
+      if constexpr (kDropout) {
+        keep = 0;
+        const uint32_t cg_first = static_cast<uint32_t>(jt * kBlockN + 64 * h) / 4;
+#pragma unroll
+        for (int g = 0; g < 16; g += 4) {
+          const uint4 w = philox::draws_row(cg_first + g, static_cast<uint32_t>(qrow), static_cast<uint32_t>(c.bh),
+                                            p.seed_lo, p.seed_hi);
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+#pragma unroll
+            for (int b = 0; b < 4; ++b)
+              if (philox::draw_byte(w, k, b) >= p.drop_t) keep |= 1ull << (4 * (g + k) + b);
+        }
+      }
       if (!(ok = mbar_wait_warp(c.bar(B::dp_full), n & 1, c.wait))) break;  // dP_n
       tc_fence_after();
       uint32_t dr[64];
@@ -721,10 +825,21 @@ __device__ __forceinline__ void query_cta(const Ctx& c, const Params& p, const C
       tmem_ld32(tl + C::kColDP2 + 64 * h + 32, *reinterpret_cast<uint32_t(*)[32]>(&dr[32]));
       tmem_ld_wait();
       uint32_t dk[32];
+      if constexpr (kDropout) {
+        // dS = P o (dP o Z - D), Z = keep * drop_scale.
+        const float zs = p.drop_scale;
 #pragma unroll
-      for (int x = 0; x < 32; ++x)
-        dk[x] = pack2<BF16>(pv[2 * x] * (__uint_as_float(dr[2 * x]) - dd),
-                            pv[2 * x + 1] * (__uint_as_float(dr[2 * x + 1]) - dd));
+        for (int x = 0; x < 32; ++x) {
+          const float z0 = (keep >> (2 * x)) & 1 ? zs : 0.0f, z1 = (keep >> (2 * x + 1)) & 1 ? zs : 0.0f;
+          dk[x] = pack2<BF16>(pv[2 * x] * fmaf(__uint_as_float(dr[2 * x]), z0, -dd),
+                              pv[2 * x + 1] * fmaf(__uint_as_float(dr[2 * x + 1]), z1, -dd));
+        }
+      } else {
+#pragma unroll
+        for (int x = 0; x < 32; ++x)
+          dk[x] = pack2<BF16>(pv[2 * x] * (__uint_as_float(dr[2 * x]) - dd),
+                              pv[2 * x + 1] * (__uint_as_float(dr[2 * x + 1]) - dd));
+      }
       tmem_st32(tl + C::kColDP2 + 64 * h, dk);
       tmem_st_wait();
       tc_fence_before();
@@ -753,7 +868,7 @@ __device__ __forceinline__ void query_cta(const Ctx& c, const Params& p, const C
 // Rank 2t: key-stationary CTA for key tile t; rank 2t+1: query-stationary CTA
 // for query tile T-1-t. Under a causal mask small key tiles and large query
 // tiles carry the most work, so the heaviest CTAs of both kinds start first.
-template <int D, bool BF16>
+template <int D, bool BF16, bool kDropout>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_bwd_main_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                        const __grid_constant__ CUtensorMap tmap_v, const __grid_constant__ CUtensorMap tmap_do,
@@ -804,6 +919,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(c.bar(B::dp_full), 1);
       mbar_init(c.bar(B::p_full), 256);
       mbar_init(c.bar(B::all_done), 1);
+      mbar_init(c.bar(B::drain), 1);
     } else {
       using B = QueryBars;
       mbar_init(c.bar(B::q_ready), 256);
@@ -819,6 +935,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(c.bar(B::ds_full), 256);
       mbar_init(c.bar(B::all_done), 1);
       mbar_init(c.bar(B::qdo_in), 1);
+      mbar_init(c.bar(B::drain), 1);
     }
     fence_barrier_init();
   }
@@ -848,12 +965,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   c.tmem = *tmem_slot;
   c.len = *tile_count;
-  c.wait = WaitCtx{abort_flag, p.status};
+  c.wait = WaitCtx{abort_flag, p.status, p.timeout_ns};
 
   if (keys) {
-    key_cta<D, BF16>(c, p, &tmap_q, &tmap_k, &tmap_v, &tmap_do, &tmap_dk, &tmap_dv, tile);
+    key_cta<D, BF16, kDropout>(c, p, &tmap_q, &tmap_k, &tmap_v, &tmap_do, &tmap_dk, &tmap_dv, tile);
   } else {
-    query_cta<D, BF16>(c, p, &tmap_q, &tmap_k, &tmap_v, &tmap_do, &tmap_dq, tile);
+    query_cta<D, BF16, kDropout>(c, p, &tmap_q, &tmap_k, &tmap_v, &tmap_do, &tmap_dq, tile);
   }
 
   tc_fence_before();

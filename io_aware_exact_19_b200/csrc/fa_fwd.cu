@@ -46,7 +46,13 @@ int launch_fwd_t(const AttnArgs& a, cudaStream_t stream) {
     p.head_group = static_cast<int>(g < 1 ? 1 : (g > BH ? BH : g));
   }
   p.scale_log2 = a.scale * 1.4426950408889634f;
-  auto kern = p.o_part != nullptr ? fwd::fa_fwd_kernel<D, BF16, true> : fwd::fa_fwd_kernel<D, BF16, false>;
+  p.drop_t = static_cast<uint32_t>(a.drop_t);
+  p.drop_scale = 256.0f / static_cast<float>(256 - a.drop_t);
+  p.seed_lo = static_cast<uint32_t>(a.drop_seed);
+  p.seed_hi = static_cast<uint32_t>(a.drop_seed >> 32);
+  auto kern = p.o_part != nullptr ? fwd::fa_fwd_kernel<D, BF16, fwd::kSplitKV>
+              : a.drop_t > 0      ? fwd::fa_fwd_kernel<D, BF16, fwd::kDropout>
+                                  : fwd::fa_fwd_kernel<D, BF16, fwd::kPlain>;
   cudaError_t e = host::ensure_dynamic_smem(reinterpret_cast<const void*>(kern), L::kAlloc);
   if (e != cudaSuccess) return static_cast<int>(e);
   dim3 grid(static_cast<unsigned>(static_cast<long long>(BH) * p.n_pairs * p.n_splits));

@@ -30,6 +30,7 @@
 // back in TMEM) is skipped for almost every tile.
 #pragma once
 
+#include "philox.cuh"
 #include "sm100.cuh"
 
 namespace fa {
@@ -65,6 +66,11 @@ struct Params {
   int n_splits;
   float* o_part;
   float* lse_part;
+  // Dropout (kDropout instances): an element is dropped iff its draw is below
+  // drop_t; kept ones are scaled by drop_scale = 256 / (256 - drop_t).
+  uint32_t drop_t;
+  float drop_scale;
+  uint32_t seed_lo, seed_hi;
   int BH;
   int n_pairs;  // ceil(T_q / 2)
   int Tc;       // ceil(Nk / 128)
@@ -116,9 +122,12 @@ __device__ __forceinline__ int causal_last_key_tile(int qt, int N, int Nk) {
   return last_key < 0 ? -1 : last_key / kBlockN;
 }
 
-// kSplit: split-KV launch (key ranges, fp32 partials); a separate instance so the
-// plain forward compiles without its bookkeeping.
-template <int D, bool BF16, bool kSplit>
+// Kernel variants, separate instances so the plain forward compiles without the
+// others' bookkeeping: kPlain; kSplitKV (key ranges, fp32 partials); kDropout
+// (P scaled by the dropout keep decisions before P V, see philox.cuh).
+enum Mode : int { kPlain = 0, kSplitKV = 1, kDropout = 2 };
+
+template <int D, bool BF16, int kMode>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                   const __grid_constant__ CUtensorMap tmap_v, const __grid_constant__ CUtensorMap tmap_o,
@@ -147,6 +156,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = threadIdx.x % 32;
   // Heads in groups of p.head_group (their K/V stay in L2); inside a group the
   // heaviest query-tile pairs (the last ones, under a causal mask) start first.
+  constexpr bool kSplit = kMode == kSplitKV;
   const int n_splits = kSplit ? p.n_splits : 1;
   int bh, rank;
   grouped_order(static_cast<int>(blockIdx.x), p.BH, p.n_pairs * n_splits, p.head_group, bh, rank);
@@ -475,6 +485,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           ls3 += s[c + 3];
         }
         l_sum += (ls0 + ls1) + (ls2 + ls3);
+
+        if constexpr (kMode == kDropout) {
+          // P V uses P o Z: the dropout keep decisions of this row's 128 keys, 16
+          // per generator block (the sum l above is of the undropped P).
+          const uint32_t cg_tile = static_cast<uint32_t>(j) * (kBlockN / 4);
+#pragma unroll
+          for (int g = 0; g < kBlockN / 4; g += 4) {
+            const uint4 w = philox::draws_row(cg_tile + g, static_cast<uint32_t>(row), static_cast<uint32_t>(bh),
+                                              p.seed_lo, p.seed_hi);
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+#pragma unroll
+              for (int b = 0; b < 4; ++b) {
+                const int c = 4 * (g + k) + b;
+                s[c] = philox::draw_byte(w, k, b) >= p.drop_t ? s[c] * p.drop_scale : 0.0f;
+              }
+          }
+        }
 
         uint32_t pk[64];
 #pragma unroll

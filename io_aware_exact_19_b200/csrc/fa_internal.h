@@ -31,6 +31,9 @@ struct AttnArgs {
   int phases = 7;  // backward launches to run: bit 0 prep, bit 1 main
   uint64_t timeout_ns = 2000000000ull;  // limit of every device-side wait
   int withhold = 0;  // debug (forward): the producer issues no load, so the first wait runs out
+  // dropout on P: threshold t (drop iff draw < t; 0 = no dropout) and seed
+  int drop_t = 0;
+  uint64_t drop_seed = 0;
   // split-KV forward: partial results per key range (see launch_splitkv_merge)
   int n_splits = 1;
   float* o_part = nullptr;    // fp32 [n_splits][B*H][N][d]
@@ -41,6 +44,11 @@ struct AttnArgs {
 int launch_fwd(const AttnArgs& a, cudaStream_t stream);
 // Merge of the split-KV partials (a.o_part, a.lse_part, a.n_splits) into a.o, a.lse.
 int launch_splitkv_merge(const AttnArgs& a, cudaStream_t stream);
+
+// Debug: the dropout draws of every (head, query row, key), through the
+// row-major and the column-major generator paths of the attention kernels.
+int launch_dropout_draws(int BH, int Nq, int Nk, uint64_t seed, uint8_t* row_major, uint8_t* col_major,
+                         cudaStream_t stream);
 
 // Workspace of the split-KV forward: partial O then partial lse, in bytes.
 struct SplitWorkspace {

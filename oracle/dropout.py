@@ -18,8 +18,9 @@ taken here:
     words (j >> 2, i >> 2, b·H + h, 0), key words (seed mod 2³², seed >> 32); the
     call's output word (i & 3) holds row i's four draws, byte (j & 3) of it
     (least significant first) is element (i, j)'s draw u ∈ {0, …, 255};
-  * the drop probability is rounded to t/256 with t = round(256·p): the element
-    is kept iff u ≥ t, so q = 1 − t/256 and kept entries of Z are 256/(256 − t).
+  * the drop probability is rounded to t/256 with t = ⌊256·p + ½⌋ (halves round
+    up): the element is kept iff u ≥ t, so q = 1 − t/256 and kept entries of Z
+    are 256/(256 − t).
 
 Backward, by the chain rule through O = (P∘Z)V: dV = (P∘Z)ᵀ dO, dP = (dO Vᵀ)∘Z,
 D = rowsum(P∘dP) (which equals rowsum(dO∘O)), dS = P∘(dP − D), dQ = scale·dS K,
@@ -81,7 +82,7 @@ def drop_threshold(p_drop: float) -> int:
     """t with drop probability t/256 (the reading above); 0 <= p < 1."""
     if not 0.0 <= p_drop < 1.0:
         raise ValueError("dropout probability must be in [0, 1)")
-    return min(255, int(round(256.0 * p_drop)))
+    return min(255, int(np.floor(256.0 * p_drop + 0.5)))
 
 
 def draws(nq: int, nk: int, bh: int, seed: int) -> np.ndarray:

@@ -95,9 +95,9 @@ G_TOL = 2e-2
 G_ELEM_TOL = 0.1
 
 
-def assert_grads(pairs, tile=128, what="dQ/dK/dV"):
+def assert_grads(pairs, tile=128, what="dQ/dK/dV", elem_tol=G_ELEM_TOL):
     """Assert the gradient bounds for a sequence of (g, G) pairs; returns their errors."""
     errs = [grad_errors(g, G, tile) for g, G in pairs]
-    bad = [e for e in errs if e["fro"] > G_TOL or e["tile"] > G_TOL or e["elem"] > G_ELEM_TOL]
+    bad = [e for e in errs if e["fro"] > G_TOL or e["tile"] > G_TOL or e["elem"] > elem_tol]
     assert not bad, f"{what} errors {errs}"
     return errs

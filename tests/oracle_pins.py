@@ -419,7 +419,7 @@ def check_dropout_statistics(draws, keep_scale):
     assert np.all(np.abs(counts - mean) <= 6 * sd), "byte draws are not uniform"
     for p in (0.1, 0.5, 0.9):
         Z = np.concatenate([keep_scale(256, 256, bh, 99, p).ravel() for bh in range(4)])
-        t = int(round(256 * p))
+        t = int(np.floor(256 * p + 0.5))
         q = 1 - t / 256
         kept = np.mean(Z > 0)
         assert abs(kept - q) <= 5 * np.sqrt(q * (1 - q) / Z.size), f"keep rate at p={p}"

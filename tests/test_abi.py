@@ -77,6 +77,15 @@ def test_host_argument_errors_return_before_launch(lib):
         == fa.FA_ERR_INVALID_ARG
     assert lib.fa_debug_timeout_probe(0, None) == fa.FA_ERR_INVALID_ARG
     assert lib.fa_debug_fwd_withhold(1, p, p, p, p, p, 1, 1, 128, 64, 0.1, 0, 0, None) == fa.FA_ERR_INVALID_ARG
+    # dropout: probability in [0, 1)
+    for pd in (-0.1, 1.0, float("nan")):
+        assert lib.fa_fwd_dropout(1, p, p, p, p, p, 1, 1, 128, 128, 64, 0.1, 0, None, pd, 1, None) \
+            == fa.FA_ERR_INVALID_ARG
+        assert lib.fa_bwd_dropout(1, p, p, p, p, p, p, p, p, p, p, 1, 1, 128, 128, 64, 0.1, 0, None, pd, 1, None) \
+            == fa.FA_ERR_INVALID_ARG
+    assert lib.fa_debug_dropout_draws(1, 1, 0, 5, 1, p, p, None) == fa.FA_ERR_INVALID_ARG
+    assert lib.fa_debug_bwd_withhold(1, p, p, p, p, p, p, p, p, p, p, 1, 1, 128, 64, 0.1, 0, 9999, None) \
+        == fa.FA_ERR_INVALID_ARG
     # split-KV: range count within 1..ceil(Nk/128), aligned workspace, sizes
     assert lib.fa_fwd_splitkv(1, p, p, p, p, p, 1, 1, 1, 1000, 64, 0.1, 1, None, 0, p, None) == fa.FA_ERR_INVALID_ARG
     assert lib.fa_fwd_splitkv(1, p, p, p, p, p, 1, 1, 1, 1000, 64, 0.1, 1, None, 9, p, None) == fa.FA_ERR_INVALID_ARG

@@ -152,3 +152,23 @@ def test_tile_trace_matches_oracle_enumeration(N, causal, use_mask, d):
         for i, exp in enumerate(query_lists):
             assert query_part[bh, i, 0] == len(exp)
             assert list(query_part[bh, i, 1:1 + len(exp)]) == [j | (1 << 16) for j in exp], (bh, i)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_backward_kernel_abort_path_reports_timeout_and_context_survives(d):
+    # The production backward main kernel with producers that issue no load: both
+    # CTA kinds' first waits run out (20 ms), every role leaves its loop, the MMA
+    # issuers wait for what they issued, the CTAs exit. The status word reports
+    # the time-out; the next, normal backward is still correct.
+    c = Case(1, 3, 700, d, "bf16", seed=23)
+    q, k, v, do = (c.dev[n] for n in ("q", "k", "v", "do"))
+    o, lse = fa.attention_forward(q, k, v, causal=True)
+    torch.cuda.synchronize()
+    assert fa.fa_device_status() == fa.FA_OK
+    dq, dk, dv = (torch.zeros_like(t) for t in (q, k, v))
+    ws = torch.empty(fa.fa_bwd_workspace_size(1, 3, 700, d), dtype=torch.uint8, device="cuda")
+    fa.fa_debug_bwd_withhold(q, k, v, o, lse, do, dq, dk, dv, ws, 20, causal=True)
+    assert fa.fa_device_status() == fa.FA_ERR_TIMEOUT
+    assert fa.fa_device_status() == fa.FA_OK
+    assert all(torch.count_nonzero(g) == 0 for g in (dq, dk, dv))
+    _check_full(c, True)
