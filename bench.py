@@ -480,6 +480,50 @@ def time_decode(dev, peaks, steps=50):
             "launches_per_step": 2, "steps": steps}
 
 
+def time_dropout(dev, peaks, p_drop=0.1, steps=30):
+    """The long-context causal workload with dropout on P (fa_fwd_dropout /
+    fa_bwd_dropout, p = 0.1): forward and backward TFLOP/s under the same FLOP
+    convention (dropout adds no credited FLOPs), beside the same calls at p = 0."""
+    import torch
+
+    import io_aware_exact_19_b200 as fa
+
+    w = WORKLOADS["long_causal_d128"]
+    prob = Problem(w, dev, 21)
+    seed = 0x5EED
+    f_fwd, f_bwd = step_flops(w)
+    stream = torch.cuda.current_stream()
+    out = {"workload": w["desc"] + ", dropout p=0.1 on P", "p_drop": p_drop, "steps": steps}
+    for label, pd in (("dropout", p_drop), ("no_dropout", 0.0)):
+        def fwd():
+            fa.fa_fwd_dropout(prob.q, prob.k, prob.v, prob.o, prob.lse, pd, seed, causal=True)
+
+        def bwd():
+            fa.fa_bwd_dropout(prob.q, prob.k, prob.v, prob.o, prob.lse, prob.do, prob.dq, prob.dk, prob.dv, prob.ws,
+                              pd, seed, causal=True)
+
+        for _ in range(3):
+            fwd()
+            bwd()
+        torch.cuda.synchronize()
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+        for e in ev:
+            e[0].record(stream)
+            fwd()
+            e[1].record(stream)
+            bwd()
+            e[2].record(stream)
+        torch.cuda.synchronize()
+        fwd_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / steps
+        bwd_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / steps
+        out[label] = {"fwd_ms": fwd_ms, "fwd_tflops": f_fwd / (fwd_ms * 1e-3) / 1e12, "bwd_ms": bwd_ms,
+                      "bwd_tflops": f_bwd / (bwd_ms * 1e-3) / 1e12,
+                      "fwd_frac_of_measured_peak": f_fwd / (fwd_ms * 1e-3) / 1e12 / peaks["bf16"],
+                      "bwd_frac_of_measured_peak": f_bwd / (bwd_ms * 1e-3) / 1e12 / peaks["bf16"]}
+    out["device_status"] = int(fa.fa_device_status())
+    return out
+
+
 def run_gpu(args, w, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -582,6 +626,8 @@ def run_gpu(args, w, rank, world, local_rank):
             del p2
             torch.cuda.empty_cache()
         per_workload["decode_splitkv_64k"] = time_decode(dev, peaks)
+        torch.cuda.empty_cache()
+        per_workload["long_causal_d128_dropout"] = time_dropout(dev, peaks)
         torch.cuda.empty_cache()
 
     if rank != 0:

@@ -30,12 +30,14 @@ __all__ = [
     "attention_inputs",
     "block_mask_recipe",
     "sample_rows",
+    "fp8_attention_input_bits",
 ]
 
 # (mantissa bits, minimum normal exponent, maximum finite value)
 FORMATS = {
     "fp16": (10, -14, 65504.0),
     "bf16": (7, -126, 3.3895313892515355e38),
+    "e4m3": (3, -6, 448.0),  # 8-bit float: 4 exponent bits (bias 7), 3 mantissa bits, no infinities
 }
 
 
@@ -67,16 +69,34 @@ def values_to_bits(vals: np.ndarray, fmt: str) -> np.ndarray:
     if fmt == "bf16":
         f = vals.astype(np.float32)  # exact: bf16 is a subset of float32
         return (f.view(np.uint32) >> np.uint32(16)).astype(np.uint16)
+    if fmt == "e4m3":
+        # sign | 4-bit biased exponent | 3-bit mantissa; exponent field 0 holds the
+        # subnormals (spacing 2**-9).
+        sign = (np.signbit(vals)).astype(np.uint8) << np.uint8(7)
+        a = np.abs(vals)
+        _, e = np.frexp(a)
+        e = np.maximum(e.astype(np.int64) - 1, -6)
+        normal = a >= 2.0 ** -6
+        mant = np.where(normal, np.rint(np.ldexp(a, -e) * 8) - 8, np.rint(np.ldexp(a, 9)))
+        field = np.where(normal, e + 7, 0)
+        return (sign | (field.astype(np.uint8) << np.uint8(3)) | mant.astype(np.uint8)).astype(np.uint8)
     raise ValueError(fmt)
 
 
 def bits_to_values(bits: np.ndarray, fmt: str) -> np.ndarray:
-    """Decode 16-bit storage words to exact float64 values."""
-    bits = np.asarray(bits, dtype=np.uint16)
+    """Decode 16-bit (or, for e4m3, 8-bit) storage words to exact float64 values."""
+    if fmt != "e4m3":
+        bits = np.asarray(bits, dtype=np.uint16)
     if fmt == "fp16":
         return bits.view(np.float16).astype(np.float64)
     if fmt == "bf16":
         return (bits.astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
+    if fmt == "e4m3":
+        b = np.asarray(bits, dtype=np.uint8).astype(np.int64)
+        field, mant = (b >> 3) & 15, b & 7
+        mag = np.where(field == 0, np.ldexp(mant.astype(np.float64), -9),
+                       np.ldexp(1.0 + mant / 8.0, field - 7))
+        return np.where(b & 128, -mag, mag)
     raise ValueError(fmt)
 
 
@@ -137,3 +157,19 @@ def sample_rows(n: int, count: int, seed: int) -> np.ndarray:
     """``count`` distinct row indices in [0, n), drawn without replacement, sorted."""
     rng = np.random.default_rng(seed)
     return np.sort(rng.choice(n, size=min(count, n), replace=False))
+
+
+def fp8_attention_input_bits(B: int, H: int, Nq: int, Nk: int, d: int, seed: int = 0):
+    """Q [B, H, Nq, d], K and V [B, H, Nk, d] for the 8-bit forward: standard
+    normals drawn in that order from ``default_rng(seed)``, each tensor divided by
+    its per-tensor scale s = max|x| / 448 and rounded to e4m3 (nearest, ties to
+    even). Returns ({name: uint8 words}, {name: s}); the tensor the attention
+    sees is s times the decoded words."""
+    rng = np.random.default_rng(seed)
+    bits, scales = {}, {}
+    for name, n in (("q", Nq), ("k", Nk), ("v", Nk)):
+        x = rng.standard_normal((B, H, n, d))
+        s = float(np.max(np.abs(x))) / 448.0
+        bits[name] = values_to_bits(round_to_format(x / s, "e4m3"), "e4m3")
+        scales[name] = s
+    return bits, scales

@@ -212,6 +212,23 @@ fa_status fa_bwd_dropout(fa_dtype dtype, const void* q, const void* k, const voi
                          unsigned long long seed, cudaStream_t stream);
 
 /*
+ * 8-bit forward (the FP8 variant the "FlashAttention" concept card's lineage
+ * table lists for FlashAttention-3). q8 [B,H,Nq,128], k8 and v8 [B,H,Nk,128]
+ * are DEVICE arrays of e4m3 values (1 sign, 4 exponent bits with bias 7, 3
+ * mantissa bits; one byte each); the tensors attended are q_scale * q8,
+ * k_scale * k8, v_scale * v8 (per-tensor scales > 0). Writes O [B,H,Nq,128] as
+ * bf16 and lse [B,H,Nq] (fp32) of exact attention on those tensors, with the
+ * masks of fa_fwd_qk (bottom-right causal, optional block_mask). S = Q K^T runs
+ * on the stored e4m3 values (kind::f8f6f4 MMAs, fp32 accumulation; the scales
+ * join the softmax scale); V is widened to bf16 on chip and P V runs in bf16.
+ * d must be 128 (else FA_ERR_UNSUPPORTED); scales must be finite and > 0 (else
+ * FA_ERR_INVALID_ARG). Otherwise as fa_fwd_qk.
+ */
+fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8, float q_scale, float k_scale, float v_scale,
+                     void* o, float* lse, int B, int H, int Nq, int Nk, int d, float softmax_scale, int causal,
+                     const uint8_t* block_mask, cudaStream_t stream);
+
+/*
  * Debug: the dropout draws u (uint8) of every (head, query row, key) for
  * B*H heads, Nq query rows, Nk keys, written to two DEVICE buffers of
  * B*H*Nq*Nk bytes, [bh][i][j]: row_major through the generator path of the

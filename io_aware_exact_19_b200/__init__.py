@@ -27,7 +27,7 @@ EXPORTED = (
     "fa_debug_fwd_trace", "fa_debug_bwd_trace", "fa_debug_bwd_phase", "fa_device_status",
     "fa_debug_timeout_probe", "fa_bwd_noalloc", "fa_fwd_qk", "fa_bwd_qk", "fa_debug_fwd_withhold",
     "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_size", "fa_fwd_splitkv_splits", "fa_debug_bwd_withhold",
-    "fa_fwd_dropout", "fa_bwd_dropout", "fa_debug_dropout_draws",
+    "fa_fwd_dropout", "fa_bwd_dropout", "fa_debug_dropout_draws", "fa_fwd_fp8",
 )
 
 
@@ -78,6 +78,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "fa_fwd_dropout": (fwd_args[:8] + [i] + fwd_args[8:] + [vp, f, ctypes.c_ulonglong, vp], i),
         "fa_bwd_dropout": (bwd_args[:13] + [i] + bwd_args[13:] + [vp, f, ctypes.c_ulonglong, vp], i),
         "fa_debug_dropout_draws": ([i, i, i, i, ctypes.c_ulonglong, vp, vp, vp], i),
+        "fa_fwd_fp8": ([vp, vp, vp, f, f, f, vp, vp, i, i, i, i, i, f, i, vp, vp], i),
     }
     for name, (argtypes, restype) in sigs.items():
         fn = getattr(lib, name)
@@ -345,6 +346,19 @@ def fa_bwd_dropout(q, k, v, o, lse, dout, dq, dk, dv, workspace, p_drop: float, 
                                        _ptr(block_mask) if block_mask is not None else None, float(p_drop),
                                        ctypes.c_ulonglong(int(seed)), _stream(stream))
     _check(st, "fa_bwd_dropout")
+
+
+def fa_fwd_fp8(q8, k8, v8, q_scale: float, k_scale: float, v_scale: float, o, lse, causal: bool = False,
+               block_mask=None, scale: float | None = None, stream=None) -> None:
+    """8-bit forward: ``q8``, ``k8``, ``v8`` are uint8 CUDA tensors of e4m3 values
+    [B, H, N, 128] with per-tensor scales; ``o`` is bf16 (see include/fa.h)."""
+    B, H, Nq, d = _shape(q8)
+    Nk = _shape(k8)[2]
+    _check_tensors(q8, k8, v8, o, lse, block_mask)
+    st = load_library().fa_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v8), float(q_scale), float(k_scale), float(v_scale),
+                                   _ptr(o), _ptr(lse), B, H, Nq, Nk, d, _scale(scale, d), int(bool(causal)),
+                                   _ptr(block_mask) if block_mask is not None else None, _stream(stream))
+    _check(st, "fa_fwd_fp8")
 
 
 def fa_debug_dropout_draws(B: int, H: int, Nq: int, Nk: int, seed: int, row_major, col_major, stream=None) -> None:

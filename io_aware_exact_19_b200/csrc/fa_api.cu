@@ -4,6 +4,7 @@
 
 #include <cuda_runtime.h>
 
+#include <cmath>
 #include <cstdint>
 #include <mutex>
 
@@ -401,6 +402,45 @@ fa_status fa_bwd_dropout(fa_dtype dtype, const void* q, const void* k, const voi
   }
   return bwd_impl(dtype, q, k, v, o, lse, dout, dq, dk, dv, workspace, B, H, Nq, d, softmax_scale, causal, block_mask,
                   nullptr, stream, 7, Nk, 0, t, seed);
+}
+
+fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8, float q_scale, float k_scale, float v_scale,
+                     void* o, float* lse, int B, int H, int Nq, int Nk, int d, float softmax_scale, int causal,
+                     const uint8_t* block_mask, cudaStream_t stream) {
+  if (Nq < 1 || Nk < 1 || B < 1 || H < 1 || d < 1) return FA_ERR_INVALID_ARG;
+  if (d != 128) return FA_ERR_UNSUPPORTED;
+  fa_status s = check_qk(FA_BF16, B, H, Nq, Nk, d);
+  if (s != FA_OK) return s;
+  if (block_mask != nullptr) {
+    s = check_mask_qk(Nq, Nk);
+    if (s != FA_OK) return s;
+  }
+  if (!(q_scale > 0.0f) || !(k_scale > 0.0f) || !(v_scale > 0.0f) || !std::isfinite(q_scale) ||
+      !std::isfinite(k_scale) || !std::isfinite(v_scale))
+    return FA_ERR_INVALID_ARG;
+  if (!aligned16(q8) || !aligned16(k8) || !aligned16(v8) || !aligned16(o) || !aligned16(lse))
+    return FA_ERR_INVALID_ARG;
+  fa::AttnArgs a{};
+  a.dtype = FA_BF16;
+  a.q = q8;
+  a.k = k8;
+  a.v = v8;
+  a.o = o;
+  a.lse = lse;
+  a.B = B;
+  a.H = H;
+  a.N = Nq;
+  a.Nk = Nk;
+  a.d = d;
+  a.scale = softmax_scale;
+  a.causal = causal ? 1 : 0;
+  a.block_mask = block_mask;
+  a.q_scale = q_scale;
+  a.k_scale = k_scale;
+  a.v_scale = v_scale;
+  a.status = status_word();
+  if (!a.status) return FA_ERR_CUDA;
+  return fa::launch_fwd_fp8(a, stream) == 0 ? FA_OK : FA_ERR_CUDA;
 }
 
 fa_status fa_debug_dropout_draws(int B, int H, int Nq, int Nk, unsigned long long seed, uint8_t* row_major,

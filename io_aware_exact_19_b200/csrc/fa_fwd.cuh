@@ -71,6 +71,7 @@ struct Params {
   uint32_t drop_t;
   float drop_scale;
   uint32_t seed_lo, seed_hi;
+  float v_scale;  // kFp8: per-tensor scale of V (those of Q and K are in scale_log2)
   int BH;
   int n_pairs;  // ceil(T_q / 2)
   int Tc;       // ceil(Nk / 128)
@@ -79,16 +80,24 @@ struct Params {
   float scale_log2;  // softmax scale * log2(e)
 };
 
-template <int D>
+// Shared memory. kF8: Q and K are e4m3 (one byte per element, so a 128 x 128 tile
+// is one 128-byte-swizzled chunk), V arrives as e4m3 in a staging ring and is
+// widened to 16 bits into the V ring. The V ring follows the K ring, so the
+// epilogue's staging (64 KB at d = 128, from the K ring on) stays inside both.
+template <int D, bool kF8 = false>
 struct Smem {
   static constexpr int kStages = (D == 128) ? 2 : 3;
-  static constexpr int kTileBytes = kBlockN * D * 2;  // one K or V tile (and one Q tile)
+  static constexpr int kTileBytes = kBlockN * D * 2;           // one 16-bit V tile
+  static constexpr int kQKBytes = kF8 ? kBlockN * D : kTileBytes;  // one Q or K tile
+  static constexpr int kV8Bytes = kBlockN * D;                  // one e4m3 V tile (kF8)
   static constexpr int kQOff = 0;
-  static constexpr int kKOff = kQOff + 2 * kTileBytes;
-  static constexpr int kVOff = kKOff + kStages * kTileBytes;
-  static constexpr int kBarOff = kVOff + kStages * kTileBytes;
+  static constexpr int kKOff = kQOff + 2 * kQKBytes;
+  static constexpr int kVOff = kKOff + kStages * kQKBytes;
+  static constexpr int kV8Off = kVOff + kStages * kTileBytes;
+  static constexpr int kBarOff = kV8Off + (kF8 ? kStages * kV8Bytes : 0);
   // barriers: q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_full[2], o_full[2], drain
-  static constexpr int kNumBars = 1 + 4 * kStages + 7;
+  // and, for kF8, v8_full[S], v8_empty[S]
+  static constexpr int kNumBars = 1 + 4 * kStages + 7 + (kF8 ? 2 * kStages : 0);
   static constexpr int kListOff = kBarOff + 8 * kNumBars + 16;  // + tmem slot, abort flag, list length
   static constexpr int kBytes = kListOff + 4 * kMaxSparseTiles;
   static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1024
@@ -124,15 +133,18 @@ __device__ __forceinline__ int causal_last_key_tile(int qt, int N, int Nk) {
 
 // Kernel variants, separate instances so the plain forward compiles without the
 // others' bookkeeping: kPlain; kSplitKV (key ranges, fp32 partials); kDropout
-// (P scaled by the dropout keep decisions before P V, see philox.cuh).
-enum Mode : int { kPlain = 0, kSplitKV = 1, kDropout = 2 };
+// (P scaled by the dropout keep decisions before P V, see philox.cuh); kFp8
+// (e4m3 Q, K, V with per-tensor scales: S = Q K^T by kind::f8f6f4 MMAs, V
+// widened to 16 bits in shared memory by warps 2-3 for the 16-bit P V; d = 128).
+enum Mode : int { kPlain = 0, kSplitKV = 1, kDropout = 2, kFp8 = 3 };
 
 template <int D, bool BF16, int kMode>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                   const __grid_constant__ CUtensorMap tmap_v, const __grid_constant__ CUtensorMap tmap_o,
                   const Params p) {
-  using L = Smem<D>;
+  constexpr bool kF8 = kMode == kFp8;
+  using L = Smem<D, kF8>;
   constexpr int S = L::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -151,6 +163,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto bar_p_full = [&](int q) { return smem_u32(&bars[1 + 4 * S + 2 + q]); };
   auto bar_o_full = [&](int q) { return smem_u32(&bars[1 + 4 * S + 4 + q]); };
   const uint32_t bar_drain = smem_u32(&bars[1 + 4 * S + 6]);
+  auto bar_v8_full = [&](int s) { return smem_u32(&bars[1 + 4 * S + 7 + s]); };
+  auto bar_v8_empty = [&](int s) { return smem_u32(&bars[1 + 4 * S + 7 + S + s]); };
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
@@ -175,8 +189,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < S; ++s) {
       mbar_init(bar_k_full(s), 1);
       mbar_init(bar_k_empty(s), 1);
-      mbar_init(bar_v_full(s), 1);
+      mbar_init(bar_v_full(s), kF8 ? 2 : 1);  // kF8: one arrival per widening warp
       mbar_init(bar_v_empty(s), 1);
+      if (kF8) {
+        mbar_init(bar_v8_full(s), 1);
+        mbar_init(bar_v8_empty(s), 2);
+      }
     }
     for (int q = 0; q < 2; ++q) {
       mbar_init(bar_s_full(q), 1);
@@ -268,11 +286,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tmap_v);
       int k_issued = 0, v_issued = 0;  // K and V loads issued (for the abort drain)
       const int nq = 1 + q1_active;
-      mbar_arrive_expect_tx(bar_q_full, nq * L::kTileBytes);
-      for (int q = 0; q < nq; ++q)
-        for (int c = 0; c < D / 64; ++c)
-          tma_load_3d(smem_u32(sQ + q * L::kTileBytes + c * kChunkBytes), &tmap_q, bar_q_full, c * 64,
-                      (q0 + q) * kBlockM, bh);
+      mbar_arrive_expect_tx(bar_q_full, nq * L::kQKBytes);
+      for (int q = 0; q < nq; ++q) {
+        if constexpr (kF8) {
+          tma_load_3d(smem_u32(sQ + q * L::kQKBytes), &tmap_q, bar_q_full, 0, (q0 + q) * kBlockM, bh);
+        } else {
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_3d(smem_u32(sQ + q * L::kQKBytes + c * kChunkBytes), &tmap_q, bar_q_full, c * 64,
+                        (q0 + q) * kBlockM, bh);
+        }
+      }
       if (p.trace) p.trace[static_cast<size_t>(cta) * (p.Tc + 1)] = tl.len;
       for (int n = 0; n < tl.len; ++n) {
         const uint32_t e = tl.entry(n);
@@ -281,16 +304,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int s = n % S;
         const uint32_t ph = ((n / S) & 1) ^ 1;
         if (!mbar_wait(bar_k_empty(s), ph, ctx)) break;
-        mbar_arrive_expect_tx(bar_k_full(s), L::kTileBytes);
-        for (int c = 0; c < D / 64; ++c)
-          tma_load_3d(smem_u32(sK + s * L::kTileBytes + c * kChunkBytes), &tmap_k, bar_k_full(s), c * 64,
-                      j * kBlockN, bh);
+        mbar_arrive_expect_tx(bar_k_full(s), L::kQKBytes);
+        if constexpr (kF8) {
+          tma_load_3d(smem_u32(sK + s * L::kQKBytes), &tmap_k, bar_k_full(s), 0, j * kBlockN, bh);
+        } else {
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_3d(smem_u32(sK + s * L::kQKBytes + c * kChunkBytes), &tmap_k, bar_k_full(s), c * 64,
+                        j * kBlockN, bh);
+        }
         ++k_issued;
-        if (!mbar_wait(bar_v_empty(s), ph, ctx)) break;
-        mbar_arrive_expect_tx(bar_v_full(s), L::kTileBytes);
-        for (int c = 0; c < D / 64; ++c)
-          tma_load_3d(smem_u32(sV + s * L::kTileBytes + c * kChunkBytes), &tmap_v, bar_v_full(s), c * 64,
-                      j * kBlockN, bh);
+        if constexpr (kF8) {
+          // e4m3 V into the staging ring; warps 2-3 widen it into the V ring.
+          if (!mbar_wait(bar_v8_empty(s), ph, ctx)) break;
+          mbar_arrive_expect_tx(bar_v8_full(s), L::kV8Bytes);
+          tma_load_3d(smem_u32(smem + L::kV8Off + s * L::kV8Bytes), &tmap_v, bar_v8_full(s), 0, j * kBlockN, bh);
+        } else {
+          if (!mbar_wait(bar_v_empty(s), ph, ctx)) break;
+          mbar_arrive_expect_tx(bar_v_full(s), L::kTileBytes);
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_3d(smem_u32(sV + s * L::kTileBytes + c * kChunkBytes), &tmap_v, bar_v_full(s), c * 64,
+                        j * kBlockN, bh);
+        }
         ++v_issued;
       }
       if (*abort_flag) {
@@ -304,7 +338,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (v_issued > s) {
             const int last = v_issued - 1 - ((v_issued - 1 - s) % S);
-            mbar_wait_bounded(bar_v_full(s), (last / S) & 1, p.timeout_ns);
+            mbar_wait_bounded(kF8 ? bar_v8_full(s) : bar_v_full(s), (last / S) & 1, p.timeout_ns);
           }
         }
         mbar_wait_bounded(bar_q_full, 0, p.timeout_ns);
@@ -326,13 +360,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto issue_s = [&](int q, int n) {
         const int s = n % S;
         const uint32_t d_tmem = tmem + q * 128;
-        const uint64_t bq = sdesc_add(dQ, static_cast<uint32_t>(q) * L::kTileBytes);
-        const uint64_t bk = sdesc_add(dK, static_cast<uint32_t>(s) * L::kTileBytes);
+        const uint64_t bq = sdesc_add(dQ, static_cast<uint32_t>(q) * L::kQKBytes);
+        const uint64_t bk = sdesc_add(dK, static_cast<uint32_t>(s) * L::kQKBytes);
+        if constexpr (kF8) {
+          // e4m3: K = 32 per MMA, 32 bytes along the 128-byte swizzled rows.
+          constexpr uint32_t idesc_s8 = idesc_e4m3(kBlockM, kBlockN);
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          const int kk = k * 16;
-          const uint32_t off = (kk / 64) * kChunkBytes + (kk % 64) * 2;
-          umma_ss(d_tmem, sdesc_add(bq, off), sdesc_add(bk, off), idesc_s, k > 0);
+          for (int k = 0; k < D / 32; ++k)
+            umma_ss_f8(d_tmem, sdesc_add(bq, 32 * k), sdesc_add(bk, 32 * k), idesc_s8, k > 0);
+        } else {
+#pragma unroll
+          for (int k = 0; k < D / 16; ++k) {
+            const int kk = k * 16;
+            const uint32_t off = (kk / 64) * kChunkBytes + (kk % 64) * 2;
+            umma_ss(d_tmem, sdesc_add(bq, off), sdesc_add(bk, off), idesc_s, k > 0);
+          }
         }
         umma_commit(bar_s_full(q));
       };
@@ -389,6 +431,47 @@ __global__ void __launch_bounds__(kThreads, 1)
         // shared-memory operands are released.
         umma_commit(bar_drain);
         mbar_wait_bounded(bar_drain, 0, p.timeout_ns);
+      }
+    }
+  } else if (kF8 && !p.withhold) {
+    // ------------------------------------------------------------ V widening (kFp8, warps 2-3)
+    // Warp 2 + h widens key rows [64h, 64h + 64) of each e4m3 V tile into the
+    // 16-bit V ring, in the layout TMA gives a 16-bit tile (64-column chunks,
+    // 128-byte swizzle: 16-byte piece x of row r at x ^ (r % 8)). Four lanes per
+    // row... a warp covers 4 rows x 128 columns per iteration, 16 columns a lane.
+    const int h = warp - 2;
+    bool ok = true;
+    for (int n = 0; n < tl.len; ++n) {
+      const int s = n % S;
+      const uint32_t ph = (n / S) & 1;
+      if (!(ok = mbar_wait_warp(bar_v8_full(s), ph, ctx))) break;
+      if (!(ok = mbar_wait_warp(bar_v_empty(s), ph ^ 1, ctx))) break;
+      const uint32_t src = smem_u32(smem + L::kV8Off + s * L::kV8Bytes);
+      const uint32_t dst = smem_u32(sV + s * L::kTileBytes);
+      const int c = lane % 8;  // columns 16c .. 16c + 15
+#pragma unroll 4
+      for (int it = 0; it < 16; ++it) {
+        const int r = 64 * h + 4 * it + lane / 8;
+        const float4 x4 = lds128(src + r * 128 + c * 16);
+        const uint32_t xw[4] = {__float_as_uint(x4.x), __float_as_uint(x4.y), __float_as_uint(x4.z),
+                                __float_as_uint(x4.w)};
+        uint32_t w[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          w[2 * i] = e4m3x2_to_bf16x2(xw[i] & 0xFFFFu);
+          w[2 * i + 1] = e4m3x2_to_bf16x2(xw[i] >> 16);
+        }
+        const uint32_t chunk = dst + static_cast<uint32_t>(c / 4) * kChunkBytes + static_cast<uint32_t>(r) * 128;
+        const uint32_t p0 = static_cast<uint32_t>(2 * (c % 4));
+        sts128(chunk + ((p0 ^ (r & 7)) * 16), w[0], w[1], w[2], w[3]);
+        sts128(chunk + (((p0 + 1) ^ (r & 7)) * 16), w[4], w[5], w[6], w[7]);
+      }
+      // The MMA reads the ring through the async proxy.
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(bar_v_full(s));
+        mbar_arrive(bar_v8_empty(s));
       }
     }
   }
@@ -532,7 +615,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const size_t row_base = static_cast<size_t>(bh) * p.N;
       const bool row_valid = row < p.N;
-      const float inv_l = (l_sum > 0.0f) ? 1.0f / l_sum : 0.0f;
+      const float inv_l = (l_sum > 0.0f) ? (kF8 ? p.v_scale : 1.0f) / l_sum : 0.0f;
       if (kSplit && ok) {
         // Split-KV partial: fp32 O / l of this key range (0 if it has no key for
         // the row) and its lse (-inf then), stored straight from the row's thread.

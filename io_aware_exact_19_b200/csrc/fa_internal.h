@@ -31,6 +31,8 @@ struct AttnArgs {
   int phases = 7;  // backward launches to run: bit 0 prep, bit 1 main
   uint64_t timeout_ns = 2000000000ull;  // limit of every device-side wait
   int withhold = 0;  // debug (forward): the producer issues no load, so the first wait runs out
+  // 8-bit forward: per-tensor scales of the e4m3 q, k, v
+  float q_scale = 1.0f, k_scale = 1.0f, v_scale = 1.0f;
   // dropout on P: threshold t (drop iff draw < t; 0 = no dropout) and seed
   int drop_t = 0;
   uint64_t drop_seed = 0;
@@ -42,6 +44,8 @@ struct AttnArgs {
 
 // Return 0 on success, a cudaError_t value otherwise.
 int launch_fwd(const AttnArgs& a, cudaStream_t stream);
+// The 8-bit forward (a.q, a.k, a.v e4m3; a.o bf16; d = 128).
+int launch_fwd_fp8(const AttnArgs& a, cudaStream_t stream);
 // Merge of the split-KV partials (a.o_part, a.lse_part, a.n_splits) into a.o, a.lse.
 int launch_splitkv_merge(const AttnArgs& a, cudaStream_t stream);
 

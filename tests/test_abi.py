@@ -77,6 +77,12 @@ def test_host_argument_errors_return_before_launch(lib):
         == fa.FA_ERR_INVALID_ARG
     assert lib.fa_debug_timeout_probe(0, None) == fa.FA_ERR_INVALID_ARG
     assert lib.fa_debug_fwd_withhold(1, p, p, p, p, p, 1, 1, 128, 64, 0.1, 0, 0, None) == fa.FA_ERR_INVALID_ARG
+    # 8-bit forward: d = 128 only, positive finite scales
+    assert lib.fa_fwd_fp8(p, p, p, 1.0, 1.0, 1.0, p, p, 1, 1, 128, 128, 64, 0.1, 0, None, None) == fa.FA_ERR_UNSUPPORTED
+    assert lib.fa_fwd_fp8(p, p, p, 0.0, 1.0, 1.0, p, p, 1, 1, 128, 128, 128, 0.1, 0, None, None) \
+        == fa.FA_ERR_INVALID_ARG
+    assert lib.fa_fwd_fp8(p, p, p, 1.0, float("inf"), 1.0, p, p, 1, 1, 128, 128, 128, 0.1, 0, None, None) \
+        == fa.FA_ERR_INVALID_ARG
     # dropout: probability in [0, 1)
     for pd in (-0.1, 1.0, float("nan")):
         assert lib.fa_fwd_dropout(1, p, p, p, p, p, 1, 1, 128, 128, 64, 0.1, 0, None, pd, 1, None) \

@@ -63,3 +63,28 @@ def test_block_mask_recipe_counts():
     rest = 64 * 64 - 64 - 63
     assert int(m.sum()) == 64 + 63 + round(0.2 * rest) == 921
     assert np.array_equal(m, S.block_mask_recipe(64))
+
+
+def test_e4m3_rounding_and_encoding_match_torch():
+    # Round to nearest (ties to even) onto the e4m3 grid, and the 8-bit encoding,
+    # against torch's float8_e4m3fn conversion (a library routine).
+    import torch
+    r = np.random.default_rng(0)
+    x = np.concatenate([r.standard_normal(50000) * 100, r.standard_normal(5000) * 0.01,
+                        np.array([0.0, -0.0, 448.0, -448.0, 2.0 ** -9, 2.0 ** -6, 3 * 2.0 ** -9, 17.0, 19.0])])
+    x = np.clip(x, -448.0, 448.0)
+    ours = S.round_to_format(x, "e4m3")
+    ref = torch.from_numpy(x.astype(np.float32)).to(torch.float8_e4m3fn)
+    assert np.array_equal(ours, ref.to(torch.float64).numpy())
+    bits = S.values_to_bits(ours, "e4m3")
+    assert np.array_equal(bits, ref.view(torch.uint8).numpy())
+    assert np.array_equal(S.bits_to_values(bits, "e4m3"), ours)
+
+
+def test_fp8_inputs_use_the_e4m3_range():
+    bits, scales = S.fp8_attention_input_bits(1, 2, 100, 300, 64, seed=3)
+    assert bits["q"].shape == (1, 2, 100, 64) and bits["k"].shape == (1, 2, 300, 64)
+    for name in ("q", "k", "v"):
+        vals = S.bits_to_values(bits[name], "e4m3")
+        assert np.max(np.abs(vals)) == 448.0  # the per-tensor scale maps max|x| to the largest e4m3 value
+        assert scales[name] > 0
