@@ -524,6 +524,45 @@ def time_dropout(dev, peaks, p_drop=0.1, steps=30):
     return out
 
 
+def time_fp8(dev, peaks, steps=50):
+    """The long-context causal workload's forward with 8-bit (e4m3) Q, K, V
+    (fa_fwd_fp8), TFLOP/s under the forward's FLOP convention. Its inputs (3 x 32
+    MiB) are under twice the L2 size, so the L2 is flushed between steps."""
+    import torch
+
+    import fa_synth
+    import io_aware_exact_19_b200 as fa
+
+    w = WORKLOADS["long_causal_d128"]
+    B, H, N, d = w["B"], w["H"], w["N"], w["d"]
+    bits, sc = fa_synth.fp8_attention_input_bits(B, H, N, N, d, seed=31)
+    q, k, v = (torch.from_numpy(bits[n]).to(dev) for n in ("q", "k", "v"))
+    o = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    f_fwd, _ = step_flops(w)
+    run = lambda: fa.fa_fwd_fp8(q, k, v, sc["q"], sc["k"], sc["v"], o, lse, causal=True)
+    for _ in range(3):
+        run()
+    torch.cuda.synchronize()
+    tot = 0.0
+    for i in range(steps):
+        flush.fill_(i & 0xFF)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        run()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        tot += e0.elapsed_time(e1)
+    ms = tot / steps
+    tf = f_fwd / (ms * 1e-3) / 1e12
+    return {"workload": w["desc"].replace("bf16, fwd+bwd", "e4m3 Q/K/V, forward"), "fwd_ms": ms, "fwd_tflops": tf,
+            "fwd_frac_of_measured_bf16_peak": tf / peaks["bf16"],
+            "note": "S = Q K^T in e4m3 (kind::f8f6f4), P V in bf16", "l2": "L2 flushed between steps",
+            "device_status": int(fa.fa_device_status()), "steps": steps}
+
+
 def run_gpu(args, w, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -629,6 +668,8 @@ def run_gpu(args, w, rank, world, local_rank):
         torch.cuda.empty_cache()
         per_workload["long_causal_d128_dropout"] = time_dropout(dev, peaks)
         torch.cuda.empty_cache()
+        per_workload["long_causal_d128_fp8_fwd"] = time_fp8(dev, peaks)
+        torch.cuda.empty_cache()
 
     if rank != 0:
         return 0
@@ -690,6 +731,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-per-workload", action="store_true",
                     help="time only the selected workload (the default also times every other one)")
+    ap.add_argument("--extra", choices=("decode_splitkv_64k", "long_causal_d128_dropout", "long_causal_d128_fp8_fwd"),
+                    help="run only this one of the extra measurements (1 GPU) and print its record")
     ap.add_argument("--reference-seconds", type=float, default=120.0,
                     help="approximate CPU time budget of the reference arm (warm-up plus timed steps)")
     args = ap.parse_args(argv)
@@ -704,6 +747,14 @@ def main(argv=None):
         return 2
     if args.impl == "reference":
         return run_reference(args, w, rank, world)
+    if args.extra:
+        import torch
+        dev = torch.device("cuda", local_rank)
+        torch.cuda.set_device(dev)
+        fn = {"decode_splitkv_64k": time_decode, "long_causal_d128_dropout": time_dropout,
+              "long_causal_d128_fp8_fwd": time_fp8}[args.extra]
+        print(json.dumps({args.extra: fn(dev, load_peaks())}), flush=True)
+        return 0
     if world > 1:
         import datetime
 

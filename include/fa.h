@@ -18,8 +18,11 @@
  *     [B, H, N]. All are DEVICE pointers, 16-byte aligned.
  *   - lse_i = ln sum_j exp(scale * q_i . k_j) over the keys row i may see
  *     (natural log, in the units of the scaled scores).
- *   - d must be 32, 64, 96 or 128 (32 and 96 run in the 64 and 128 kernels
- *     with the missing columns zero-filled, at the cost of the padded width);
+ *   - d must be 32, 64, 96 or 128, or 256 for the forward entry points
+ *     (fa_fwd, fa_fwd_qk, fa_blocksparse_fwd, fa_fwd_splitkv; the backward,
+ *     dropout and 8-bit entry points return FA_ERR_UNSUPPORTED for it). 32 and
+ *     96 run in the 64 and 128 kernels with the missing columns zero-filled, at
+ *     the cost of the padded width; 256 runs one query tile per CTA;
  *     N >= 1 (any value; ragged last tiles are handled); B, H >= 1 and
  *     B*H <= 65535.
  *   - causal != 0 masks key j > query i (top-left aligned; the essay's
@@ -49,7 +52,7 @@ extern "C" {
 typedef enum {
   FA_OK = 0,
   FA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, non-positive size, bad dtype */
-  FA_ERR_UNSUPPORTED = 2, /* valid but unsupported shape (d not 32/64/96/128, size limits) */
+  FA_ERR_UNSUPPORTED = 2, /* valid but unsupported shape (head dimension, size limits) */
   FA_ERR_CUDA = 3,        /* a CUDA runtime call or kernel launch failed */
   FA_ERR_TIMEOUT = 4      /* a device-side wait gave up (see fa_device_status) */
 } fa_status;

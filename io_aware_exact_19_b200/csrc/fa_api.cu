@@ -125,6 +125,7 @@ fa_status bwd_impl(fa_dtype dtype, const void* q, const void* k, const void* v, 
                    uint64_t drop_seed = 0) {
   fa_status s = Nk > 0 ? check_qk(dtype, B, H, N, Nk, d) : check_common(dtype, B, H, N, d);
   if (s != FA_OK) return s;
+  if (!fa::bwd_head_dim_supported(d)) return FA_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) || !aligned16(dout) ||
       !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
     return FA_ERR_INVALID_ARG;
@@ -166,7 +167,9 @@ fa_status bwd_impl(fa_dtype dtype, const void* q, const void* k, const void* v, 
 
 int* fa::device_status_word() { return status_word(); }
 
-bool fa::head_dim_supported(int d) { return d == 32 || d == 64 || d == 96 || d == 128; }
+bool fa::head_dim_supported(int d) { return d == 32 || d == 64 || d == 96 || d == 128 || d == 256; }
+
+bool fa::bwd_head_dim_supported(int d) { return d == 32 || d == 64 || d == 96 || d == 128; }
 
 fa_status fa::check_common(fa_dtype dtype, int B, int H, int N, int d) {
   if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_INVALID_ARG;
@@ -206,7 +209,7 @@ fa_status fa_blocksparse_fwd(fa_dtype dtype, const void* q, const void* k, const
 }
 
 size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
-  if (B < 1 || H < 1 || N < 1 || !fa::head_dim_supported(d)) return 0;
+  if (B < 1 || H < 1 || N < 1 || !fa::bwd_head_dim_supported(d)) return 0;
   return fa::bwd_workspace_layout(B, H, N, d).total;
 }
 
@@ -260,7 +263,7 @@ size_t fa_fwd_trace_size(int B, int H, int N) {
 }
 
 size_t fa_bwd_trace_size(int B, int H, int N, int d) {
-  if (B < 1 || H < 1 || N < 1 || !fa::head_dim_supported(d)) return 0;
+  if (B < 1 || H < 1 || N < 1 || !fa::bwd_head_dim_supported(d)) return 0;
   const size_t t = (static_cast<size_t>(N) + 127) / 128;
   const size_t br = static_cast<size_t>(fa::bwd_row_tile(d));
   const size_t tq = (static_cast<size_t>(N) + br - 1) / br;
@@ -271,6 +274,7 @@ fa_status fa_debug_fwd_trace(fa_dtype dtype, const void* q, const void* k, const
                              int B, int H, int N, int d, float softmax_scale, int causal,
                              const uint8_t* block_mask, int32_t* trace, cudaStream_t stream) {
   if (trace == nullptr) return FA_ERR_INVALID_ARG;
+  if (d == 256) return FA_ERR_UNSUPPORTED;  // the trace records pairs of query tiles
   if (block_mask) {
     fa_status s = check_mask(N, d, block_mask);
     if (s != FA_OK) return s;
@@ -381,6 +385,7 @@ fa_status fa_fwd_dropout(fa_dtype dtype, const void* q, const void* k, const voi
   if (Nq < 1 || Nk < 1) return FA_ERR_INVALID_ARG;
   const int t = drop_threshold(p_drop);
   if (t < 0) return FA_ERR_INVALID_ARG;
+  if (d == 256 && t > 0) return FA_ERR_UNSUPPORTED;  // dropout has a backward; d = 256 is forward-only
   if (block_mask != nullptr) {
     fa_status s = check_mask_qk(Nq, Nk);
     if (s != FA_OK) return s;

@@ -65,6 +65,7 @@ extern "C" fa_status fa_bwd_noalloc(fa_dtype dtype, const void* q, const void* k
   // The same limits as fa_bwd, then the size of the static array.
   const fa_status st = fa::check_common(dtype, B, H, N, d);
   if (st != FA_OK) return st;
+  if (!fa::bwd_head_dim_supported(d)) return FA_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) || !aligned16(dout) ||
       !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
     return FA_ERR_INVALID_ARG;

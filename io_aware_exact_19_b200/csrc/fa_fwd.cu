@@ -36,7 +36,7 @@ int launch_fwd_t(const AttnArgs& a, cudaStream_t stream) {
   p.lse_part = a.lse_part;
   p.BH = BH;
   const int Tq = (a.N + fwd::kBlockM - 1) / fwd::kBlockM;
-  p.n_pairs = (Tq + 1) / 2;
+  p.n_pairs = (Tq + L::kQTiles - 1) / L::kQTiles;  // work items per head
   p.Tc = (Nk + fwd::kBlockN - 1) / fwd::kBlockN;
   p.causal = a.causal;
   // Heads per CTA-order group: their K and V (2*N*d*2 bytes each) fit ~48 MB of L2.
@@ -50,8 +50,11 @@ int launch_fwd_t(const AttnArgs& a, cudaStream_t stream) {
   p.drop_scale = 256.0f / static_cast<float>(256 - a.drop_t);
   p.seed_lo = static_cast<uint32_t>(a.drop_seed);
   p.seed_hi = static_cast<uint32_t>(a.drop_seed >> 32);
+  // d = 256 (a forward-only head dimension) has the plain and split-KV variants.
+  constexpr int kDropMode = D == 256 ? fwd::kPlain : fwd::kDropout;
+  if (D == 256 && a.drop_t > 0) return static_cast<int>(cudaErrorInvalidValue);
   auto kern = p.o_part != nullptr ? fwd::fa_fwd_kernel<D, BF16, fwd::kSplitKV>
-              : a.drop_t > 0      ? fwd::fa_fwd_kernel<D, BF16, fwd::kDropout>
+              : a.drop_t > 0      ? fwd::fa_fwd_kernel<D, BF16, kDropMode>
                                   : fwd::fa_fwd_kernel<D, BF16, fwd::kPlain>;
   cudaError_t e = host::ensure_dynamic_smem(reinterpret_cast<const void*>(kern), L::kAlloc);
   if (e != cudaSuccess) return static_cast<int>(e);
@@ -122,6 +125,7 @@ int launch_fwd_fp8(const AttnArgs& a, cudaStream_t stream) { return launch_fwd_f
 // nothing to S or to P V) and the O stores skip or clip them.
 int launch_fwd(const AttnArgs& a, cudaStream_t stream) {
   if (a.d <= 64) return a.dtype == 1 ? launch_fwd_t<64, true>(a, stream) : launch_fwd_t<64, false>(a, stream);
+  if (a.d == 256) return a.dtype == 1 ? launch_fwd_t<256, true>(a, stream) : launch_fwd_t<256, false>(a, stream);
   return a.dtype == 1 ? launch_fwd_t<128, true>(a, stream) : launch_fwd_t<128, false>(a, stream);
 }
 

@@ -84,14 +84,17 @@ struct Params {
 // is one 128-byte-swizzled chunk), V arrives as e4m3 in a staging ring and is
 // widened to 16 bits into the V ring. The V ring follows the K ring, so the
 // epilogue's staging (64 KB at d = 128, from the K ring on) stays inside both.
+// D = 256: one query tile per CTA (S 128 + O 256 TMEM columns) and single K and
+// V stages (64 KB tiles).
 template <int D, bool kF8 = false>
 struct Smem {
-  static constexpr int kStages = (D == 128) ? 2 : 3;
+  static constexpr int kStages = D == 256 ? 1 : (D == 128 ? 2 : 3);
+  static constexpr int kQTiles = D == 256 ? 1 : 2;  // query tiles per CTA
   static constexpr int kTileBytes = kBlockN * D * 2;           // one 16-bit V tile
   static constexpr int kQKBytes = kF8 ? kBlockN * D : kTileBytes;  // one Q or K tile
   static constexpr int kV8Bytes = kBlockN * D;                  // one e4m3 V tile (kF8)
   static constexpr int kQOff = 0;
-  static constexpr int kKOff = kQOff + 2 * kQKBytes;
+  static constexpr int kKOff = kQOff + kQTiles * kQKBytes;
   static constexpr int kVOff = kKOff + kStages * kQKBytes;
   static constexpr int kV8Off = kVOff + kStages * kTileBytes;
   static constexpr int kBarOff = kV8Off + (kF8 ? kStages * kV8Bytes : 0);
@@ -178,9 +181,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int split = kSplit ? rank % n_splits : 0;
   const int key_lo = kSplit ? static_cast<int>(static_cast<long long>(split) * p.Tc / n_splits) : 0;
   const int key_hi = kSplit ? static_cast<int>(static_cast<long long>(split + 1) * p.Tc / n_splits) : p.Tc;
-  const int q0 = 2 * pair;
+  const int q0 = L::kQTiles * pair;  // an item's query tiles: q0 and (a pair) q0 + 1
   const int Tq = (p.N + kBlockM - 1) / kBlockM;
-  const int q1_active = (q0 + 1) < Tq;
+  const int q1_active = L::kQTiles == 2 && (q0 + 1) < Tq;
   const int cta = bh * p.n_pairs + pair;  // trace record (never split)
 
   if (threadIdx.x == 0) {

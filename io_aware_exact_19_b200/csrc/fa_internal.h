@@ -75,9 +75,11 @@ int bwd_row_tile(int d);
 // Device address of the per-device status word (nullptr on failure).
 int* device_status_word();
 
-// Head dimensions the kernels take: 64 and 128 natively, 32 and 96 inside the
-// 64 and 128 kernels with the missing columns zero-filled by TMA.
+// Head dimensions the forward takes: 64, 128 and 256 natively, 32 and 96 inside
+// the 64 and 128 kernels with the missing columns zero-filled by TMA. The
+// backward takes all but 256.
 bool head_dim_supported(int d);
+bool bwd_head_dim_supported(int d);
 
 // Limits every entry point applies to the element type and sizes of a square
 // (N queries, N keys) problem: FA_OK, FA_ERR_INVALID_ARG or FA_ERR_UNSUPPORTED.

@@ -47,8 +47,8 @@ __global__ void __launch_bounds__(kMergeThreads) fa_splitkv_merge_kernel(const f
   }
 #pragma unroll
   for (int k = 16; k > 0; k >>= 1) z += __shfl_xor_sync(0xffffffffu, z, k);
-  // Weighted sum of the partial rows: lanes over columns (d <= 128).
-  float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+  // Weighted sum of the partial rows: lanes over columns (d <= 256).
+  float acc[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
   if (z > 0.0f) {
     const float inv_z = 1.0f / z;
     for (int s = 0; s < n_splits; ++s) {
@@ -57,14 +57,14 @@ __global__ void __launch_bounds__(kMergeThreads) fa_splitkv_merge_kernel(const f
       const float w = expf(l - m) * inv_z;
       const float* src = o_part + (s * rows + row) * d;
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
+      for (int k = 0; k < 8; ++k) {
         const int c = lane + 32 * k;
         if (c < d) acc[k] = fmaf(w, src[c], acc[k]);
       }
     }
   }
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
+  for (int k = 0; k < 8; ++k) {
     const int c = lane + 32 * k;
     if (c < d) {
       if constexpr (BF16) {

@@ -77,6 +77,12 @@ def test_host_argument_errors_return_before_launch(lib):
         == fa.FA_ERR_INVALID_ARG
     assert lib.fa_debug_timeout_probe(0, None) == fa.FA_ERR_INVALID_ARG
     assert lib.fa_debug_fwd_withhold(1, p, p, p, p, p, 1, 1, 128, 64, 0.1, 0, 0, None) == fa.FA_ERR_INVALID_ARG
+    # d = 256 is forward-only
+    assert lib.fa_bwd(1, p, p, p, p, p, p, p, p, p, p, 1, 1, 128, 256, 0.1, 0, None) == fa.FA_ERR_UNSUPPORTED
+    assert lib.fa_bwd_workspace_size(1, 1, 128, 256) == 0
+    assert lib.fa_bwd_noalloc(1, p, p, p, p, p, p, p, p, p, 1, 1, 128, 256, 0.1, 0, None) == fa.FA_ERR_UNSUPPORTED
+    assert lib.fa_fwd_dropout(1, p, p, p, p, p, 1, 1, 128, 128, 256, 0.1, 0, None, 0.5, 1, None) \
+        == fa.FA_ERR_UNSUPPORTED
     # 8-bit forward: d = 128 only, positive finite scales
     assert lib.fa_fwd_fp8(p, p, p, 1.0, 1.0, 1.0, p, p, 1, 1, 128, 128, 64, 0.1, 0, None, None) == fa.FA_ERR_UNSUPPORTED
     assert lib.fa_fwd_fp8(p, p, p, 0.0, 1.0, 1.0, p, p, 1, 1, 128, 128, 128, 0.1, 0, None, None) \

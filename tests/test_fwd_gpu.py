@@ -48,6 +48,9 @@ def test_tiny_fp16_exact_check():
     # head dimensions 32 and 96 (inside the 64 and 128 kernels, zero-filled columns)
     (2, 3, 1000, 32, "bf16", False), (1, 2, 777, 32, "fp16", True), (1, 1, 1, 32, "bf16", True),
     (2, 2, 1000, 96, "bf16", True), (1, 2, 129, 96, "fp16", False), (1, 1, 1, 96, "bf16", False),
+    # head dimension 256 (forward only): one query tile per CTA
+    (1, 2, 1000, 256, "bf16", True), (2, 1, 777, 256, "fp16", False), (1, 1, 1, 256, "bf16", True),
+    (1, 3, 384, 256, "bf16", False),
 ])
 def test_ragged_and_small(B, H, N, d, fmt, causal):
     _check_full(Case(B, H, N, d, fmt, seed=N + d), causal)
@@ -85,7 +88,7 @@ def test_block_sparse_workload_sampled_rows():
 
 
 @pytest.mark.parametrize("causal", [False, True])
-@pytest.mark.parametrize("d", [32, 64, 96, 128])
+@pytest.mark.parametrize("d", [32, 64, 96, 128, 256])
 def test_block_sparse_full(causal, d):
     mask = S.block_mask_recipe(8, seed=4)
     _check_full(Case(2, 2, 1024, d, "bf16", seed=9), causal, mask=mask)
@@ -190,3 +193,16 @@ def test_forward_kernel_abort_path_reports_timeout_and_context_survives():
     assert fa.fa_device_status() == fa.FA_OK
     assert torch.count_nonzero(o) == 0 and torch.count_nonzero(lse) == 0
     _check_full(c, True)
+
+
+def test_head_dim_256_unequal_lengths():
+    # Forward-only head dimension with N_q != N_k (bottom-right causal).
+    B, H, Nq, Nk, d = 1, 2, 300, 777, 256
+    cq, ck = Case(B, H, Nq, d, "bf16", seed=41), Case(B, H, Nk, d, "bf16", seed=42)
+    o = torch.empty_like(cq.dev["q"])
+    lse = torch.empty((B, H, Nq), dtype=torch.float32, device="cuda")
+    fa.fa_fwd_qk(cq.dev["q"], ck.dev["k"], ck.dev["v"], o, lse, causal=True)
+    torch.cuda.synchronize()
+    assert fa.fa_device_status() == fa.FA_OK
+    O, L = oracle.forward(cq.values("q"), ck.values("k"), ck.values("v"), cq.scale, causal=True)
+    assert max_abs(cq.flat(o), O) <= O_TOL and max_abs(cq.flat(lse), L) <= LSE_TOL

@@ -66,6 +66,7 @@ def _run(B, H, Nq, Nk, d, fmt, causal, n_splits=None, mask=None, seed=0):
     (1, 1, 1024, 1024, 64, "bf16", True, 8),      # square causal: rows < 896 see nothing of range 7
     (1, 2, 5, 777, 128, "bf16", False, 7),        # one 128-key tile per range, ragged last tile
     (1, 1, 1, 1, 64, "bf16", False, 1),
+    (1, 2, 3, 2000, 256, "bf16", True, 6),       # head dimension 256 (forward only)
 ])
 def test_splitkv_matches_oracle(B, H, Nq, Nk, d, fmt, causal, n_splits):
     _run(B, H, Nq, Nk, d, fmt, causal, n_splits)
