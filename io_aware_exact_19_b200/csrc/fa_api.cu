@@ -332,6 +332,7 @@ int fa_fwd_splitkv_splits(int B, int H, int Nq, int Nk) {
   const long long base = static_cast<long long>(B) * H * ((tq + 1) / 2);  // CTAs without splitting
   const long long tk = (static_cast<long long>(Nk) + 127) / 128;
   long long ns = base >= sms ? 1 : sms / base;  // one wave of CTAs
+  if (tq == 1) ns *= 2;  // one query tile: a CTA takes two consecutive ranges
   if (ns > tk) ns = tk;
   return static_cast<int>(ns < 1 ? 1 : ns);
 }

@@ -34,6 +34,10 @@ int launch_fwd_t(const AttnArgs& a, cudaStream_t stream) {
   p.n_splits = a.n_splits > 1 || a.o_part != nullptr ? a.n_splits : 1;
   p.o_part = a.o_part;
   p.lse_part = a.lse_part;
+  {
+    const int tq = (a.N + fwd::kBlockM - 1) / fwd::kBlockM;
+    p.dual = (a.o_part != nullptr && tq == 1 && p.n_splits >= 2 && a.block_mask == nullptr && D <= 128) ? 1 : 0;
+  }
   p.BH = BH;
   const int Tq = (a.N + fwd::kBlockM - 1) / fwd::kBlockM;
   p.n_pairs = (Tq + L::kQTiles - 1) / L::kQTiles;  // work items per head
@@ -58,7 +62,8 @@ int launch_fwd_t(const AttnArgs& a, cudaStream_t stream) {
                                   : fwd::fa_fwd_kernel<D, BF16, fwd::kPlain>;
   cudaError_t e = host::ensure_dynamic_smem(reinterpret_cast<const void*>(kern), L::kAlloc);
   if (e != cudaSuccess) return static_cast<int>(e);
-  dim3 grid(static_cast<unsigned>(static_cast<long long>(BH) * p.n_pairs * p.n_splits));
+  const int split_items = p.dual ? (p.n_splits + 1) / 2 : p.n_splits;
+  dim3 grid(static_cast<unsigned>(static_cast<long long>(BH) * p.n_pairs * split_items));
   kern<<<grid, fwd::kThreads, L::kAlloc, stream>>>(tq, tk, tv, to, p);
   return static_cast<int>(cudaGetLastError());
 }

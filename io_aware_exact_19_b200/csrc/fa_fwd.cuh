@@ -66,6 +66,10 @@ struct Params {
   int n_splits;
   float* o_part;
   float* lse_part;
+  // Split-KV with one query tile per head (decoding): a CTA takes two
+  // consecutive key ranges, one per softmax warpgroup ("slot"), both against
+  // that query tile, so two dependency chains share the tensor core. No block mask.
+  int dual;
   // Dropout (kDropout instances): an element is dropped iff its draw is below
   // drop_t; kept ones are scaled by drop_scale = 256 / (256 - drop_t).
   uint32_t drop_t;
@@ -111,13 +115,27 @@ struct Smem {
 // those of the CTA's key range [lo, hi) (all of them unless split-KV).
 struct TileList {
   int len;
-  int mode;        // 0 dense, 1 causal, 2 list in shared memory
-  int lo;          // first key tile of the range
+  int mode;        // 0 dense, 1 causal, 2 list in shared memory, 3 two key ranges (dual)
+  int lo;          // first key tile of the range (mode 3: of slot 0's range)
   int lim0, lim1;  // last key tile query tile 0 / 1 uses (-1: none, e.g. no tile 1)
   const uint32_t* list;
+  int lo1, len0, len1;  // mode 3: slot 1's first key tile; tiles of each slot
 
   __device__ __forceinline__ uint32_t entry(int n) const {
     if (mode == 2) return list[n];
+    if (mode == 3) {
+      // The two slots' tiles alternate while both have some, then the longer one's rest.
+      const int both = 2 * min(len0, len1);
+      int slot, idx;
+      if (n < both) {
+        slot = n & 1;
+        idx = n >> 1;
+      } else {
+        slot = len0 > len1 ? 0 : 1;
+        idx = both / 2 + (n - both);
+      }
+      return static_cast<uint32_t>((slot ? lo1 : lo) + idx) | ((1u << slot) << 16);
+    }
     const int j = lo + n;
     const uint32_t f = (j <= lim0 ? 1u : 0u) | (j <= lim1 ? 2u : 0u);
     return static_cast<uint32_t>(j) | (f << 16);
@@ -175,15 +193,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   // heaviest query-tile pairs (the last ones, under a causal mask) start first.
   constexpr bool kSplit = kMode == kSplitKV;
   const int n_splits = kSplit ? p.n_splits : 1;
+  const bool dual = kSplit && p.dual != 0;
+  const int split_items = dual ? (n_splits + 1) / 2 : n_splits;  // CTAs per query-tile pair
   int bh, rank;
-  grouped_order(static_cast<int>(blockIdx.x), p.BH, p.n_pairs * n_splits, p.head_group, bh, rank);
-  const int pair = p.n_pairs - 1 - rank / n_splits;
-  const int split = kSplit ? rank % n_splits : 0;
-  const int key_lo = kSplit ? static_cast<int>(static_cast<long long>(split) * p.Tc / n_splits) : 0;
-  const int key_hi = kSplit ? static_cast<int>(static_cast<long long>(split + 1) * p.Tc / n_splits) : p.Tc;
+  grouped_order(static_cast<int>(blockIdx.x), p.BH, p.n_pairs * split_items, p.head_group, bh, rank);
+  const int pair = p.n_pairs - 1 - rank / split_items;
+  // Key range(s): split (slot 0) and, in dual mode, split + 1 (slot 1).
+  const int split = kSplit ? (dual ? 2 : 1) * (rank % split_items) : 0;
+  auto range_lo = [&](int sp) { return static_cast<int>(static_cast<long long>(sp) * p.Tc / n_splits); };
+  const int key_lo = kSplit ? range_lo(split) : 0;
+  const int key_hi = kSplit ? range_lo(split + 1) : p.Tc;
   const int q0 = L::kQTiles * pair;  // an item's query tiles: q0 and (a pair) q0 + 1
   const int Tq = (p.N + kBlockM - 1) / kBlockM;
-  const int q1_active = L::kQTiles == 2 && (q0 + 1) < Tq;
+  // Slot 1 holds query tile q0 + 1, or in dual mode key range split + 1 of q0.
+  const int q1_active = dual ? (split + 1 < n_splits) : (L::kQTiles == 2 && (q0 + 1) < Tq);
+  // Dual mode with at most 96 query rows: slot 1 takes the rows 32 TMEM lanes
+  // lower (its Q is loaded from row -32), so the two slots' valid rows are worked
+  // on by warps of different SM sub-partitions (a warp may only reach the 32
+  // lanes of its own quarter).
+  const int shift1 = (dual && p.N <= 96) ? 32 : 0;
   const int cta = bh * p.n_pairs + pair;  // trace record (never split)
 
   if (threadIdx.x == 0) {
@@ -215,7 +243,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // role derives it where it needs it, so it is not live across the register split.
   auto reach = [&](int qi) {
     if (qi == 1 && !q1_active) return -1;
-    return p.causal ? causal_last_key_tile(q0 + qi, p.N, p.Nk) : p.Tc - 1;
+    return p.causal ? causal_last_key_tile(q0 + (dual ? 0 : qi), p.N, p.Nk) : p.Tc - 1;
   };
   if (warp == 2) {
     const int lim0 = reach(0), lim1 = reach(1);
@@ -255,7 +283,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     tl.lim1 = reach(1);
     tl.list = list;
     tl.lo = key_lo;
-    if (p.block_mask != nullptr) {
+    if (dual) {
+      // Slot s covers key range split + s, clipped at the causal reach.
+      tl.mode = 3;
+      tl.lo1 = key_hi;
+      const int hi1 = q1_active ? range_lo(split + 2) : key_hi;
+      tl.len0 = max(0, min(key_hi, tl.lim0 + 1) - key_lo);
+      tl.len1 = q1_active ? max(0, min(hi1, tl.lim1 + 1) - key_hi) : 0;
+      tl.len = tl.len0 + tl.len1;
+    } else if (p.block_mask != nullptr) {
       tl.mode = 2;
       tl.len = *list_len;
     } else if (p.causal) {
@@ -288,15 +324,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tmap_k);
       prefetch_tmap(&tmap_v);
       int k_issued = 0, v_issued = 0;  // K and V loads issued (for the abort drain)
-      const int nq = 1 + q1_active;
+      // Dual mode: slot 1 reads query tile q0 too, from slot 0's buffer or, when its
+      // rows are shifted, from its own copy loaded from row -32 (zero-filled there).
+      const int nq = dual ? (shift1 ? 2 : 1) : 1 + q1_active;
       mbar_arrive_expect_tx(bar_q_full, nq * L::kQKBytes);
       for (int q = 0; q < nq; ++q) {
+        const int qrow = dual ? q0 * kBlockM - q * shift1 : (q0 + q) * kBlockM;
         if constexpr (kF8) {
-          tma_load_3d(smem_u32(sQ + q * L::kQKBytes), &tmap_q, bar_q_full, 0, (q0 + q) * kBlockM, bh);
+          tma_load_3d(smem_u32(sQ + q * L::kQKBytes), &tmap_q, bar_q_full, 0, qrow, bh);
         } else {
           for (int c = 0; c < D / 64; ++c)
-            tma_load_3d(smem_u32(sQ + q * L::kQKBytes + c * kChunkBytes), &tmap_q, bar_q_full, c * 64,
-                        (q0 + q) * kBlockM, bh);
+            tma_load_3d(smem_u32(sQ + q * L::kQKBytes + c * kChunkBytes), &tmap_q, bar_q_full, c * 64, qrow, bh);
         }
       }
       if (p.trace) p.trace[static_cast<size_t>(cta) * (p.Tc + 1)] = tl.len;
@@ -363,7 +401,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto issue_s = [&](int q, int n) {
         const int s = n % S;
         const uint32_t d_tmem = tmem + q * 128;
-        const uint64_t bq = sdesc_add(dQ, static_cast<uint32_t>(q) * L::kQKBytes);
+        const uint64_t bq = sdesc_add(dQ, static_cast<uint32_t>(dual && !shift1 ? 0 : q) * L::kQKBytes);
         const uint64_t bk = sdesc_add(dK, static_cast<uint32_t>(s) * L::kQKBytes);
         if constexpr (kF8) {
           // e4m3: K = 32 per MMA, 32 bytes along the 128-byte swizzled rows.
@@ -410,6 +448,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t fn = has_next ? (tl.entry(n + 1) >> 16) : 0u;
         if (has_next) {
           if (!(ok = mbar_wait(bar_k_full((n + 1) % S), ((n + 1) / S) & 1, ctx))) break;
+          // A slot the next tile uses but this one does not gets its S first: its
+          // S/P columns were last read by a P V issued in an earlier step, so its
+          // softmax can run while this step waits for V and the other slot's P.
+          if (fn & ~f) {
+            tc_fence_after();
+            for (int q = 0; q < 2; ++q)
+              if ((fn & ~f) & (1u << q)) issue_s(q, n + 1);
+          }
         }
         if (!(ok = mbar_wait(bar_v_full(n % S), (n / S) & 1, ctx))) break;
         tc_fence_after();
@@ -419,8 +465,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             ++p_count[q];
             tc_fence_after();
             issue_pv(q, n);
+            if (fn & (1u << q)) issue_s(q, n + 1);
           }
-          if (fn & (1u << q)) issue_s(q, n + 1);
         }
         if (!ok) break;
         umma_commit(bar_v_empty(n % S));
@@ -484,9 +530,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ softmax
     const int q = (warp - 4) / 4;  // query tile within the pair
     const int wq = warp % 4;       // TMEM lane quarter
-    const int qt = q0 + q;
+    const int qt = q0 + (dual ? 0 : q);
     const int row_local = wq * 32 + lane;
-    const int row = qt * kBlockM + row_local;
+    const int row = qt * kBlockM + row_local - (q == 1 ? shift1 : 0);  // query row of this TMEM lane
+    // A warp whose 32 rows are all outside [0, N) (padding of a short last tile, or
+    // the shifted slot) keeps the barrier protocol but skips the arithmetic: rows
+    // of P V are independent, and such rows are never stored.
+    const int warp_row0 = row - lane;
+    const bool warp_rows = warp_row0 + 31 >= 0 && warp_row0 < p.N;
     const bool tile_active = (q == 0) || q1_active;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t t_s = tmem + lane_off + q * 128;
@@ -505,6 +556,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int j = static_cast<int>(e & 0xFFFFu);
         if (!(ok = mbar_wait_warp(bar_s_full(q), count & 1, ctx))) break;
         tc_fence_after();
+        if (!warp_rows) {
+          tc_fence_before();
+          mbar_arrive(bar_p_full(q));
+          ++count;
+          continue;
+        }
         uint32_t sr[128];
         tmem_ld32(t_s + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
         tmem_ld32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
@@ -617,12 +674,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       const size_t row_base = static_cast<size_t>(bh) * p.N;
-      const bool row_valid = row < p.N;
+      const bool row_valid = row >= 0 && row < p.N;
       const float inv_l = (l_sum > 0.0f) ? (kF8 ? p.v_scale : 1.0f) / l_sum : 0.0f;
       if (kSplit && ok) {
         // Split-KV partial: fp32 O / l of this key range (0 if it has no key for
         // the row) and its lse (-inf then), stored straight from the row's thread.
-        const size_t prow = (static_cast<size_t>(split) * p.BH + bh) * p.N + row;
+        const size_t prow = (static_cast<size_t>(split + (dual ? q : 0)) * p.BH + bh) * p.N + row;
 #pragma unroll
         for (int c = 0; c < D; c += 32) {
           uint32_t o[32];

@@ -67,6 +67,8 @@ def _run(B, H, Nq, Nk, d, fmt, causal, n_splits=None, mask=None, seed=0):
     (1, 2, 5, 777, 128, "bf16", False, 7),        # one 128-key tile per range, ragged last tile
     (1, 1, 1, 1, 64, "bf16", False, 1),
     (1, 2, 3, 2000, 256, "bf16", True, 6),       # head dimension 256 (forward only)
+    (2, 3, 7, 5000, 64, "fp16", True, 9),         # one query tile, odd range count: a CTA with one range
+    (1, 2, 100, 1000, 128, "bf16", True, 8),      # causal: ranges past a row's reach are empty
 ])
 def test_splitkv_matches_oracle(B, H, Nq, Nk, d, fmt, causal, n_splits):
     _run(B, H, Nq, Nk, d, fmt, causal, n_splits)
@@ -92,7 +94,11 @@ def test_splitkv_agrees_with_unsplit_forward():
 
 
 def test_suggested_splits_fill_the_gpu():
+    # One query tile: a CTA takes two consecutive ranges, so B*H*ceil(n/2) CTAs.
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     ns = fa.fa_fwd_splitkv_splits(1, 16, 1, 65536)
-    assert 1 <= ns <= 512 and 16 * ns <= sms and 16 * (ns + 1) > sms
+    ctas = 16 * ((ns + 1) // 2)
+    assert 2 <= ns <= 512 and ctas <= sms and ctas + 16 > sms
     assert fa.fa_fwd_splitkv_splits(8, 64, 4096, 4096) == 1
+    ns2 = fa.fa_fwd_splitkv_splits(1, 4, 256, 65536)  # two query tiles: a CTA per range
+    assert 4 * ns2 <= sms < 4 * (ns2 + 1)
