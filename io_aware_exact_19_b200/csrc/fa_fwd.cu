@@ -60,11 +60,12 @@ int launch_fwd_t(const AttnArgs& a, cudaStream_t stream) {
   auto kern = p.o_part != nullptr ? fwd::fa_fwd_kernel<D, BF16, fwd::kSplitKV>
               : a.drop_t > 0      ? fwd::fa_fwd_kernel<D, BF16, kDropMode>
                                   : fwd::fa_fwd_kernel<D, BF16, fwd::kPlain>;
-  cudaError_t e = host::ensure_dynamic_smem(reinterpret_cast<const void*>(kern), L::kAlloc);
+  const int smem_bytes = p.o_part != nullptr ? fwd::Smem<D, false, true>::kAlloc : L::kAlloc;
+  cudaError_t e = host::ensure_dynamic_smem(reinterpret_cast<const void*>(kern), smem_bytes);
   if (e != cudaSuccess) return static_cast<int>(e);
   const int split_items = p.dual ? (p.n_splits + 1) / 2 : p.n_splits;
   dim3 grid(static_cast<unsigned>(static_cast<long long>(BH) * p.n_pairs * split_items));
-  kern<<<grid, fwd::kThreads, L::kAlloc, stream>>>(tq, tk, tv, to, p);
+  kern<<<grid, fwd::kThreads, smem_bytes, stream>>>(tq, tk, tv, to, p);
   return static_cast<int>(cudaGetLastError());
 }
 

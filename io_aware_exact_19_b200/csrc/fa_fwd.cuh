@@ -89,10 +89,11 @@ struct Params {
 // widened to 16 bits into the V ring. The V ring follows the K ring, so the
 // epilogue's staging (64 KB at d = 128, from the K ring on) stays inside both.
 // D = 256: one query tile per CTA (S 128 + O 256 TMEM columns) and single K and
-// V stages (64 KB tiles).
-template <int D, bool kF8 = false>
+// V stages (64 KB tiles). kDeep (split-KV at D = 64, i.e. decoding, which streams
+// K and V from HBM once): five stages, so more bytes are in flight per SM.
+template <int D, bool kF8 = false, bool kDeep = false>
 struct Smem {
-  static constexpr int kStages = D == 256 ? 1 : (D == 128 ? 2 : 3);
+  static constexpr int kStages = D == 256 ? 1 : (D == 128 ? 2 : (kDeep ? 5 : 3));
   static constexpr int kQTiles = D == 256 ? 1 : 2;  // query tiles per CTA
   static constexpr int kTileBytes = kBlockN * D * 2;           // one 16-bit V tile
   static constexpr int kQKBytes = kF8 ? kBlockN * D : kTileBytes;  // one Q or K tile
@@ -165,7 +166,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                   const __grid_constant__ CUtensorMap tmap_v, const __grid_constant__ CUtensorMap tmap_o,
                   const Params p) {
   constexpr bool kF8 = kMode == kFp8;
-  using L = Smem<D, kF8>;
+  using L = Smem<D, kF8, kMode == kSplitKV>;
   constexpr int S = L::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
