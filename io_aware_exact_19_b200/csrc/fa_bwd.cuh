@@ -473,11 +473,27 @@ __device__ __forceinline__ void key_cta(const Ctx& c, const Params& p, const CUt
     const bool key_valid = key < p.Nk;
     const uint32_t tl = c.tmem + (static_cast<uint32_t>(wq * 32) << 16);
     const float sl2 = p.scale_log2;
+    const uint32_t drop_c7 = philox::keep_bias(p.drop_t);
     const int qo = 64 * h;
     bool ok = true;
     for (int n = 0; n < len; ++n) {
       const int i = cur.next();
       const int s = n % S;
+      // Dropout: keep flags of this key against query rows i*128 + qo .. +63
+      // (group g: rows 4g .. 4g + 3), drawn while S^T is computed.
+      uint32_t kb[kDropout ? 2 : 1] = {};
+      if constexpr (kDropout) {
+        const uint32_t rg_first = static_cast<uint32_t>(i * kBR + qo) / 4;
+#pragma unroll
+        for (int g = 0; g < 16; g += 4) {
+          const uint4 w = philox::draws_col(rg_first + g, static_cast<uint32_t>(key), static_cast<uint32_t>(c.bh),
+                                            p.seed_lo, p.seed_hi);
+          philox::add_keep_flags(kb, g, w.x, drop_c7);
+          philox::add_keep_flags(kb, g + 1, w.y, drop_c7);
+          philox::add_keep_flags(kb, g + 2, w.z, drop_c7);
+          philox::add_keep_flags(kb, g + 3, w.w, drop_c7);
+        }
+      }
       if (!(ok = mbar_wait_warp(c.bar(B::s_full), n & 1, c.wait))) break;
       tc_fence_after();
       uint32_t sr[64];
@@ -510,23 +526,6 @@ __device__ __forceinline__ void key_cta(const Ctx& c, const Params& p, const CUt
         for (int x = 0; x < 64; ++x)
           if (x < lim) pv[x] = 0.0f;
       }
-      // Dropout: keep decisions of this key against query rows i*128 + qo .. +63
-      // (bit x), drawn while the dP^T MMA runs.
-      uint64_t keep = ~0ull;
-      if constexpr (kDropout) {
-        keep = 0;
-        const uint32_t rg_first = static_cast<uint32_t>(i * kBR + qo) / 4;
-#pragma unroll
-        for (int g = 0; g < 16; g += 4) {
-          const uint4 w = philox::draws_col(rg_first + g, static_cast<uint32_t>(key), static_cast<uint32_t>(c.bh),
-                                            p.seed_lo, p.seed_hi);
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-#pragma unroll
-            for (int b = 0; b < 4; ++b)
-              if (philox::draw_byte(w, k, b) >= p.drop_t) keep |= 1ull << (4 * (g + k) + b);
-        }
-      }
       if (!(ok = mbar_wait_warp(c.bar(B::dp_full), n & 1, c.wait))) break;
       tc_fence_after();
       uint32_t dr[64];
@@ -536,15 +535,21 @@ __device__ __forceinline__ void key_cta(const Ctx& c, const Params& p, const CUt
       const uint32_t aD = smem_u32(sDv + s * kBR + qo);
       uint32_t pk[32], dk[32];
       if constexpr (kDropout) {
-        // dV takes (P o Z)^T, dS^T = P^T o (dP^T o Z - D), Z = keep * drop_scale.
-        const float zs = p.drop_scale;
+        // dV takes (P o M)^T (the factor 256 / (256 - t) of Z = M * 256 / (256 - t)
+        // is applied in the dV epilogue); dS^T = P^T o (dP^T o Z - D).
+        const uint32_t zs = __float_as_uint(p.drop_scale);
 #pragma unroll
         for (int x = 0; x < 64; x += 4) {
           const float4 d4 = lds128(aD + x * 4);
-          const float z0 = (keep >> x) & 1 ? zs : 0.0f, z1 = (keep >> (x + 1)) & 1 ? zs : 0.0f;
-          const float z2 = (keep >> (x + 2)) & 1 ? zs : 0.0f, z3 = (keep >> (x + 3)) & 1 ? zs : 0.0f;
-          pk[x / 2] = pack2<BF16>(pv[x] * z0, pv[x + 1] * z1);
-          pk[x / 2 + 1] = pack2<BF16>(pv[x + 2] * z2, pv[x + 3] * z3);
+          const uint32_t f = philox::group_flags(kb, x / 4);
+          uint32_t m01, m23;
+          philox::pair_masks(f, m01, m23);
+          const float z0 = __uint_as_float(philox::elem_mask<0>(f) & zs);
+          const float z1 = __uint_as_float(philox::elem_mask<1>(f) & zs);
+          const float z2 = __uint_as_float(philox::elem_mask<2>(f) & zs);
+          const float z3 = __uint_as_float(philox::elem_mask<3>(f) & zs);
+          pk[x / 2] = pack2<BF16>(pv[x], pv[x + 1]) & m01;
+          pk[x / 2 + 1] = pack2<BF16>(pv[x + 2], pv[x + 3]) & m23;
           dk[x / 2] = pack2<BF16>(pv[x] * fmaf(__uint_as_float(dr[x]), z0, -d4.x),
                                   pv[x + 1] * fmaf(__uint_as_float(dr[x + 1]), z1, -d4.y));
           dk[x / 2 + 1] = pack2<BF16>(pv[x + 2] * fmaf(__uint_as_float(dr[x + 2]), z2, -d4.z),
@@ -578,7 +583,8 @@ __device__ __forceinline__ void key_cta(const Ctx& c, const Params& p, const CUt
     tc_fence_after();
     if (ok) {
       const uint32_t stage = smem_u32(sQ) + static_cast<uint32_t>(c.warp - 4) * (32 * D * 2);
-      store_rows_tma<BF16, D>(tl + 256 + h * D, h == 0 ? 1.0f : p.scale, have, stage, h == 0 ? tdv : tdk, 0,
+      const float dv_scale = kDropout ? p.drop_scale : 1.0f;
+      store_rows_tma<BF16, D>(tl + 256 + h * D, h == 0 ? dv_scale : p.scale, have, stage, h == 0 ? tdv : tdk, 0,
                               j * kBlockN + wq * 32, c.bh, p.Nk, p.d);
     }
     if (c.lane == 0) bulk_wait_group_read<0>();  // shared memory read; the writes complete on their own
@@ -727,6 +733,7 @@ __device__ __forceinline__ void query_cta(const Ctx& c, const Params& p, const C
     const bool row_valid = qrow < p.N;
     const uint32_t tl = c.tmem + (static_cast<uint32_t>(wq * 32) << 16);
     const float sl2 = p.scale_log2;
+    const uint32_t drop_c7 = philox::keep_bias(p.drop_t);
     const size_t vo = static_cast<size_t>(c.bh) * p.Npad + static_cast<size_t>(i) * kBlockQ + r;
     const float l2 = p.lse2[vo];  // +inf on padding rows: P = 0
     const float dd = p.delta[vo];
@@ -780,6 +787,21 @@ __device__ __forceinline__ void query_cta(const Ctx& c, const Params& p, const C
     bool ok = true;
     for (int n = 0; n < len; ++n) {
       const int jt = cur.next();
+      // Dropout: keep flags of this query row against keys jt*128 + 64h .. +63
+      // (group g: keys 4g .. 4g + 3), drawn while S is computed.
+      uint32_t kb[kDropout ? 2 : 1] = {};
+      if constexpr (kDropout) {
+        const uint32_t cg_first = static_cast<uint32_t>(jt * kBlockN + 64 * h) / 4;
+#pragma unroll
+        for (int g = 0; g < 16; g += 4) {
+          const uint4 w = philox::draws_row(cg_first + g, static_cast<uint32_t>(qrow), static_cast<uint32_t>(c.bh),
+                                            p.seed_lo, p.seed_hi);
+          philox::add_keep_flags(kb, g, w.x, drop_c7);
+          philox::add_keep_flags(kb, g + 1, w.y, drop_c7);
+          philox::add_keep_flags(kb, g + 2, w.z, drop_c7);
+          philox::add_keep_flags(kb, g + 3, w.w, drop_c7);
+        }
+      }
       if (!(ok = mbar_wait_warp(c.bar(B::s_full), n & 1, c.wait))) break;
       tc_fence_after();
       uint32_t sr[64];
@@ -801,23 +823,6 @@ __device__ __forceinline__ void query_cta(const Ctx& c, const Params& p, const C
         for (int x = 0; x < 64; ++x)
           if (x > lim) pv[x] = 0.0f;
       }
-      // Dropout: keep decisions of this query row against keys jt*128 + 64h .. +63
-      // (bit x), drawn while the dP MMA runs.
-      uint64_t keep = ~0ull;
-      if constexpr (kDropout) {
-        keep = 0;
-        const uint32_t cg_first = static_cast<uint32_t>(jt * kBlockN + 64 * h) / 4;
-#pragma unroll
-        for (int g = 0; g < 16; g += 4) {
-          const uint4 w = philox::draws_row(cg_first + g, static_cast<uint32_t>(qrow), static_cast<uint32_t>(c.bh),
-                                            p.seed_lo, p.seed_hi);
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-#pragma unroll
-            for (int b = 0; b < 4; ++b)
-              if (philox::draw_byte(w, k, b) >= p.drop_t) keep |= 1ull << (4 * (g + k) + b);
-        }
-      }
       if (!(ok = mbar_wait_warp(c.bar(B::dp_full), n & 1, c.wait))) break;  // dP_n
       tc_fence_after();
       uint32_t dr[64];
@@ -826,13 +831,19 @@ __device__ __forceinline__ void query_cta(const Ctx& c, const Params& p, const C
       tmem_ld_wait();
       uint32_t dk[32];
       if constexpr (kDropout) {
-        // dS = P o (dP o Z - D), Z = keep * drop_scale.
-        const float zs = p.drop_scale;
+        // dS = P o (dP o Z - D), Z = M * drop_scale.
+        const uint32_t zs = __float_as_uint(p.drop_scale);
 #pragma unroll
-        for (int x = 0; x < 32; ++x) {
-          const float z0 = (keep >> (2 * x)) & 1 ? zs : 0.0f, z1 = (keep >> (2 * x + 1)) & 1 ? zs : 0.0f;
-          dk[x] = pack2<BF16>(pv[2 * x] * fmaf(__uint_as_float(dr[2 * x]), z0, -dd),
-                              pv[2 * x + 1] * fmaf(__uint_as_float(dr[2 * x + 1]), z1, -dd));
+        for (int x = 0; x < 64; x += 4) {
+          const uint32_t f = philox::group_flags(kb, x / 4);
+          const float z0 = __uint_as_float(philox::elem_mask<0>(f) & zs);
+          const float z1 = __uint_as_float(philox::elem_mask<1>(f) & zs);
+          const float z2 = __uint_as_float(philox::elem_mask<2>(f) & zs);
+          const float z3 = __uint_as_float(philox::elem_mask<3>(f) & zs);
+          dk[x / 2] = pack2<BF16>(pv[x] * fmaf(__uint_as_float(dr[x]), z0, -dd),
+                                  pv[x + 1] * fmaf(__uint_as_float(dr[x + 1]), z1, -dd));
+          dk[x / 2 + 1] = pack2<BF16>(pv[x + 2] * fmaf(__uint_as_float(dr[x + 2]), z2, -dd),
+                                      pv[x + 3] * fmaf(__uint_as_float(dr[x + 3]), z3, -dd));
         }
       } else {
 #pragma unroll

@@ -544,6 +544,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t t_s = tmem + lane_off + q * 128;
     const uint32_t t_o = tmem + lane_off + 256 + q * D;
     const float sl2 = p.scale_log2;
+    const uint32_t drop_c7 = philox::keep_bias(p.drop_t);
 
     float m_ref = -INFINITY;  // log2-domain reference max
     float l_sum = 0.0f;
@@ -555,6 +556,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t e = tl.entry(n);
         if (!((e >> 16) & (1u << q))) continue;
         const int j = static_cast<int>(e & 0xFFFFu);
+        // Dropout keep decisions of this row's 128 keys, 16 draws per generator
+        // block, made while S is still being computed. Key group w (keys 4w ..
+        // 4w + 3) is bit 7 - w % 8 of the bytes of word w / 8, byte k for key 4w + k.
+        uint32_t kb[kMode == kDropout ? 4 : 1] = {};
+        if constexpr (kMode == kDropout) {
+          if (warp_rows) {
+            const uint32_t cg_tile = static_cast<uint32_t>(j) * (kBlockN / 4);
+#pragma unroll
+            for (int g = 0; g < kBlockN / 4; g += 4) {
+              const uint4 w = philox::draws_row(cg_tile + g, static_cast<uint32_t>(row), static_cast<uint32_t>(bh),
+                                                p.seed_lo, p.seed_hi);
+              philox::add_keep_flags(kb, g, w.x, drop_c7);
+              philox::add_keep_flags(kb, g + 1, w.y, drop_c7);
+              philox::add_keep_flags(kb, g + 2, w.z, drop_c7);
+              philox::add_keep_flags(kb, g + 3, w.w, drop_c7);
+            }
+          }
+        }
         if (!(ok = mbar_wait_warp(bar_s_full(q), count & 1, ctx))) break;
         tc_fence_after();
         if (!warp_rows) {
@@ -630,27 +649,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         l_sum += (ls0 + ls1) + (ls2 + ls3);
 
-        if constexpr (kMode == kDropout) {
-          // P V uses P o Z: the dropout keep decisions of this row's 128 keys, 16
-          // per generator block (the sum l above is of the undropped P).
-          const uint32_t cg_tile = static_cast<uint32_t>(j) * (kBlockN / 4);
-#pragma unroll
-          for (int g = 0; g < kBlockN / 4; g += 4) {
-            const uint4 w = philox::draws_row(cg_tile + g, static_cast<uint32_t>(row), static_cast<uint32_t>(bh),
-                                              p.seed_lo, p.seed_hi);
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-#pragma unroll
-              for (int b = 0; b < 4; ++b) {
-                const int c = 4 * (g + k) + b;
-                s[c] = philox::draw_byte(w, k, b) >= p.drop_t ? s[c] * p.drop_scale : 0.0f;
-              }
-          }
-        }
-
         uint32_t pk[64];
 #pragma unroll
         for (int i = 0; i < 64; ++i) pk[i] = pack2<BF16>(s[2 * i], s[2 * i + 1]);
+        if constexpr (kMode == kDropout) {
+          // P V uses P o M, M the keep decisions (the sum l above is of the
+          // undropped P); the factor 256 / (256 - t) of Z = M * 256 / (256 - t) is
+          // applied with 1 / l in the epilogue.
+#pragma unroll
+          for (int w = 0; w < kBlockN / 4; ++w) {
+            uint32_t m01, m23;
+            philox::pair_masks(philox::group_flags(kb, w), m01, m23);
+            pk[2 * w] &= m01;
+            pk[2 * w + 1] &= m23;
+          }
+        }
         tmem_st32(t_s + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
         tmem_st32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
         tmem_st_wait();
@@ -676,7 +689,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const size_t row_base = static_cast<size_t>(bh) * p.N;
       const bool row_valid = row >= 0 && row < p.N;
-      const float inv_l = (l_sum > 0.0f) ? (kF8 ? p.v_scale : 1.0f) / l_sum : 0.0f;
+      const float o_scale = kF8 ? p.v_scale : (kMode == kDropout ? p.drop_scale : 1.0f);
+      const float inv_l = (l_sum > 0.0f) ? o_scale / l_sum : 0.0f;
       if (kSplit && ok) {
         // Split-KV partial: fp32 O / l of this key range (0 if it has no key for
         // the row) and its lse (-inf then), stored straight from the row's thread.

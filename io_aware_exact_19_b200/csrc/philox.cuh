@@ -103,6 +103,52 @@ __device__ __forceinline__ uint4 draws_col(uint32_t rg0, uint32_t key, uint32_t 
   return exchange4(tr);
 }
 
+// Keep decisions of four draws (bytes 0..3 of x, four consecutive keys of a row):
+// byte k of the result is 0xFF where draw k >= t (kept) and 0 where it is below
+// (dropped). c7 = keep_bias(t).
+//
+// Byte u >= t exactly when u + 256 - t reaches 256: the even bytes, then the odd
+// ones, are spread to the top of 16-bit lanes (u << 7) and added to (256 - t) << 7,
+// which sets bit 15 of the lane exactly for kept bytes (no carry crosses a lane:
+// u + 256 - t < 512). prmt's sign-replicating selectors (nibble 8 | i: the sign
+// bit of input byte i over the whole result byte) gather the four bits.
+__host__ __device__ __forceinline__ uint32_t keep_bias(uint32_t t) { return ((256u - t) << 7) * 0x10001u; }
+
+__device__ __forceinline__ uint32_t keep_bytes(uint32_t x, uint32_t c7) {
+  const uint32_t even = ((x & 0x00FF00FFu) << 7) + c7;  // keys 0, 2 -> bits 15, 31
+  const uint32_t odd = ((x >> 1) & 0x7F807F80u) + c7;   // keys 1, 3 -> bits 15, 31
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, 0xFBD9;" : "=r"(r) : "r"(even), "r"(odd));
+  return r;
+}
+
+// Keep flags of a row (or key) against 4G consecutive keys (or rows), G groups of
+// four: group g is bit 7 - g % 8 of the four bytes of word g / 8, byte k for its
+// element k. add_keep_flags puts the flags of group g, from its draws word x, in.
+__device__ __forceinline__ void add_keep_flags(uint32_t* kb, int g, uint32_t x, uint32_t c7) {
+  kb[g / 8] |= keep_bytes(x, c7) & (0x80808080u >> (g % 8));
+}
+
+// Group g's flags with the bit of each byte moved to its top.
+__device__ __forceinline__ uint32_t group_flags(const uint32_t* kb, int g) { return kb[g / 8] << (g % 8); }
+
+// All ones where element b of a group is kept, zero where it is dropped (flags
+// from group_flags).
+template <int b>
+__device__ __forceinline__ uint32_t elem_mask(uint32_t flags) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %1, %2;" : "=r"(r) : "r"(flags), "n"((8 | b) * 0x1111));
+  return r;
+}
+
+// Masks for two packed 16-bit pairs from a word whose byte k has keep(key k) in
+// its top bit: m01 covers keys 0 and 1, m23 keys 2 and 3; each half is 0xFFFF for
+// a kept key and 0 for a dropped one, so a pair is dropped with one AND.
+__device__ __forceinline__ void pair_masks(uint32_t flags, uint32_t& m01, uint32_t& m23) {
+  asm("prmt.b32 %0, %1, %1, 0x9988;" : "=r"(m01) : "r"(flags));
+  asm("prmt.b32 %0, %1, %1, 0xBBAA;" : "=r"(m23) : "r"(flags));
+}
+
 // Byte b of word k of a draws_* result.
 __device__ __forceinline__ uint32_t draw_byte(const uint4& w, int k, int b) {
   const uint32_t x = k == 0 ? w.x : (k == 1 ? w.y : (k == 2 ? w.z : w.w));

@@ -115,3 +115,102 @@ def test_zero_probability_is_the_plain_kernel_and_seeds_matter():
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
     assert torch.equal(o3, o4) and torch.equal(l3, l4)
     assert not torch.equal(o3, o5) and torch.equal(l3, l5)
+
+
+@pytest.mark.parametrize("d,p", [(128, 0.1), (128, 0.5), (64, 0.998), (64, 0.3)])
+def test_keep_decisions_across_key_tiles(d, p):
+    # Q = 0 makes P uniform (every exponential is 1, l = Nk); V[j] = 2^(j // d) e_(j % d)
+    # sums the keep decisions of keys c, c + d, c + 2d, c + 3d of a row into one integer
+    # O[i, c] * Nk / Z_kept, so every decision of four key groups is checked exactly,
+    # at thresholds t = 26, 128, 255 and 77.
+    B, H, Nq, Nk, seed = 1, 2, 256, 4 * d, 0x5EED0FD40F
+    c = Case(B, H, Nk, d, "bf16", seed=21)
+    q = torch.zeros((B, H, Nq, d), dtype=torch.bfloat16, device="cuda")
+    j = np.arange(Nk)
+    vals = np.zeros((Nk, d), dtype=np.float32)
+    vals[j, j % d] = 2.0 ** (j // d)
+    v = torch.from_numpy(vals).to(torch.bfloat16).cuda().expand(B, H, Nk, d).contiguous()
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, Nq), dtype=torch.float32, device="cuda")
+    fa.fa_fwd_dropout(q, c.dev["k"], v, o, lse, p, seed)
+    torch.cuda.synchronize()
+    assert fa.fa_device_status() == fa.FA_OK
+    t = Dr.drop_threshold(p)
+    z_kept = 256.0 / (256 - t)
+    for bh in range(B * H):
+        kept = (Dr.keep_scale(Nq, Nk, bh, seed, p) > 0).astype(np.int64)      # [Nq, Nk]
+        expect = sum(kept[:, g * d:(g + 1) * d] << g for g in range(4))      # [Nq, d]
+        got = o.reshape(B * H, Nq, d)[bh].float().cpu().numpy() * Nk / z_kept
+        assert np.array_equal(np.rint(got).astype(np.int64), expect), f"head {bh}"
+        assert float(np.abs(got - np.rint(got)).max()) < 0.05
+
+
+def _one_hot_powers(n, d):
+    """[n, d]: row r is 2^(r // d) at column r % d (n = 4d rows: four groups)."""
+    r = np.arange(n)
+    x = np.zeros((n, d), dtype=np.float32)
+    x[r, r % d] = 2.0 ** (r // d)
+    return x
+
+
+@pytest.mark.parametrize("grad,d,p", [("dv", 128, 0.1), ("dv", 64, 0.998), ("dq", 128, 0.5), ("dq", 64, 0.3),
+                                      ("dk", 128, 0.25), ("dk", 64, 0.7)])
+def test_backward_keep_decisions_exact(grad, d, p):
+    # S = Q K^T = 0 (Q = 0, or K = 0 for dK) makes P = 1/Nk exactly. Then, with one-hot
+    # powers of two, each gradient element is an integer combination of the keep
+    # decisions of four rows (or keys), decoded exactly:
+    #   dv: dO[i] = 2^(i//d) e_(i%d)            -> dV[j, c] Nk / zq = sum_g M[gd+c, j] 2^g
+    #   dq: K[j] likewise, V[j] = dO[i] = e_0    -> dS = (Z - D_i) / Nk,
+    #       (dQ[i, c] Nk / scale + 15 D_i) / zq  = sum_g M[i, gd+c] 2^g
+    #   dk: Q[i] likewise, K = 0, V = dO = e_0   -> (dK[j, c] Nk / scale + sum_g 2^g D_(gd+c)) / zq
+    #                                             = sum_g M[gd+c, j] 2^g
+    # with zq = 256 / (256 - t) and D_i = O[i, 0] (the 16-bit O the prep reads).
+    B, H, seed = 1, 2, 0xD0D0CAFE
+    Nq, Nk = (4 * d, 256) if grad in ("dv", "dk") else (256, 4 * d)
+    dev = dict(dtype=torch.bfloat16, device="cuda")
+    rnd = Case(B, H, max(Nq, Nk), d, "bf16", seed=31)
+    e0 = torch.zeros(d, **dev)
+    e0[0] = 1
+    powers_q = torch.from_numpy(_one_hot_powers(Nq, d)).to(**dev).expand(B, H, Nq, d).contiguous()
+    powers_k = torch.from_numpy(_one_hot_powers(Nk, d)).to(**dev).expand(B, H, Nk, d).contiguous()
+    if grad == "dv":
+        q = torch.zeros((B, H, Nq, d), **dev)
+        k = rnd.dev["k"][:, :, :Nk].contiguous()
+        v = rnd.dev["v"][:, :, :Nk].contiguous()
+        do = powers_q
+    elif grad == "dq":
+        q = torch.zeros((B, H, Nq, d), **dev)
+        k = powers_k
+        v = e0.expand(B, H, Nk, d).contiguous()
+        do = e0.expand(B, H, Nq, d).contiguous()
+    else:
+        q = powers_q
+        k = torch.zeros((B, H, Nk, d), **dev)
+        v = e0.expand(B, H, Nk, d).contiguous()
+        do = e0.expand(B, H, Nq, d).contiguous()
+    scale = 1.0 / np.sqrt(d)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, Nq), dtype=torch.float32, device="cuda")
+    fa.fa_fwd_dropout(q, k, v, o, lse, p, seed, scale=scale)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(fa.fa_bwd_workspace_size(B, H, Nq, d), dtype=torch.uint8, device="cuda")
+    fa.fa_bwd_dropout(q, k, v, o, lse, do, dq, dk, dv, ws, p, seed, scale=scale)
+    torch.cuda.synchronize()
+    assert fa.fa_device_status() == fa.FA_OK
+    zq = 256.0 / (256 - Dr.drop_threshold(p))
+    w = 2 ** np.arange(4)
+    for bh in range(B * H):
+        kept = (Dr.keep_scale(Nq, Nk, bh, seed, p) > 0).astype(np.int64)          # [Nq, Nk]
+        D = o.reshape(B * H, Nq, d)[bh, :, 0].float().cpu().numpy().astype(np.float64)
+        if grad == "dv":
+            got = dv.reshape(B * H, Nk, d)[bh].double().cpu().numpy() * Nk / zq
+            expect = sum(kept[g * d:(g + 1) * d, :].T << g for g in range(4))     # [Nk, d]
+        elif grad == "dq":
+            got = (dq.reshape(B * H, Nq, d)[bh].double().cpu().numpy() * Nk / scale + 15 * D[:, None]) / zq
+            expect = sum(kept[:, g * d:(g + 1) * d] << g for g in range(4))      # [Nq, d]
+        else:
+            dsum = (D.reshape(4, d) * w[:, None]).sum(axis=0)                     # [d]
+            got = (dk.reshape(B * H, Nk, d)[bh].double().cpu().numpy() * Nk / scale + dsum[None, :]) / zq
+            expect = sum(kept[g * d:(g + 1) * d, :].T << g for g in range(4))     # [Nk, d]
+        assert float(np.abs(got - np.rint(got)).max()) < 0.25, f"{grad} head {bh}: not near integers"
+        assert np.array_equal(np.rint(got).astype(np.int64), expect), f"{grad} head {bh}"
