@@ -46,8 +46,7 @@ int launch_bwd_t(const AttnArgs& a, cudaStream_t stream) {
   p.withhold = a.withhold;
   p.drop_t = static_cast<uint32_t>(a.drop_t);
   p.drop_scale = 256.0f / static_cast<float>(256 - a.drop_t);
-  p.seed_lo = static_cast<uint32_t>(a.drop_seed);
-  p.seed_hi = static_cast<uint32_t>(a.drop_seed >> 32);
+  p.drop_keys = philox::round_keys(a.drop_seed);
   const int Nk = a.Nk > 0 ? a.Nk : a.N;
   p.N = a.N;
   p.Nk = Nk;

@@ -181,7 +181,7 @@ struct Params {
   // draw is below drop_t; kept ones are scaled by drop_scale = 256 / (256 - drop_t).
   uint32_t drop_t;
   float drop_scale;
-  uint32_t seed_lo, seed_hi;
+  philox::Keys drop_keys;  // round keys of the dropout seed
   int N;     // query rows
   int Nk;    // key / value rows
   int d;     // head dimension of the tensors (<= D; columns d..D-1 are zero in the kernel)
@@ -487,7 +487,7 @@ __device__ __forceinline__ void key_cta(const Ctx& c, const Params& p, const CUt
 #pragma unroll
         for (int g = 0; g < 16; g += 4) {
           const uint4 w = philox::draws_col(rg_first + g, static_cast<uint32_t>(key), static_cast<uint32_t>(c.bh),
-                                            p.seed_lo, p.seed_hi);
+                                            p.drop_keys);
           philox::add_keep_flags(kb, g, w.x, drop_c7);
           philox::add_keep_flags(kb, g + 1, w.y, drop_c7);
           philox::add_keep_flags(kb, g + 2, w.z, drop_c7);
@@ -795,7 +795,7 @@ __device__ __forceinline__ void query_cta(const Ctx& c, const Params& p, const C
 #pragma unroll
         for (int g = 0; g < 16; g += 4) {
           const uint4 w = philox::draws_row(cg_first + g, static_cast<uint32_t>(qrow), static_cast<uint32_t>(c.bh),
-                                            p.seed_lo, p.seed_hi);
+                                            p.drop_keys);
           philox::add_keep_flags(kb, g, w.x, drop_c7);
           philox::add_keep_flags(kb, g + 1, w.y, drop_c7);
           philox::add_keep_flags(kb, g + 2, w.z, drop_c7);

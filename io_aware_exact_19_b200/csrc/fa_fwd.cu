@@ -52,8 +52,7 @@ int launch_fwd_t(const AttnArgs& a, cudaStream_t stream) {
   p.scale_log2 = a.scale * 1.4426950408889634f;
   p.drop_t = static_cast<uint32_t>(a.drop_t);
   p.drop_scale = 256.0f / static_cast<float>(256 - a.drop_t);
-  p.seed_lo = static_cast<uint32_t>(a.drop_seed);
-  p.seed_hi = static_cast<uint32_t>(a.drop_seed >> 32);
+  p.drop_keys = philox::round_keys(a.drop_seed);
   // d = 256 (a forward-only head dimension) has the plain and split-KV variants.
   constexpr int kDropMode = D == 256 ? fwd::kPlain : fwd::kDropout;
   if (D == 256 && a.drop_t > 0) return static_cast<int>(cudaErrorInvalidValue);

@@ -74,7 +74,7 @@ struct Params {
   // drop_t; kept ones are scaled by drop_scale = 256 / (256 - drop_t).
   uint32_t drop_t;
   float drop_scale;
-  uint32_t seed_lo, seed_hi;
+  philox::Keys drop_keys;  // round keys of the dropout seed
   float v_scale;  // kFp8: per-tensor scale of V (those of Q and K are in scale_log2)
   int BH;
   int n_pairs;  // ceil(T_q / 2)
@@ -566,7 +566,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int g = 0; g < kBlockN / 4; g += 4) {
               const uint4 w = philox::draws_row(cg_tile + g, static_cast<uint32_t>(row), static_cast<uint32_t>(bh),
-                                                p.seed_lo, p.seed_hi);
+                                                p.drop_keys);
               philox::add_keep_flags(kb, g, w.x, drop_c7);
               philox::add_keep_flags(kb, g + 1, w.y, drop_c7);
               philox::add_keep_flags(kb, g + 2, w.z, drop_c7);

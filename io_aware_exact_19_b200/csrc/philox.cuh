@@ -13,7 +13,7 @@
 // The four lanes of a warp that hold four consecutive rows (or keys) all need
 // the same blocks. Each of them computes a different one and the words are
 // exchanged with four shuffles, so a lane pays one generator block per 16 of
-// its elements.
+// its elements. The round keys come from the host (round_keys).
 #pragma once
 
 #include <cstdint>
@@ -21,18 +21,32 @@
 namespace fa {
 namespace philox {
 
-__device__ __forceinline__ uint4 philox4x32_10(uint32_t c0, uint32_t c1, uint32_t c2, uint32_t c3, uint32_t k0,
-                                               uint32_t k1) {
+// The key words of the ten rounds: round r uses (seed low + r * 0x9E3779B9,
+// seed high + r * 0xBB67AE85) mod 2^32. They are computed once on the host and
+// read from the kernel parameters, so the rounds spend no instructions on them.
+struct Keys {
+  uint32_t k[20];  // k[2r], k[2r + 1]: round r
+};
+
+__host__ __device__ inline Keys round_keys(uint64_t seed) {
+  Keys r;
+  uint32_t k0 = static_cast<uint32_t>(seed), k1 = static_cast<uint32_t>(seed >> 32);
+  for (int i = 0; i < 10; ++i) {
+    r.k[2 * i] = k0;
+    r.k[2 * i + 1] = k1;
+    k0 += 0x9E3779B9u;
+    k1 += 0xBB67AE85u;
+  }
+  return r;
+}
+
+__device__ __forceinline__ uint4 philox4x32_10(uint32_t c0, uint32_t c1, uint32_t c2, uint32_t c3, const Keys& key) {
 #pragma unroll
   for (int r = 0; r < 10; ++r) {
-    if (r > 0) {
-      k0 += 0x9E3779B9u;
-      k1 += 0xBB67AE85u;
-    }
     const uint32_t hi0 = __umulhi(0xD2511F53u, c0), lo0 = 0xD2511F53u * c0;
     const uint32_t hi1 = __umulhi(0xCD9E8D57u, c2), lo1 = 0xCD9E8D57u * c2;
-    const uint32_t n0 = hi1 ^ c1 ^ k0;
-    const uint32_t n2 = hi0 ^ c3 ^ k1;
+    const uint32_t n0 = hi1 ^ c1 ^ key.k[2 * r];
+    const uint32_t n2 = hi0 ^ c3 ^ key.k[2 * r + 1];
     c0 = n0;
     c1 = lo1;
     c2 = n2;
@@ -41,58 +55,53 @@ __device__ __forceinline__ uint4 philox4x32_10(uint32_t c0, uint32_t c1, uint32_
   return make_uint4(c0, c1, c2, c3);
 }
 
-__device__ __forceinline__ uint32_t pick4(const uint4& v, uint32_t k) {
-  const uint32_t a = (k & 1u) ? v.y : v.x;
-  const uint32_t b = (k & 1u) ? v.w : v.z;
-  return (k & 2u) ? b : a;
-}
-
-__device__ __forceinline__ void place4(uint4& v, uint32_t k, uint32_t x) {
-  v.x = k == 0 ? x : v.x;
-  v.y = k == 1 ? x : v.y;
-  v.z = k == 2 ? x : v.z;
-  v.w = k == 3 ? x : v.w;
-}
-
-// Four rounds of exchange inside each group of four lanes: lane a holds `mine`,
-// four words meant for lanes 0..3 of its group (word r for lane r); afterwards
-// word s of the result is what lane s of the group held for this lane.
+// A 4 x 4 transpose across each group of four lanes: lane a holds `mine`, four
+// words meant for lanes 0..3 of its group (word r for lane r); afterwards word s
+// of the result is what lane s of the group held for this lane. Two butterfly
+// rounds: lanes a and a^1 swap the 2 x 2 blocks' off-diagonal words, then lanes
+// a and a^2 swap the off-diagonal 2 x 2 blocks.
 __device__ __forceinline__ uint4 exchange4(const uint4& mine) {
-  const uint32_t lane = threadIdx.x & 31u;
-  const uint32_t a = lane & 3u;
-  uint4 out = make_uint4(0, 0, 0, 0);
-#pragma unroll
-  for (uint32_t k = 0; k < 4; ++k) {
-    // Round k: lane a sends its word for lane (a + k) & 3 and receives from lane (a - k) & 3.
-    const uint32_t send = pick4(mine, (a + k) & 3u);
-    const uint32_t src = (a - k) & 3u;
-    const uint32_t got = __shfl_sync(0xffffffffu, send, static_cast<int>((lane & ~3u) | src));
-    place4(out, src, got);
-  }
-  return out;
+  const bool b0 = (threadIdx.x & 1u) != 0;
+  const bool b1 = (threadIdx.x & 2u) != 0;
+  uint32_t w0 = mine.x, w1 = mine.y, w2 = mine.z, w3 = mine.w;
+  // Round 1: send word (b0 ^ 1) of each column pair; the partner's arrives in its place.
+  uint32_t r0 = __shfl_xor_sync(0xffffffffu, b0 ? w0 : w1, 1);
+  uint32_t r1 = __shfl_xor_sync(0xffffffffu, b0 ? w2 : w3, 1);
+  w0 = b0 ? r0 : w0;
+  w1 = b0 ? w1 : r0;
+  w2 = b0 ? r1 : w2;
+  w3 = b0 ? w3 : r1;
+  // Round 2: send the column pair (b1 ^ 1); the partner's arrives in its place.
+  r0 = __shfl_xor_sync(0xffffffffu, b1 ? w0 : w2, 2);
+  r1 = __shfl_xor_sync(0xffffffffu, b1 ? w1 : w3, 2);
+  w0 = b1 ? r0 : w0;
+  w1 = b1 ? r1 : w1;
+  w2 = b1 ? w2 : r0;
+  w3 = b1 ? w3 : r1;
+  return make_uint4(w0, w1, w2, w3);
 }
 
 // Row-major use (forward, query-stationary backward): this lane holds query row
 // `row`; the four lanes of its group hold rows 4*(row>>2) .. +3. Returns the
 // draws of 16 columns, column groups cg0 .. cg0+3 (4 columns each): word k,
 // byte b = draw of column 4*(cg0+k)+b in this row.
-__device__ __forceinline__ uint4 draws_row(uint32_t cg0, uint32_t row, uint32_t bh, uint32_t k0, uint32_t k1) {
+__device__ __forceinline__ uint4 draws_row(uint32_t cg0, uint32_t row, uint32_t bh, const Keys& key) {
   const uint32_t a = threadIdx.x & 3u;
   // This lane's block: column group cg0 + a, its word r belongs to row 4*(row>>2) + r.
-  const uint4 blk = philox4x32_10(cg0 + a, row >> 2, bh, 0u, k0, k1);
+  const uint4 blk = philox4x32_10(cg0 + a, row >> 2, bh, 0u, key);
   return exchange4(blk);
 }
 
-// Column-major use (key-stationary backward): this lane holds key `key`; the
-// four lanes of its group hold keys 4*(key>>2) .. +3. Returns the draws of 16
+// Column-major use (key-stationary backward): this lane holds key `col`; the
+// four lanes of its group hold keys 4*(col>>2) .. +3. Returns the draws of 16
 // query rows, row groups rg0 .. rg0+3: word k, byte b = draw of element
 // (query row 4*(rg0+k)+b, this key).
-__device__ __forceinline__ uint4 draws_col(uint32_t rg0, uint32_t key, uint32_t bh, uint32_t k0, uint32_t k1) {
+__device__ __forceinline__ uint4 draws_col(uint32_t rg0, uint32_t col, uint32_t bh, const Keys& key) {
   const uint32_t a = threadIdx.x & 3u;
   // This lane's block: row group rg0 + a; its word w is query row 4*(rg0+a) + w,
-  // byte c of that word is key 4*(key>>2) + c. Lane c of the group needs byte c
+  // byte c of that word is key 4*(col>>2) + c. Lane c of the group needs byte c
   // of each word: transpose the 4 x 4 bytes so word c gathers them.
-  const uint4 blk = philox4x32_10(key >> 2, rg0 + a, bh, 0u, k0, k1);
+  const uint4 blk = philox4x32_10(col >> 2, rg0 + a, bh, 0u, key);
   const uint32_t t01lo = __byte_perm(blk.x, blk.y, 0x5140), t01hi = __byte_perm(blk.x, blk.y, 0x7362);
   const uint32_t t23lo = __byte_perm(blk.z, blk.w, 0x5140), t23hi = __byte_perm(blk.z, blk.w, 0x7362);
   uint4 tr;
