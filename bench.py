@@ -563,6 +563,77 @@ def time_fp8(dev, peaks, steps=50):
             "device_status": int(fa.fa_device_status()), "steps": steps}
 
 
+def _time_pair(fwd, bwd, flush, steps, stream):
+    """Mean device milliseconds of fwd and bwd (bwd may be None), L2 flushed before each step."""
+    import torch
+
+    for _ in range(3):
+        fwd()
+        if bwd is not None:
+            bwd()
+    torch.cuda.synchronize()
+    tf = tb = 0.0
+    for i in range(steps):
+        flush.fill_(i & 0xFF)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        ev[0].record(stream)
+        fwd()
+        ev[1].record(stream)
+        if bwd is not None:
+            bwd()
+        ev[2].record(stream)
+        torch.cuda.synchronize()
+        tf += ev[0].elapsed_time(ev[1])
+        tb += ev[1].elapsed_time(ev[2])
+    return tf / steps, (tb / steps if bwd is not None else None)
+
+
+def time_head_dims(dev, peaks, steps=30):
+    """The long-context causal shape (B=4 H=16 N=4096, bf16) at head dimensions 32,
+    96 and 256 (forward only: the backward supports d <= 128), and a chunked-prefill
+    shape with N_q != N_k (1024 queries against 8192 keys, bottom-right causal,
+    d = 128) through fa_fwd_qk / fa_bwd_qk. TFLOP/s count the allowed (query, key)
+    pairs: 4 d per pair forward, 2.5 times that backward. L2 flushed between steps."""
+    import torch
+
+    import fa_synth
+    import io_aware_exact_19_b200 as fa
+
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+    out = {}
+    cases = [("d32", 4, 16, 4096, 4096, 32), ("d96", 4, 16, 4096, 4096, 96), ("d256", 4, 16, 4096, 4096, 256),
+             ("nq1024_nk8192_d128", 4, 16, 1024, 8192, 128)]
+    for label, B, H, Nq, Nk, d in cases:
+        bq = fa_synth.attention_input_bits(B, H, Nq, d, "bf16", seed=41, names=("q", "do"))
+        bk = fa_synth.attention_input_bits(B, H, Nk, d, "bf16", seed=42, names=("k", "v"))
+        t = lambda b: torch.from_numpy(b.view("int16")).view(torch.bfloat16).to(dev)
+        q, do, k, v = t(bq["q"]), t(bq["do"]), t(bk["k"]), t(bk["v"])
+        o = torch.empty_like(q)
+        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=dev)
+        fwd = lambda: fa.fa_fwd_qk(q, k, v, o, lse, causal=True)
+        bwd = None
+        if d <= 128:
+            dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+            ws = torch.empty(fa.fa_bwd_workspace_size(B, H, Nq, d), dtype=torch.uint8, device=dev)
+            bwd = lambda: fa.fa_bwd_qk(q, k, v, o, lse, do, dq, dk, dv, ws, causal=True)
+        fms, bms = _time_pair(fwd, bwd, flush, steps, stream)
+        pairs = Nq * (Nk - Nq) + Nq * (Nq + 1) / 2
+        f_fwd = 4.0 * d * pairs * B * H
+        rec = {"B": B, "H": H, "N_q": Nq, "N_k": Nk, "d": d, "causal": True, "fwd_ms": fms,
+               "fwd_tflops": f_fwd / (fms * 1e-3) / 1e12,
+               "fwd_frac_of_measured_peak": f_fwd / (fms * 1e-3) / 1e12 / peaks["bf16"]}
+        if bms is not None:
+            rec.update({"bwd_ms": bms, "bwd_tflops": 2.5 * f_fwd / (bms * 1e-3) / 1e12,
+                        "bwd_frac_of_measured_peak": 2.5 * f_fwd / (bms * 1e-3) / 1e12 / peaks["bf16"]})
+        out[label] = rec
+        del q, k, v, do, o
+        torch.cuda.empty_cache()
+    out["device_status"] = int(fa.fa_device_status())
+    out["l2"] = "L2 flushed between steps"
+    return out
+
+
 def run_gpu(args, w, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -670,6 +741,8 @@ def run_gpu(args, w, rank, world, local_rank):
         torch.cuda.empty_cache()
         per_workload["long_causal_d128_fp8_fwd"] = time_fp8(dev, peaks)
         torch.cuda.empty_cache()
+        per_workload["head_dims_and_unequal_lengths"] = time_head_dims(dev, peaks)
+        torch.cuda.empty_cache()
 
     if rank != 0:
         return 0
@@ -731,7 +804,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-per-workload", action="store_true",
                     help="time only the selected workload (the default also times every other one)")
-    ap.add_argument("--extra", choices=("decode_splitkv_64k", "long_causal_d128_dropout", "long_causal_d128_fp8_fwd"),
+    ap.add_argument("--extra", choices=("decode_splitkv_64k", "long_causal_d128_dropout", "long_causal_d128_fp8_fwd",
+                                        "head_dims_and_unequal_lengths"),
                     help="run only this one of the extra measurements (1 GPU) and print its record")
     ap.add_argument("--reference-seconds", type=float, default=120.0,
                     help="approximate CPU time budget of the reference arm (warm-up plus timed steps)")
@@ -752,7 +826,7 @@ def main(argv=None):
         dev = torch.device("cuda", local_rank)
         torch.cuda.set_device(dev)
         fn = {"decode_splitkv_64k": time_decode, "long_causal_d128_dropout": time_dropout,
-              "long_causal_d128_fp8_fwd": time_fp8}[args.extra]
+              "long_causal_d128_fp8_fwd": time_fp8, "head_dims_and_unequal_lengths": time_head_dims}[args.extra]
         print(json.dumps({args.extra: fn(dev, load_peaks())}), flush=True)
         return 0
     if world > 1:
