@@ -88,8 +88,8 @@ struct Params {
 // is one 128-byte-swizzled chunk), V arrives as e4m3 in a staging ring and is
 // widened to 16 bits into the V ring. The V ring follows the K ring, so the
 // epilogue's staging (64 KB at d = 128, from the K ring on) stays inside both.
-// D = 256: one query tile per CTA (S 128 + O 256 TMEM columns) and single K and
-// V stages (64 KB tiles). kDeep (split-KV at D = 64, i.e. decoding, which streams
+// D = 256: one query tile per CTA (two S buffers of 128 + O 256 TMEM columns) and
+// single K and V stages (64 KB tiles). kDeep (split-KV at D = 64, i.e. decoding, which streams
 // K and V from HBM once): five stages, so more bytes are in flight per SM.
 template <int D, bool kF8 = false, bool kDeep = false>
 struct Smem {
@@ -103,9 +103,9 @@ struct Smem {
   static constexpr int kVOff = kKOff + kStages * kQKBytes;
   static constexpr int kV8Off = kVOff + kStages * kTileBytes;
   static constexpr int kBarOff = kV8Off + (kF8 ? kStages * kV8Bytes : 0);
-  // barriers: q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_full[2], o_full[2], drain
-  // and, for kF8, v8_full[S], v8_empty[S]
-  static constexpr int kNumBars = 1 + 4 * kStages + 7 + (kF8 ? 2 * kStages : 0);
+  // barriers: q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_full[2], o_full[2], drain,
+  // for kF8 v8_full[S], v8_empty[S], and last pv_done (D = 256: P V of a key tile completed)
+  static constexpr int kNumBars = 1 + 4 * kStages + 7 + (kF8 ? 2 * kStages : 0) + 1;
   static constexpr int kListOff = kBarOff + 8 * kNumBars + 16;  // + tmem slot, abort flag, list length
   static constexpr int kBytes = kListOff + 4 * kMaxSparseTiles;
   static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1024
@@ -187,6 +187,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t bar_drain = smem_u32(&bars[1 + 4 * S + 6]);
   auto bar_v8_full = [&](int s) { return smem_u32(&bars[1 + 4 * S + 7 + s]); };
   auto bar_v8_empty = [&](int s) { return smem_u32(&bars[1 + 4 * S + 7 + S + s]); };
+  const uint32_t bar_pv_done = smem_u32(&bars[L::kNumBars - 1]);
+  // D = 256 (one query tile per CTA): key tile n's S goes to TMEM columns
+  // 128 * (n % 2), so S of tile n + 1 is computed while the softmax warps work on
+  // tile n; otherwise query tile q's S is at columns 128 * q.
+  constexpr bool kTwoS = D == 256;
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
@@ -234,6 +239,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar_o_full(q), 1);
     }
     mbar_init(bar_drain, 1);
+    mbar_init(bar_pv_done, 1);
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -401,7 +407,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t dV = sdesc_sw128(smem_u32(sV), kChunkBytes, 1024);    // MN-major B of P V
       auto issue_s = [&](int q, int n) {
         const int s = n % S;
-        const uint32_t d_tmem = tmem + q * 128;
+        const int region = kTwoS ? (n & 1) : q;
+        const uint32_t d_tmem = tmem + region * 128;
         const uint64_t bq = sdesc_add(dQ, static_cast<uint32_t>(dual && !shift1 ? 0 : q) * L::kQKBytes);
         const uint64_t bk = sdesc_add(dK, static_cast<uint32_t>(s) * L::kQKBytes);
         if constexpr (kF8) {
@@ -418,12 +425,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             umma_ss(d_tmem, sdesc_add(bq, off), sdesc_add(bk, off), idesc_s, k > 0);
           }
         }
-        umma_commit(bar_s_full(q));
+        umma_commit(bar_s_full(region));
       };
       auto issue_pv = [&](int q, int n) {
         const int s = n % S;
         const uint32_t d_tmem = tmem + 256 + q * D;
-        const uint32_t a_tmem = tmem + q * 128;
+        const uint32_t a_tmem = tmem + (kTwoS ? (n & 1) : q) * 128;
         const uint64_t bv = sdesc_add(dV, static_cast<uint32_t>(s) * L::kTileBytes);
 #pragma unroll
         for (int k = 0; k < kBlockN / 16; ++k) {
@@ -452,7 +459,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           // A slot the next tile uses but this one does not gets its S first: its
           // S/P columns were last read by a P V issued in an earlier step, so its
           // softmax can run while this step waits for V and the other slot's P.
-          if (fn & ~f) {
+          if (kTwoS) {
+            // The other S buffer was last read by P V of tile n - 1, issued earlier.
+            tc_fence_after();
+            issue_s(0, n + 1);
+            umma_commit(bar_k_empty((n + 1) % S));
+          } else if (fn & ~f) {
             tc_fence_after();
             for (int q = 0; q < 2; ++q)
               if ((fn & ~f) & (1u << q)) issue_s(q, n + 1);
@@ -462,16 +474,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         for (int q = 0; q < 2; ++q) {
           if (f & (1u << q)) {
-            if (!(ok = mbar_wait(bar_p_full(q), p_count[q] & 1, ctx))) break;
-            ++p_count[q];
+            const int pr = kTwoS ? (n & 1) : q;
+            if (!(ok = mbar_wait(bar_p_full(pr), p_count[pr] & 1, ctx))) break;
+            ++p_count[pr];
             tc_fence_after();
             issue_pv(q, n);
-            if (fn & (1u << q)) issue_s(q, n + 1);
+            if (kTwoS) umma_commit(bar_pv_done);
+            else if (fn & (1u << q)) issue_s(q, n + 1);
           }
         }
         if (!ok) break;
         umma_commit(bar_v_empty(n % S));
-        if (has_next) umma_commit(bar_k_empty((n + 1) % S));
+        if (has_next && !kTwoS) umma_commit(bar_k_empty((n + 1) % S));
       }
       if (ok) {
         for (int q = 0; q < 2; ++q)
@@ -541,7 +555,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool warp_rows = warp_row0 + 31 >= 0 && warp_row0 < p.N;
     const bool tile_active = (q == 0) || q1_active;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-    const uint32_t t_s = tmem + lane_off + q * 128;
     const uint32_t t_o = tmem + lane_off + 256 + q * D;
     const float sl2 = p.scale_log2;
     const uint32_t drop_c7 = philox::keep_bias(p.drop_t);
@@ -574,11 +587,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        if (!(ok = mbar_wait_warp(bar_s_full(q), count & 1, ctx))) break;
+        const int region = kTwoS ? (count & 1) : q;
+        const uint32_t t_s = tmem + lane_off + region * 128;
+        const uint32_t s_parity = kTwoS ? ((count >> 1) & 1) : (count & 1);
+        if (!(ok = mbar_wait_warp(bar_s_full(region), s_parity, ctx))) break;
         tc_fence_after();
         if (!warp_rows) {
           tc_fence_before();
-          mbar_arrive(bar_p_full(q));
+          mbar_arrive(bar_p_full(region));
           ++count;
           continue;
         }
@@ -616,6 +632,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
           const bool need = mx > m_ref + kRescaleThreshold;
           if (__any_sync(0xffffffffu, need)) {
+            if (kTwoS) {
+              // P V of the previous tile may still be accumulating into O.
+              if (!(ok = mbar_wait_warp(bar_pv_done, (count - 1) & 1, ctx))) break;
+              tc_fence_after();
+            }
             const float alpha = need ? ex2(m_ref - mx) : 1.0f;
             if (need) {
               l_sum *= alpha;
@@ -668,7 +689,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_st32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(bar_p_full(q));
+        mbar_arrive(bar_p_full(region));
         ++count;
       }
 
