@@ -85,7 +85,7 @@ struct Cfg {
   static constexpr int k2V = k2K + kS2 * kTile;
   static constexpr int k2End = k2V + kS2 * kTile;
   static constexpr int kOffBar = ((k1End > k2End ? k1End : k2End) + 15) / 16 * 16;
-  static constexpr int kNumBars = 20;
+  static constexpr int kNumBars = 21;
   static constexpr int kOffMisc = kOffBar + 8 * kNumBars;  // tmem slot, abort flag, tile count
   static constexpr int kBytes = kOffMisc + 16;
   static constexpr int kAlloc = kBytes + 1024;
@@ -99,11 +99,12 @@ struct Cfg {
 // `drain` (both kinds) lets the MMA issuer wait for its own MMAs on the abort path.
 struct KeyBars {
   static constexpr int kv_full = 0, qdo_full = 1, qdo_empty = 4, s_full = 7, s_free = 8, dp_full = 9,
-                       p_full = 10, all_done = 11, drain = 19;
+                       p_full = 10, all_done = 11, dp_full1 = 12, drain = 19;
 };
 struct QueryBars {
   static constexpr int q_ready = 0, k_full = 1, k_empty = 4, v_full = 7, v_empty = 10, s_full = 13,
-                       s_free = 14, dp_full = 15, ds_full = 16, all_done = 17, qdo_in = 18, drain = 19;
+                       s_free = 14, dp_full = 15, ds_full = 16, all_done = 17, qdo_in = 18, drain = 19,
+                       dp_full1 = 20;
 };
 
 // Abort path of a producer: wait (bounded, whatever the abort flag says) for the
@@ -348,6 +349,12 @@ __device__ __forceinline__ void key_cta(const Ctx& c, const Params& p, const CUt
   float* sL = reinterpret_cast<float*>(c.smem + C::k1L);
   float* sDv = reinterpret_cast<float*>(c.smem + C::k1Dv);
   const int len = c.len;
+  // TMEM: S^T at columns 0-127, dP^T (then P^T and dS^T over it) at 128-255, dV and dK
+  // from 256. At d = 64 columns 384-511 are free and hold a second dP^T buffer: tile
+  // n uses buffer n % 2, so dP^T of tile n + 1 is computed before dV and dK of tile n.
+  constexpr bool kTwoDP = D == 64;
+  auto dp_col = [&](int n) -> uint32_t { return (kTwoDP && (n & 1)) ? 384u : 128u; };
+  auto dp_bar = [&](int n) { return (kTwoDP && (n & 1)) ? B::dp_full1 : B::dp_full; };
 
   if (c.warp < 4) {
     reg_dealloc<kRegsLow>();
@@ -409,14 +416,14 @@ __device__ __forceinline__ void key_cta(const Ctx& c, const Params& p, const CUt
         }
         umma_commit(c.bar(B::s_full));
       };
-      auto issue_dp = [&](int n) {  // dP^T_n (stage resident)
+      auto issue_dp = [&](int n) {  // dP^T_n (stage resident), into dP^T buffer n % 2 at d = 64
         const uint64_t bdo = sdesc_add(dDOk, static_cast<uint32_t>(n % S) * C::kTile);
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
           const uint32_t off = ((k * 16) / 64) * kChunk + ((k * 16) % 64) * 2;
-          umma_ss(t + 128, sdesc_add(dV, off), sdesc_add(bdo, off), idesc_sp, k > 0);
+          umma_ss(t + dp_col(n), sdesc_add(dV, off), sdesc_add(bdo, off), idesc_sp, k > 0);
         }
-        umma_commit(c.bar(B::dp_full));
+        umma_commit(c.bar(dp_bar(n)));
       };
       bool ok = mbar_wait(c.bar(B::kv_full), 0, c.wait) && mbar_wait(c.bar(B::qdo_full), 0, c.wait);
       const bool issued = ok;  // MMAs are issued from here on
@@ -433,6 +440,8 @@ __device__ __forceinline__ void key_cta(const Ctx& c, const Params& p, const CUt
           if (!(ok = mbar_wait(c.bar(B::qdo_full + (n + 1) % S), ((n + 1) / S) & 1, c.wait))) break;
           tc_fence_after();
           issue_s(n + 1);
+          // dP^T_{n+1} into the other buffer, last read by dV_{n-1} and dK_{n-1} (issued earlier).
+          if (kTwoDP) issue_dp(n + 1);
         }
         if (!(ok = mbar_wait(c.bar(B::p_full), n & 1, c.wait))) break;
         tc_fence_after();
@@ -442,16 +451,16 @@ __device__ __forceinline__ void key_cta(const Ctx& c, const Params& p, const CUt
 #pragma unroll
         for (int k = 0; k < kBR / 16; ++k) {
           // P^T columns of query rows 16k..16k+15: warpgroup h = k/4 wrote them at 128 + 64h.
-          umma_ts(t + 256, t + 128 + 64 * (k / 4) + 8 * (k % 4), sdesc_add(bdo, k * 16 * 128), idesc_kv,
+          umma_ts(t + 256, t + dp_col(n) + 64 * (k / 4) + 8 * (k % 4), sdesc_add(bdo, k * 16 * 128), idesc_kv,
                   acc | static_cast<uint32_t>(k > 0));
         }
 #pragma unroll
         for (int k = 0; k < kBR / 16; ++k) {
-          umma_ts(t + 256 + D, t + 128 + 64 * (k / 4) + 32 + 8 * (k % 4), sdesc_add(bq, k * 16 * 128), idesc_kv,
+          umma_ts(t + 256 + D, t + dp_col(n) + 64 * (k / 4) + 32 + 8 * (k % 4), sdesc_add(bq, k * 16 * 128), idesc_kv,
                   acc | static_cast<uint32_t>(k > 0));
         }
         umma_commit(c.bar(B::qdo_empty + s));
-        if (n + 1 < len) issue_dp(n + 1);  // dP^T columns: ordered after dV, dK read P^T, dS^T
+        if (!kTwoDP && n + 1 < len) issue_dp(n + 1);  // dP^T columns: ordered after dV, dK read P^T, dS^T
       }
       if (ok) {
         umma_commit(c.bar(B::all_done));
@@ -526,11 +535,11 @@ __device__ __forceinline__ void key_cta(const Ctx& c, const Params& p, const CUt
         for (int x = 0; x < 64; ++x)
           if (x < lim) pv[x] = 0.0f;
       }
-      if (!(ok = mbar_wait_warp(c.bar(B::dp_full), n & 1, c.wait))) break;
+      if (!(ok = mbar_wait_warp(c.bar(dp_bar(n)), kTwoDP ? ((n >> 1) & 1) : (n & 1), c.wait))) break;
       tc_fence_after();
       uint32_t dr[64];
-      tmem_ld32(tl + 128 + qo, *reinterpret_cast<uint32_t(*)[32]>(&dr[0]));
-      tmem_ld32(tl + 128 + qo + 32, *reinterpret_cast<uint32_t(*)[32]>(&dr[32]));
+      tmem_ld32(tl + dp_col(n) + qo, *reinterpret_cast<uint32_t(*)[32]>(&dr[0]));
+      tmem_ld32(tl + dp_col(n) + qo + 32, *reinterpret_cast<uint32_t(*)[32]>(&dr[32]));
       tmem_ld_wait();
       const uint32_t aD = smem_u32(sDv + s * kBR + qo);
       uint32_t pk[32], dk[32];
@@ -567,8 +576,8 @@ __device__ __forceinline__ void key_cta(const Ctx& c, const Params& p, const CUt
                                       pv[x + 3] * (__uint_as_float(dr[x + 3]) - d4.w));
         }
       }
-      tmem_st32(tl + 128 + qo, pk);
-      tmem_st32(tl + 128 + qo + 32, dk);
+      tmem_st32(tl + dp_col(n) + qo, pk);
+      tmem_st32(tl + dp_col(n) + qo + 32, dk);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(c.bar(B::p_full));
@@ -608,6 +617,11 @@ __device__ __forceinline__ void query_cta(const Ctx& c, const Params& p, const C
   // TMA: per-thread row loads from global memory would touch 32 rows per warp
   // instruction. At d = 64 the rows are read directly (measured faster there).
   constexpr bool kStageQdo = D == 128;
+  // At d = 64 TMEM columns 384-511 are free and hold a second dP buffer: tile n uses
+  // buffer n % 2, so dP of tile n + 1 is computed before dQ of tile n.
+  constexpr bool kTwoDP = D == 64;
+  auto dp_col = [&](int n) -> uint32_t { return (kTwoDP && (n & 1)) ? 384u : static_cast<uint32_t>(C::kColDP2); };
+  auto dp_bar = [&](int n) { return (kTwoDP && (n & 1)) ? B::dp_full1 : B::dp_full; };
 
   if (c.warp < 4) {
     reg_dealloc<kRegsLow>();
@@ -682,9 +696,9 @@ __device__ __forceinline__ void query_cta(const Ctx& c, const Params& p, const C
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
           const uint32_t off = ((k * 16) / 64) * kChunk + ((k * 16) % 64) * 2;
-          umma_ts(t + C::kColDP2, t + C::kColDO + 8 * k, sdesc_add(bv, off), idesc_sp, k > 0);
+          umma_ts(t + dp_col(n), t + C::kColDO + 8 * k, sdesc_add(bv, off), idesc_sp, k > 0);
         }
-        umma_commit(c.bar(B::dp_full));
+        umma_commit(c.bar(dp_bar(n)));
         umma_commit(c.bar(B::v_empty + s));
         return true;
       };
@@ -700,6 +714,8 @@ __device__ __forceinline__ void query_cta(const Ctx& c, const Params& p, const C
           // S_{n+1} overwrites S_n once the elementwise warps hold it in registers.
           if (!(ok = mbar_wait(c.bar(B::s_free), n & 1, c.wait))) break;
           if (!(ok = issue_s(n + 1))) break;
+          // dP_{n+1} into the other buffer, last read by dQ_{n-1} (issued earlier).
+          if (kTwoDP && !(ok = issue_dp(n + 1))) break;
         }
         if (!(ok = mbar_wait(c.bar(B::ds_full), n & 1, c.wait))) break;  // dS_n written over dP_n
         tc_fence_after();
@@ -707,11 +723,11 @@ __device__ __forceinline__ void query_cta(const Ctx& c, const Params& p, const C
 #pragma unroll
         for (int k = 0; k < kBlockN / 16; ++k) {
           // dS columns of keys 16k..16k+15: warpgroup h = k/4 wrote them at dP + 64h.
-          umma_ts(t + C::kColDQ, t + C::kColDP2 + 64 * (k / 4) + 8 * (k % 4), sdesc_add(bk, k * 16 * 128),
+          umma_ts(t + C::kColDQ, t + dp_col(n) + 64 * (k / 4) + 8 * (k % 4), sdesc_add(bk, k * 16 * 128),
                   idesc_q, (n > 0 || k > 0) ? 1u : 0u);
         }
         umma_commit(c.bar(B::k_empty + s));               // K_n free once dQ_n is done
-        if (n + 1 < len && !(ok = issue_dp(n + 1))) break;  // dP columns: ordered after dQ_n read dS_n
+        if (!kTwoDP && n + 1 < len && !(ok = issue_dp(n + 1))) break;  // dP columns: after dQ_n read dS_n
       }
       if (ok) {
         umma_commit(c.bar(B::all_done));
@@ -823,11 +839,11 @@ __device__ __forceinline__ void query_cta(const Ctx& c, const Params& p, const C
         for (int x = 0; x < 64; ++x)
           if (x > lim) pv[x] = 0.0f;
       }
-      if (!(ok = mbar_wait_warp(c.bar(B::dp_full), n & 1, c.wait))) break;  // dP_n
+      if (!(ok = mbar_wait_warp(c.bar(dp_bar(n)), kTwoDP ? ((n >> 1) & 1) : (n & 1), c.wait))) break;  // dP_n
       tc_fence_after();
       uint32_t dr[64];
-      tmem_ld32(tl + C::kColDP2 + 64 * h, *reinterpret_cast<uint32_t(*)[32]>(&dr[0]));
-      tmem_ld32(tl + C::kColDP2 + 64 * h + 32, *reinterpret_cast<uint32_t(*)[32]>(&dr[32]));
+      tmem_ld32(tl + dp_col(n) + 64 * h, *reinterpret_cast<uint32_t(*)[32]>(&dr[0]));
+      tmem_ld32(tl + dp_col(n) + 64 * h + 32, *reinterpret_cast<uint32_t(*)[32]>(&dr[32]));
       tmem_ld_wait();
       uint32_t dk[32];
       if constexpr (kDropout) {
@@ -851,7 +867,7 @@ __device__ __forceinline__ void query_cta(const Ctx& c, const Params& p, const C
           dk[x] = pack2<BF16>(pv[2 * x] * (__uint_as_float(dr[2 * x]) - dd),
                               pv[2 * x + 1] * (__uint_as_float(dr[2 * x + 1]) - dd));
       }
-      tmem_st32(tl + C::kColDP2 + 64 * h, dk);
+      tmem_st32(tl + dp_col(n) + 64 * h, dk);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(c.bar(B::ds_full));
@@ -929,6 +945,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(c.bar(B::s_free), 256);
       mbar_init(c.bar(B::dp_full), 1);
       mbar_init(c.bar(B::p_full), 256);
+      mbar_init(c.bar(B::dp_full1), 1);
       mbar_init(c.bar(B::all_done), 1);
       mbar_init(c.bar(B::drain), 1);
     } else {
@@ -944,6 +961,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(c.bar(B::s_free), 256);
       mbar_init(c.bar(B::dp_full), 1);
       mbar_init(c.bar(B::ds_full), 256);
+      mbar_init(c.bar(B::dp_full1), 1);
       mbar_init(c.bar(B::all_done), 1);
       mbar_init(c.bar(B::qdo_in), 1);
       mbar_init(c.bar(B::drain), 1);
