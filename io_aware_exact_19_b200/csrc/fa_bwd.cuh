@@ -29,7 +29,10 @@
 // (or S) into registers, so the MMA for the next tile's S^T (S) overlaps their
 // work on the current tile; dP^T (dP) shares its TMEM columns with the P^T and
 // dS^T (dS) written back from it, so the next dP^T waits for the dV/dK (dQ)
-// MMAs that read them, which run in issue order.
+// MMAs that read them, which run in issue order. At d = 64 the TMEM columns
+// 384-511 are free in both kinds and hold a second dP^T (dP) buffer: tile n
+// uses buffer n % 2, so the next tile's dP^T (dP) runs before this tile's
+// dV/dK (dQ).
 //
 // Roles (384 threads, one CTA per SM, both kinds):
 //   warp 0      TMA producer          warp 1      MMA issuer, TMEM owner
@@ -40,9 +43,10 @@
 // TMEM (512 columns):
 //   key-stationary:   S^T at 0; dP^T at 128, where warpgroup h later writes its
 //                     P^T (32 columns) at 128+64h and dS^T at 128+64h+32;
-//                     dV at 256, dK at 256+d.
+//                     dV at 256, dK at 256+d; at d = 64 odd tiles use 384 for dP^T.
 //   query-stationary: Q_i at 0 and dO_i at d/2 (bf16 pairs), S at d, dP at
-//                     d+128 (warpgroup h writes its dS at d+128+64h), dQ at d+256.
+//                     d+128 (warpgroup h writes its dS at d+128+64h), dQ at d+256;
+//                     at d = 64 odd tiles use 384 for dP.
 #pragma once
 
 #include <cuda_fp16.h>
