@@ -192,6 +192,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   // 128 * (n % 2), so S of tile n + 1 is computed while the softmax warps work on
   // tile n; otherwise query tile q's S is at columns 128 * q.
   constexpr bool kTwoS = D == 256;
+  // D = 256 (single-stage K and V rings): warp 3 loads V, so the load of the next
+  // K tile never waits in one thread's program order behind a V slot that the
+  // current P V still reads. At smaller D (deeper rings) one producer is faster.
+  constexpr bool kSplitV = D == 256 && !kF8;
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
@@ -366,14 +370,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!mbar_wait(bar_v8_empty(s), ph, ctx)) break;
           mbar_arrive_expect_tx(bar_v8_full(s), L::kV8Bytes);
           tma_load_3d(smem_u32(smem + L::kV8Off + s * L::kV8Bytes), &tmap_v, bar_v8_full(s), 0, j * kBlockN, bh);
-        } else {
+          ++v_issued;
+        } else if (!kSplitV) {
           if (!mbar_wait(bar_v_empty(s), ph, ctx)) break;
           mbar_arrive_expect_tx(bar_v_full(s), L::kTileBytes);
           for (int c = 0; c < D / 64; ++c)
             tma_load_3d(smem_u32(sV + s * L::kTileBytes + c * kChunkBytes), &tmap_v, bar_v_full(s), c * 64,
                         j * kBlockN, bh);
+          ++v_issued;
         }
-        ++v_issued;
       }
       if (*abort_flag) {
         // Aborting: wait (bounded, whatever the flag says) for every load this
@@ -390,6 +395,31 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         mbar_wait_bounded(bar_q_full, 0, p.timeout_ns);
+      }
+    }
+  } else if (kSplitV && warp == 3) {
+    // ------------------------------------------------------------ V producer (D = 256)
+    if (lane == 0 && tl.len > 0 && !p.withhold) {
+      prefetch_tmap(&tmap_v);
+      int v_issued = 0;
+      for (int n = 0; n < tl.len; ++n) {
+        const int j = static_cast<int>(tl.entry(n) & 0xFFFFu);
+        const int s = n % S;
+        if (!mbar_wait(bar_v_empty(s), ((n / S) & 1) ^ 1, ctx)) break;
+        mbar_arrive_expect_tx(bar_v_full(s), L::kTileBytes);
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_3d(smem_u32(sV + s * L::kTileBytes + c * kChunkBytes), &tmap_v, bar_v_full(s), c * 64,
+                      j * kBlockN, bh);
+        ++v_issued;
+      }
+      if (*abort_flag) {
+        // Aborting: wait (bounded) for the last load into each stage.
+        for (int s = 0; s < S; ++s) {
+          if (v_issued > s) {
+            const int last = v_issued - 1 - ((v_issued - 1 - s) % S);
+            mbar_wait_bounded(bar_v_full(s), (last / S) & 1, p.timeout_ns);
+          }
+        }
       }
     }
   } else if (warp == 1) {
