@@ -179,12 +179,14 @@ def test_device_timeout_is_reported_and_cleared():
     assert fa.fa_device_status() == fa.FA_OK
 
 
-def test_forward_kernel_abort_path_reports_timeout_and_context_survives():
-    # The production forward kernel with a producer that issues no load: the MMA
-    # issuer's wait for Q runs out (20 ms), every role leaves its loop and the CTAs
-    # exit with nothing in flight. The status word reports the time-out and the
-    # next, normal launch is still correct.
-    c = Case(2, 3, 1000, 128, "bf16", seed=17)
+@pytest.mark.parametrize("d", [64, 128, 256])
+def test_forward_kernel_abort_path_reports_timeout_and_context_survives(d):
+    # The production forward kernel with producers that issue no load (at d = 256
+    # both the Q/K and the V producer warp): the MMA issuer's wait for Q runs out
+    # (20 ms), every role leaves its loop and the CTAs exit with nothing in flight.
+    # The status word reports the time-out and the next, normal launch is still
+    # correct.
+    c = Case(2, 3, 1000, d, "bf16", seed=17)
     assert fa.fa_device_status() == fa.FA_OK
     o = torch.zeros_like(c.dev["q"])
     lse = torch.zeros((2, 3, 1000), dtype=torch.float32, device="cuda")
