@@ -180,7 +180,9 @@ fa_status fa_bwd_qk(fa_dtype dtype, const void* q, const void* k, const void* v,
  *             completes) it holds the partials: O_s as fp32
  *             [n_splits][B*H][Nq][d] at offset 0, then lse_s as fp32
  *             [n_splits][B*H][Nq] at the next 256-byte boundary after O_s.
- * Two launches on `stream`; asynchronous, allocates nothing.
+ * Two launches on `stream`; asynchronous, allocates nothing. With Nq <= 4
+ * (decoding) step 1 runs on the CUDA cores, which read each range's K and V
+ * once; larger Nq use the tensor-core forward. The partials are the same.
  */
 size_t fa_fwd_splitkv_workspace_size(int B, int H, int Nq, int d, int n_splits);
 int fa_fwd_splitkv_splits(int B, int H, int Nq, int Nk);

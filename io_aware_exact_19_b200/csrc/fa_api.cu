@@ -333,6 +333,11 @@ int fa_fwd_splitkv_splits(int B, int H, int Nq, int Nk) {
   const long long tk = (static_cast<long long>(Nk) + 127) / 128;
   long long ns = base >= sms ? 1 : sms / base;  // one wave of CTAs
   if (tq == 1) ns *= 2;  // one query tile: a CTA takes two consecutive ranges
+  if (Nq <= fa::kDecodeMaxRows) {
+    // CUDA-core decoding: one range per CTA, two CTAs per SM, one wave.
+    const long long heads = static_cast<long long>(B) * H;
+    ns = heads >= 2LL * sms ? 1 : (2LL * sms) / heads;
+  }
   if (ns > tk) ns = tk;
   return static_cast<int>(ns < 1 ? 1 : ns);
 }
@@ -376,7 +381,10 @@ fa_status fa_fwd_splitkv(fa_dtype dtype, const void* q, const void* k, const voi
   a.lse_part = reinterpret_cast<float*>(base + ws.lse_part);
   a.status = status_word();
   if (!a.status) return FA_ERR_CUDA;
-  if (fa::launch_fwd(a, stream) != 0) return FA_ERR_CUDA;
+  // A few query rows (decoding): the ranges' partials on the CUDA cores, which
+  // stream K and V once; otherwise the tensor-core forward's split-KV instance.
+  const int st = Nq <= fa::kDecodeMaxRows ? fa::launch_decode_splitkv(a, stream) : fa::launch_fwd(a, stream);
+  if (st != 0) return FA_ERR_CUDA;
   return fa::launch_splitkv_merge(a, stream) == 0 ? FA_OK : FA_ERR_CUDA;
 }
 

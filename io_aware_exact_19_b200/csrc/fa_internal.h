@@ -48,6 +48,9 @@ int launch_fwd(const AttnArgs& a, cudaStream_t stream);
 int launch_fwd_fp8(const AttnArgs& a, cudaStream_t stream);
 // Merge of the split-KV partials (a.o_part, a.lse_part, a.n_splits) into a.o, a.lse.
 int launch_splitkv_merge(const AttnArgs& a, cudaStream_t stream);
+// Split-KV step 1 on the CUDA cores for at most kDecodeMaxRows query rows (fa_decode.cu).
+constexpr int kDecodeMaxRows = 4;
+int launch_decode_splitkv(const AttnArgs& a, cudaStream_t stream);
 
 // Debug: the dropout draws of every (head, query row, key), through the
 // row-major and the column-major generator paths of the attention kernels.

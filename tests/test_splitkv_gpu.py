@@ -4,9 +4,10 @@ The keys are cut into n_splits ranges of whole 128-key tiles; each range's
 partial (O_s, lse_s) is checked against ``oracle.split_kv_forward`` on the same
 ranges, and the merged (O, lse) against ``oracle.forward``. Tolerances as for
 the forward: O max-abs <= 1e-2 (partials too, in fp32), lse max-abs <= 1e-3.
-Decoding shapes (one or a few query rows against up to 64K keys), ragged sizes,
-head dimensions 64/96/128, causal (bottom-right) and block-sparse masks, and
-ranges in which a row has no allowed key (lse_s = -inf, O_s = 0)."""
+Decoding shapes (one or a few query rows against up to 64K keys; at most 4 rows
+run on the CUDA-core kernel), ragged sizes, head dimensions 32/64/96/128/256,
+causal (bottom-right) and block-sparse masks, and ranges in which a row has no
+allowed key (lse_s = -inf, O_s = 0)."""
 import numpy as np
 import pytest
 import torch
@@ -69,6 +70,11 @@ def _run(B, H, Nq, Nk, d, fmt, causal, n_splits=None, mask=None, seed=0):
     (1, 2, 3, 2000, 256, "bf16", True, 6),       # head dimension 256 (forward only)
     (2, 3, 7, 5000, 64, "fp16", True, 9),         # one query tile, odd range count: a CTA with one range
     (1, 2, 100, 1000, 128, "bf16", True, 8),      # causal: ranges past a row's reach are empty
+    # at most 4 query rows: the CUDA-core decoding kernel
+    (1, 16, 1, 65536, 64, "fp16", False, None),   # the decoding benchmark's shape
+    (2, 2, 2, 3000, 96, "fp16", True, 5),         # padded head dimension, causal shift per row
+    (1, 3, 4, 1029, 32, "bf16", True, 9),         # ragged last tile, d = 32
+    (1, 1, 4, 4, 128, "bf16", True, 1),           # rows 0-2 see 1-3 keys
 ])
 def test_splitkv_matches_oracle(B, H, Nq, Nk, d, fmt, causal, n_splits):
     _run(B, H, Nq, Nk, d, fmt, causal, n_splits)
@@ -94,9 +100,12 @@ def test_splitkv_agrees_with_unsplit_forward():
 
 
 def test_suggested_splits_fill_the_gpu():
-    # One query tile: a CTA takes two consecutive ranges, so B*H*ceil(n/2) CTAs.
     sms = torch.cuda.get_device_properties(0).multi_processor_count
+    # At most 4 query rows (CUDA-core decoding): one range per CTA, two CTAs per SM.
     ns = fa.fa_fwd_splitkv_splits(1, 16, 1, 65536)
+    assert 2 <= ns <= 512 and 16 * ns <= 2 * sms < 16 * (ns + 1)
+    # One query tile of more rows: a CTA takes two consecutive ranges, B*H*ceil(n/2) CTAs.
+    ns = fa.fa_fwd_splitkv_splits(1, 16, 64, 65536)
     ctas = 16 * ((ns + 1) // 2)
     assert 2 <= ns <= 512 and ctas <= sms and ctas + 16 > sms
     assert fa.fa_fwd_splitkv_splits(8, 64, 4096, 4096) == 1
