@@ -64,14 +64,14 @@ __device__ __forceinline__ uint4 exchange4(const uint4& mine) {
   const bool b0 = (threadIdx.x & 1u) != 0;
   const bool b1 = (threadIdx.x & 2u) != 0;
   uint32_t w0 = mine.x, w1 = mine.y, w2 = mine.z, w3 = mine.w;
-  // Round 1: send word (b0 ^ 1) of each column pair; the partner's arrives in its place.
+  // First butterfly step: send word (b0 ^ 1) of each column pair; the partner's arrives in its place.
   uint32_t r0 = __shfl_xor_sync(0xffffffffu, b0 ? w0 : w1, 1);
   uint32_t r1 = __shfl_xor_sync(0xffffffffu, b0 ? w2 : w3, 1);
   w0 = b0 ? r0 : w0;
   w1 = b0 ? w1 : r0;
   w2 = b0 ? r1 : w2;
   w3 = b0 ? w3 : r1;
-  // Round 2: send the column pair (b1 ^ 1); the partner's arrives in its place.
+  // Second butterfly step: send the column pair (b1 ^ 1); the partner's arrives in its place.
   r0 = __shfl_xor_sync(0xffffffffu, b1 ? w0 : w2, 2);
   r1 = __shfl_xor_sync(0xffffffffu, b1 ? w1 : w3, 2);
   w0 = b1 ? r0 : w0;
