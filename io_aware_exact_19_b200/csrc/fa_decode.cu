@@ -24,6 +24,7 @@
 #include <cstdint>
 
 #include "fa_internal.h"
+#include "tma_host.h"
 
 namespace fa {
 namespace {
@@ -209,11 +210,8 @@ int launch_decode_q(const DecodeParams& p, cudaStream_t stream) {
   static_assert((2 * NQ * (kDecThreads / (D / 8)) + NQ * (kDecThreads / (D / 8)) * D + NQ) * 4 <= kDecSmem,
                 "merge arrays exceed the ring");
   auto kern = fa_decode_split_kernel<D, BF16, NQ>;
-  static bool attr = false;  // set once per instance (the attribute persists)
-  if (!attr) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmem) != cudaSuccess) return 1;
-    attr = true;
-  }
+  const cudaError_t e = host::ensure_dynamic_smem(reinterpret_cast<const void*>(kern), kDecSmem);
+  if (e != cudaSuccess) return static_cast<int>(e);
   dim3 grid(static_cast<unsigned>(p.n_splits), static_cast<unsigned>(p.BH));
   kern<<<grid, kDecThreads, kDecSmem, stream>>>(p);
   return static_cast<int>(cudaGetLastError());
